@@ -1,0 +1,325 @@
+/*
+ * fp64 CPU oracle for RecSA tree sparse attention — TEST INFRASTRUCTURE.
+ *
+ * Plain, slow and meant to be checked by eye against the method's pages:
+ * "Recursive Sparse Attention: Million-Token Length Extrapolation at
+ * Logarithmic Cost" (arXiv 2611.07232, abstract) and the kongchang.com
+ * article on RecSA ("Core Idea", "Position Encoding"). No blocking, no
+ * fusion, no reordering: every quantity is formed from its definition.
+ * Only the tests, the smoke check and the benchmark's CPU-baseline leg may
+ * call it. It shares no code with the CUDA path.
+ *
+ * What the pages fix:
+ *   - a tree over the KV cache; the bottom level is the exact tokens and each
+ *     node summarises its subtree with one key and one value (abstract;
+ *     "Core Idea");
+ *   - a node's value is the mean of all token values in its subtree
+ *     ("Core Idea", mean pooling paragraph);
+ *   - node keys come from one pooler per layer, shared by all levels
+ *     (abstract);
+ *   - each level above the tokens keeps at most k candidates; queries filter
+ *     at the top and drill down level by level (abstract; "Core Idea");
+ *   - summaries of unselected candidates share one softmax with the exact
+ *     tokens (abstract);
+ *   - each entry's RoPE position is its index among the candidates of its
+ *     level (abstract; "Position Encoding").
+ *
+ * Readings where the pages are silent (each one is a choice of this oracle):
+ *   R1 pooler: a d x d linear map W (no bias) applied to the arithmetic mean
+ *      of the node's children's stored keys; one W for all levels and heads.
+ *   R2 top level J: the first level with at most b nodes (J >= 1).
+ *   R3 the last node of each level may be partial; its value is the mean of
+ *      the tokens it has, its key uses the mean of the children it has.
+ *   R4 "at most k" means exactly min(k, |candidates|).
+ *   R5 candidates are ordered by ascending node id; the top-k ranks by the
+ *      selection score, ties going to the smaller node id.
+ *   R6 at a level with n candidates the query sits at RoPE position n - 1.
+ *   R7 logits are scaled by 1/sqrt(d), with no size bias; a selected node
+ *      contributes no summary (its children replace it); tokens are never
+ *      top-k'd.
+ *   R8 decode: the query at position T-1 descends the tree over all T tokens.
+ *   R9 prefill: a chunk [s, s+C) sees the tree over [0, s) plus its own
+ *      causal tokens, which follow the level-0 candidates in the index order.
+ *   R10 GQA: one selection per KV head, ranked by the sum of the G query
+ *      heads' logits.
+ *   R11 RoPE: rotate-half pairs (i, i + d/2), theta_i = base^(-2i/d).
+ *   R12 node keys and values are rounded to the storage type once, when
+ *      formed; child keys are read as stored.
+ */
+#include "recsa_oracle.h"
+
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------ helpers */
+
+static double tok_at(const void* p, int tok_dtype, long long idx) {
+    if (tok_dtype == ORC_TOK_BF16) {
+        uint32_t u = (uint32_t)((const uint16_t*)p)[idx] << 16;
+        float f;
+        memcpy(&f, &u, 4);
+        return (double)f;
+    }
+    return (double)((const float*)p)[idx];
+}
+
+/* bf16 keeps 8 significant bits; nearest-even via nearbyint in the default
+ * rounding mode. Subnormals keep a fixed quantum of 2^-133. */
+static double round_bf16(double x) {
+    if (x == 0.0 || !isfinite(x)) return x;
+    int e;
+    double m = frexp(x, &e); /* x = m 2^e, 0.5 <= |m| < 1 */
+    int bits = 8;
+    if (e + 133 < bits) bits = e + 133;
+    if (bits < 0) return copysign(0.0, x);
+    double y = ldexp(nearbyint(ldexp(m, bits)), e - bits);
+    if (fabs(y) > 3.38953138925153547590470800371487866880e38) return copysign(INFINITY, x);
+    return y;
+}
+
+double orc_round(double x, int storage) {
+    if (storage == ORC_STORE_F32) return (double)(float)x;
+    if (storage == ORC_STORE_BF16) return round_bf16(x);
+    return x;
+}
+
+int orc_levels(long long T, int b, long long* n) {
+    for (int j = 0; j <= ORC_MAXLEV; j++) n[j] = T > 0 ? 1 : 0;
+    n[0] = T;
+    if (T <= 0 || b < 2) return 0;
+    int J = 0;
+    for (int j = 1; j <= ORC_MAXLEV; j++) {
+        n[j] = (n[j - 1] + b - 1) / b;
+        if (J == 0 && n[j] <= b) J = j;
+        if (n[j] == 1 && J != 0) break;
+    }
+    return J;
+}
+
+/* b^j, saturating */
+static long long ipow_sat(int b, int j) {
+    long long p = 1;
+    for (int i = 0; i < j; i++) {
+        if (p > (1LL << 61) / b) return 1LL << 61;
+        p *= b;
+    }
+    return p;
+}
+
+/* --------------------------------------------------------------- tree */
+
+int orc_build(const void* Ktok, const void* Vtok, int tok_dtype, long long T, int d, int b, const float* W,
+              int storage, long long t_from, int J_keep, double* const* Knode, double* const* Vnode) {
+    long long n[ORC_MAXLEV + 1];
+    int J = orc_levels(T, b, n);
+    if (J == 0) return 0;
+    int Jb = J > J_keep ? J : J_keep;
+    if (Jb > ORC_MAXLEV) Jb = ORC_MAXLEV;
+    double* mean = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!mean) return -1;
+    for (int j = 1; j <= Jb; j++) {
+        long long span = ipow_sat(b, j); /* tokens under one node of level j */
+        long long m0 = t_from / span;
+        for (long long m = m0; m < n[j]; m++) {
+            /* value: mean of the subtree's token values ("Core Idea") */
+            long long t_lo = m * span, t_hi = (m + 1) * span < T ? (m + 1) * span : T;
+            for (int i = 0; i < d; i++) {
+                double s = 0.0;
+                for (long long t = t_lo; t < t_hi; t++) s += tok_at(Vtok, tok_dtype, t * d + i);
+                Vnode[j][m * d + i] = orc_round(s / (double)(t_hi - t_lo), storage);
+            }
+            /* key: pooler applied to the mean of the children's stored keys (R1) */
+            long long c_lo = m * b, c_hi = (m + 1) * b < n[j - 1] ? (m + 1) * b : n[j - 1];
+            for (int i = 0; i < d; i++) {
+                double s = 0.0;
+                for (long long c = c_lo; c < c_hi; c++)
+                    s += (j == 1) ? tok_at(Ktok, tok_dtype, c * d + i) : Knode[j - 1][c * d + i];
+                mean[i] = s / (double)(c_hi - c_lo);
+            }
+            for (int r = 0; r < d; r++) {
+                double y = 0.0;
+                for (int c = 0; c < d; c++) y += (double)W[r * d + c] * mean[c];
+                Knode[j][m * d + r] = orc_round(y, storage);
+            }
+        }
+    }
+    free(mean);
+    return Jb;
+}
+
+/* --------------------------------------------------------------- RoPE */
+
+/* rope(x, p): rotate-half pairs (i, i + d/2) by p * theta_i (R11). */
+static void rope(const double* x, long long p, int d, double base, double* y) {
+    int h = d / 2;
+    for (int i = 0; i < h; i++) {
+        double th = pow(base, -2.0 * (double)i / (double)d);
+        double c = cos((double)p * th), s = sin((double)p * th);
+        y[i] = x[i] * c - x[i + h] * s;
+        y[i + h] = x[i + h] * c + x[i] * s;
+    }
+}
+
+/* -------------------------------------------------------------- query */
+
+typedef struct {
+    double S;
+    long long m;
+} scored;
+
+/* descending score, ascending node id on ties (R5) */
+static int by_score(const void* a, const void* b) {
+    const scored* x = (const scored*)a;
+    const scored* y = (const scored*)b;
+    if (x->S > y->S) return -1;
+    if (x->S < y->S) return 1;
+    return (x->m > y->m) - (x->m < y->m);
+}
+
+static int by_id(const void* a, const void* b) {
+    long long x = *(const long long*)a, y = *(const long long*)b;
+    return (x > y) - (x < y);
+}
+
+typedef struct {
+    int level;      /* 0 = token, -1 = local token, j >= 1 = node summary */
+    long long id;
+} entry;
+
+int orc_query(int d, int b, int k, int G, double rope_base, long long T, const double* const* Knode,
+              const double* const* Vnode, const void* Ktok, const void* Vtok, int tok_dtype, const void* Kloc,
+              const void* Vloc, long long nloc, const float* q, double* out, int* sel, double* margin,
+              long long* rows) {
+    if (d <= 0 || d % 2 || b < 2 || k < 1 || G < 1 || T < 0 || nloc < 0 || (T == 0 && nloc == 0)) return -1;
+    long long n[ORC_MAXLEV + 1];
+    int J = orc_levels(T, b, n);
+    double scale = 1.0 / sqrt((double)d);
+
+    long long max_cand = (long long)k * b > b ? (long long)k * b : b;
+    long long max_entries = (long long)J * max_cand + max_cand + nloc + 1;
+    long long* cand = (long long*)malloc(sizeof(long long) * (size_t)max_cand);
+    long long* next = (long long*)malloc(sizeof(long long) * (size_t)max_cand);
+    scored* sc = (scored*)malloc(sizeof(scored) * (size_t)max_cand);
+    double* lg = (double*)malloc(sizeof(double) * (size_t)(max_cand * G));
+    entry* ent = (entry*)malloc(sizeof(entry) * (size_t)max_entries);
+    double* elog = (double*)malloc(sizeof(double) * (size_t)(max_entries * G));
+    double* qd = (double*)malloc(sizeof(double) * (size_t)d);
+    double* qr = (double*)malloc(sizeof(double) * (size_t)(G * d));
+    double* kv = (double*)malloc(sizeof(double) * (size_t)d);
+    double* kr = (double*)malloc(sizeof(double) * (size_t)d);
+    long long* sl = (long long*)malloc(sizeof(long long) * (size_t)(k + 1));
+    if (!cand || !next || !sc || !lg || !ent || !elog || !qd || !qr || !kv || !kr || !sl) {
+        free(cand); free(next); free(sc); free(lg); free(ent); free(elog); free(qd); free(qr); free(kv); free(kr);
+        free(sl);
+        return -1;
+    }
+    if (sel)
+        for (long long i = 0; i < (long long)J * k; i++) sel[i] = -1;
+    long long n_ent = 0, k_rows = 0;
+
+    /* the top level's candidates are all its nodes */
+    long long nc = (J > 0) ? n[J] : 0;
+    for (long long i = 0; i < nc; i++) cand[i] = i;
+
+    for (int j = J; j >= 1; j--) {
+        long long P = nc - 1; /* query position at this level (R6) */
+        for (int g = 0; g < G; g++) {
+            for (int i = 0; i < d; i++) qd[i] = (double)q[g * d + i];
+            rope(qd, P, d, rope_base, qr + g * d);
+        }
+        for (long long i = 0; i < nc; i++) {
+            const double* krow = Knode[j] + cand[i] * d;
+            rope(krow, i, d, rope_base, kr); /* RoPE at the candidate's index (abstract) */
+            double S = 0.0;
+            for (int g = 0; g < G; g++) {
+                double dot = 0.0;
+                for (int e = 0; e < d; e++) dot += qr[g * d + e] * kr[e];
+                lg[i * G + g] = dot * scale;
+                S += lg[i * G + g];
+            }
+            sc[i].S = S;
+            sc[i].m = cand[i];
+        }
+        k_rows += nc;
+        qsort(sc, (size_t)nc, sizeof(scored), by_score);
+        long long kk = nc < k ? nc : k; /* R4 */
+        if (margin) margin[j - 1] = (nc > kk) ? sc[kk - 1].S - sc[kk].S : HUGE_VAL;
+        for (long long r = 0; r < kk; r++) sl[r] = sc[r].m;
+        qsort(sl, (size_t)kk, sizeof(long long), by_id);
+        if (sel)
+            for (long long r = 0; r < kk; r++) sel[(long long)(j - 1) * k + r] = (int)sl[r];
+        /* unselected candidates enter the softmax as summaries (abstract) */
+        for (long long i = 0; i < nc; i++) {
+            int chosen = 0;
+            for (long long r = 0; r < kk; r++) chosen |= (sl[r] == cand[i]);
+            if (chosen) continue;
+            ent[n_ent].level = j;
+            ent[n_ent].id = cand[i];
+            for (int g = 0; g < G; g++) elog[n_ent * G + g] = lg[i * G + g];
+            n_ent++;
+        }
+        /* next candidates: children of the selected nodes, ascending (R5) */
+        long long nn = 0;
+        for (long long r = 0; r < kk; r++) {
+            long long c_lo = sl[r] * b, c_hi = (sl[r] + 1) * b < n[j - 1] ? (sl[r] + 1) * b : n[j - 1];
+            for (long long c = c_lo; c < c_hi; c++) next[nn++] = c;
+        }
+        memcpy(cand, next, sizeof(long long) * (size_t)nn);
+        nc = nn;
+    }
+
+    /* level 0: the exact tokens under the selected leaf-parents, then the
+     * local causal tokens (R9); RoPE index = rank in this list */
+    long long P0 = nc + nloc - 1;
+    for (int g = 0; g < G; g++) {
+        for (int i = 0; i < d; i++) qd[i] = (double)q[g * d + i];
+        rope(qd, P0, d, rope_base, qr + g * d);
+    }
+    for (long long i = 0; i < nc + nloc; i++) {
+        int local = i >= nc;
+        for (int e = 0; e < d; e++)
+            kv[e] = local ? tok_at(Kloc, tok_dtype, (i - nc) * d + e) : tok_at(Ktok, tok_dtype, cand[i] * d + e);
+        rope(kv, i, d, rope_base, kr);
+        ent[n_ent].level = local ? -1 : 0;
+        ent[n_ent].id = local ? i - nc : cand[i];
+        for (int g = 0; g < G; g++) {
+            double dot = 0.0;
+            for (int e = 0; e < d; e++) dot += qr[g * d + e] * kr[e];
+            elog[n_ent * G + g] = dot * scale;
+        }
+        n_ent++;
+    }
+    k_rows += nc + nloc;
+
+    /* one softmax per query head over every entry */
+    for (int g = 0; g < G; g++) {
+        double mx = -HUGE_VAL;
+        for (long long e = 0; e < n_ent; e++) mx = elog[e * G + g] > mx ? elog[e * G + g] : mx;
+        double den = 0.0;
+        for (int i = 0; i < d; i++) out[g * d + i] = 0.0;
+        for (long long e = 0; e < n_ent; e++) {
+            double w = exp(elog[e * G + g] - mx);
+            den += w;
+            for (int i = 0; i < d; i++) {
+                double v;
+                if (ent[e].level >= 1)
+                    v = Vnode[ent[e].level][ent[e].id * d + i];
+                else if (ent[e].level == 0)
+                    v = tok_at(Vtok, tok_dtype, ent[e].id * d + i);
+                else
+                    v = tok_at(Vloc, tok_dtype, ent[e].id * d + i);
+                out[g * d + i] += w * v;
+            }
+        }
+        for (int i = 0; i < d; i++) out[g * d + i] /= den;
+    }
+    if (rows) {
+        rows[0] = k_rows;
+        rows[1] = n_ent;
+    }
+    free(cand); free(next); free(sc); free(lg); free(ent); free(elog); free(qd); free(qr); free(kv); free(kr);
+    free(sl);
+    return J;
+}
