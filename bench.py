@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""RecSA decode benchmark on B200.
+
+Workload (default): one Qwen3-4B-shaped attention layer (32 query heads, 8 KV
+heads, head_dim 128, bf16), L = 524288 cached tokens per sequence, batch 4,
+branching 64, k = 16. One step = append one token to every sequence
+(recsa_append) + one decode query per sequence (recsa_decode). Inputs are
+seeded synthetic data (Gaussian-mixture keys in token runs, N(0,1) values,
+queries aimed at a planted run, random pooler) resident in HBM before timing.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own batch of
+independent sequences (weak scaling, no collective on the data path); the
+step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "RecSA layer decode query-tok/s & prefill tok/s at 524K; % of HBM roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="recsa", choices=["recsa", "reference"])
+    ap.add_argument("--workload", default="decode_524k_b4")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU-baseline sample")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)[kernel]
+        src = open(os.path.join(ROOT, d["source"]), "rb").read()
+        if hashlib.sha256(src).hexdigest()[:16] != d["source_sha"]:
+            return None
+        return d["bytes_per_launch"]
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.lines = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world, local):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier(device_ids=[local])
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------- oracle baseline
+
+
+def oracle_decode_steps(w, K, V, Wp, runs, length0, n_steps, budget_s, seq_ids, threads):
+    """The fp64 oracle doing the decode workload's steps for the given
+    sequences: per step and per KV head, refresh the nodes the new token
+    touched, then one query. Stops at n_steps or when budget_s is spent.
+    Returns (steps done, seconds, query tokens)."""
+    import oracle
+
+    storage = oracle.STORE_BF16 if w.bf16 else oracle.STORE_F32
+    Wf = synth.as_f32(Wp)
+    trees = {}
+    pool = oracle.pool(threads)
+    futs = {}
+    for b in seq_ids:
+        for h in range(w.n_kv_heads):
+            futs[(b, h)] = pool.submit(
+                lambda b=b, h=h: oracle.Tree(w.head_dim, w.branching, length0 + n_steps + 1, storage).build(
+                    K[b, h], V[b, h], length0, Wf))
+    for key, f in futs.items():
+        trees[key] = f.result()
+    L = length0
+    t0 = time.perf_counter()
+    done = 0
+    for s in range(n_steps):
+        L += 1
+
+        def unit(b, h, L=L, s=s):
+            tr = trees[(b, h)]
+            tr.build(K[b, h], V[b, h], L, Wf, t_from=L - 1)
+            q, _ = synth.decode_query(w.seed, b, s, L, w.n_kv_heads, w.group, w.head_dim, w.centroids,
+                                      w.sigma_noise, runs[b], w.bf16)
+            qu = synth.as_f32(np.ascontiguousarray(q[h * w.group:(h + 1) * w.group]))
+            return oracle.query_tree(tr, K[b, h], V[b, h], qu, w.k, w.group, w.rope_base)
+
+        list(pool.map(lambda bh: unit(*bh), [(b, h) for b in seq_ids for h in range(w.n_kv_heads)]))
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    pool.shutdown()
+    return done, dt, done * len(seq_ids)
+
+
+def run_reference(args, w, world, rank):
+    """Reference arm: the fp64 CPU oracle on the same workload and metric."""
+    if rank != 0:
+        return
+    threads = os.cpu_count() or 1
+    L0 = w.length
+    n_seq = 1  # one sequence per step: a bounded sample of the batch
+    sub = w.with_(batch=n_seq)
+    K, V, runs = synth.cache_arrays(sub, L0 + args.warmup + args.steps + 1)
+    Wp = synth.workload_pooler(w)
+    budget = max(30.0, 0.5 * (args.steps + args.warmup))
+    if args.warmup:
+        oracle_decode_steps(sub, K, V, Wp, runs, L0, args.warmup, budget, [0], threads)
+    done, dt, toks = oracle_decode_steps(sub, K, V, Wp, runs, L0 + args.warmup, args.steps, 150.0, [0], threads)
+    v = toks / dt
+    line = {"metric": METRIC, "impl": "reference", "value": v, "unit": "query-tok/s", "n_gpus": args.gpus,
+            "steps": done, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(done, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "L": L0, "batch_sampled": n_seq, "n_q_heads": w.n_q_heads,
+                       "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "branching": w.branching, "k": w.k},
+            "cpu_baseline": {"value": v, "unit": "query-tok/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{done} decode steps of 1 of {w.batch} sequences (8 KV heads each): "
+                                       "right-edge node refresh + one query per KV head, fp64"},
+            "e2e": {"value": v, "unit": "query-tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------------- main
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args.gpus)
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
+
+    from hierarchical_sparse_attention_tree_b200 import RecsaLayer, dense_decode, dense_decode_scratch_bytes
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    B, H, Hq, D = w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim
+    L0 = w.length
+    W_, K_ = args.warmup, args.steps
+    n_total = 2 * (W_ + K_) + 1
+    cap = L0 + n_total
+    seq_off = rank * B
+    bf = torch.bfloat16
+
+    # ---- inputs: host (pinned), then resident in HBM
+    t_gen = time.perf_counter()
+    Kh = torch.empty((B, H, cap, D), dtype=torch.int16, pin_memory=True)
+    Vh = torch.empty((B, H, cap, D), dtype=torch.int16, pin_memory=True)
+    _, _, runs = synth.cache_arrays(w, cap, seq_offset=seq_off, out=(Kh.numpy(), Vh.numpy()))
+    Wp = synth.workload_pooler(w)
+    q_h = torch.from_numpy(np.stack([synth.decode_queries(w, runs, s, L0 + s + 1, seq_off) for s in range(n_total)]))
+    q_h = q_h.view(bf).pin_memory()                                        # [S][B][Hq][D]
+    kn_h = Kh[:, :, L0:L0 + n_total].permute(2, 0, 1, 3).contiguous().view(bf).unsqueeze(2).pin_memory()
+    vn_h = Vh[:, :, L0:L0 + n_total].permute(2, 0, 1, 3).contiguous().view(bf).unsqueeze(2).pin_memory()
+    gen_s = time.perf_counter() - t_gen                                    # kn_h: [S][B][1][H][D]
+
+    layer = RecsaLayer(B, H, Hq, D, w.branching, w.k, cap, torch.from_numpy(Wp).view(bf).to(dev), dtype=bf,
+                       rope_base=w.rope_base, device=dev)
+    layer.k_cache[:, :, :L0].copy_(Kh[:, :, :L0].view(bf))
+    layer.v_cache[:, :, :L0].copy_(Vh[:, :, :L0].view(bf))
+    q_d, kn_d, vn_d = q_h.to(dev), kn_h.to(dev), vn_h.to(dev)
+    out = torch.empty((B, Hq, D), dtype=bf, device=dev)
+    rows = torch.zeros((K_, B, H, 2), dtype=torch.int64, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+
+    # ---- tree build (once), timed on its own
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush.fill_(1.0)
+    e0.record(stream)
+    layer.ctx.build_tree([L0] * B)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    layer.check()
+    build_ms = e0.elapsed_time(e1)
+    es = 2  # bf16
+    n1 = -(-L0 // w.branching)
+    build_bytes = B * H * (2 * L0 * D * es + n1 * D * (2 * es + 4))
+    for j in range(2, layer.tree_shape()[0] + 1):
+        nj = -(-L0 // w.branching ** j)
+        nprev = -(-L0 // w.branching ** (j - 1))
+        build_bytes += B * H * (nprev * D * (es + 4) + nj * D * (2 * es + 4))
+
+    # ---- device-resident decode steps: warm-up, then K timed steps
+    def step(s, ev=None, rows_slot=None):
+        if ev is not None:
+            ev[0].record(stream)
+        layer.append(kn_d[s], vn_d[s])
+        if ev is not None:
+            ev[1].record(stream)
+        layer.decode(q_d[s], out, rows_out=rows_slot)
+        if ev is not None:
+            ev[2].record(stream)
+
+    s_idx = 0
+    for _ in range(W_):
+        flush.fill_(float(s_idx))
+        step(s_idx)
+        s_idx += 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_)]
+    torch.cuda.synchronize(dev)
+    barrier(world, local)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev.index)
+    t_wall = time.perf_counter()
+    for i in range(K_):
+        flush.fill_(float(s_idx))
+        step(s_idx, evs[i], rows[i])
+        s_idx += 1
+    torch.cuda.synchronize(dev)
+    wall_s = time.perf_counter() - t_wall
+    barrier(world, local)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    layer.check()
+    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    app_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    total_s = max_over_ranks(sum(step_ms) / 1e3, world)
+    value = world * B * K_ / total_s
+
+    rows_np = rows.cpu().numpy()
+    dec_bytes = int(rows_np.sum()) * D * es + K_ * 2 * B * Hq * D * es  # gathered K/V rows + q + out
+    dec_bytes_per_launch = dec_bytes / K_
+    peaks, peak_src = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    dec_avg_s = sum(dec_ms) / K_ / 1e3
+    achieved = dec_bytes_per_launch / dec_avg_s / 1e9
+
+    # ---- end to end through the public API: pinned host inputs in, output out
+    e2e = None
+    if not args.no_e2e:
+        out_h = torch.empty((B, Hq, D), dtype=bf, pin_memory=True)
+        qb, kb, vb = torch.empty_like(q_d[0]), torch.empty_like(kn_d[0]), torch.empty_like(vn_d[0])
+
+        def e2e_step(s, ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            qb.copy_(q_h[s], non_blocking=True)
+            kb.copy_(kn_h[s], non_blocking=True)
+            vb.copy_(vn_h[s], non_blocking=True)
+            layer.append(kb, vb)
+            layer.decode(qb, out)
+            out_h.copy_(out, non_blocking=True)
+            if ev is not None:
+                ev[1].record(stream)
+
+        for _ in range(W_):
+            flush.fill_(0.0)
+            e2e_step(s_idx)
+            s_idx += 1
+        ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_)]
+        torch.cuda.synchronize(dev)
+        barrier(world, local)
+        for i in range(K_):
+            flush.fill_(0.0)
+            e2e_step(s_idx, ev2[i])
+            s_idx += 1
+        torch.cuda.synchronize(dev)
+        barrier(world, local)
+        e2e_s = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev2) / 1e3, world)
+        e2e = {"value": world * B * K_ / e2e_s, "unit": "query-tok/s",
+               "h2d_bytes_per_step": int((q_h[0].numel() + kn_h[0].numel() + vn_h[0].numel()) * es),
+               "d2h_bytes_per_step": int(out_h.numel() * es)}
+        layer.check()
+
+    # ---- dense flash-decode comparator on the same cache
+    dense = None
+    if not args.no_dense:
+        Ld = layer.lengths()[0]
+        scratch = torch.empty(dense_decode_scratch_bytes(B, Hq, D), dtype=torch.uint8, device=dev)
+        dout = torch.empty_like(out)
+        for _ in range(3):
+            dense_decode(layer.k_cache, layer.v_cache, q_d[0], dout, Ld, scratch)
+        dms = []
+        for _ in range(10):
+            flush.fill_(2.0)
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            dense_decode(layer.k_cache, layer.v_cache, q_d[0], dout, Ld, scratch)
+            b_.record(stream)
+            torch.cuda.synchronize(dev)
+            dms.append(a.elapsed_time(b_))
+        dmed = statistics.median(dms)
+        dbytes = 2 * B * H * Ld * D * es
+        dense = {"ms": dmed, "query_tok_s": B / (dmed / 1e3), "gbs": dbytes / (dmed / 1e3) / 1e9,
+                 "frac_hbm": dbytes / (dmed / 1e3) / 1e9 / hbm, "length": Ld,
+                 "recsa_step_speedup": dmed / (sum(step_ms) / K_)}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        sub = w.with_(batch=1)
+        Kn, Vn = Kh.numpy(), Vh.numpy()
+        done, dt, toks = oracle_decode_steps(sub, Kn[:1], Vn[:1], Wp, runs[:1], L0, 64, args.cpu_seconds, [0],
+                                             threads)
+        cpu = {"value": toks / dt, "unit": "query-tok/s", "cores": min(threads, H), "kind": "oracle",
+               "sample": f"{done} decode steps of sequence 0 of {B} (8 KV heads in parallel): refresh of the "
+                         "nodes the new token touched + one query per KV head, fp64"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "query-tok/s", "n_gpus": world, "steps": K_, "warmup": W_,
+            "ms_per_step": 1e3 * total_s / K_, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "L": L0, "batch_per_gpu": B, "n_q_heads": Hq, "n_kv_heads": H,
+                       "head_dim": D, "branching": w.branching, "k": w.k,
+                       "step": "recsa_append(1 token/seq) + recsa_decode(1 query/seq)",
+                       "l2": "flushed between steps (256 MB write, outside the events)",
+                       "value_is": "decode query-tok/s; prefill not measured in this line"},
+            "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": achieved, "peak": hbm,
+                         "unit": "GB/s", "frac": achieved / hbm, "peak_source": peak_src,
+                         "traffic": kernel_traffic("decode_kernel"),
+                         "algorithmic_bytes_per_launch": dec_bytes_per_launch, "launch_ms": dec_avg_s * 1e3},
+            "append_ms": sum(app_ms) / K_, "decode_ms": sum(dec_ms) / K_,
+            "rows_per_query": {"k_rows": float(rows_np[..., 0].mean()), "v_rows": float(rows_np[..., 1].mean())},
+            "build_tree": {"ms": build_ms, "gbs": build_bytes / (build_ms / 1e3) / 1e9,
+                           "frac_hbm": build_bytes / (build_ms / 1e3) / 1e9 / hbm},
+            "e2e": e2e, "gpu_launches": 2 * K_, "clocks": clk, "dense_decode": dense, "cpu_baseline": cpu,
+            "wall_s_timed_loop": wall_s, "input_gen_s": gen_s,
+        }
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,392 @@
+// Host side of the C ABI declared in include/recsa.h: argument checks,
+// workspace layout, RoPE table, kernel dispatch. Every launch goes on the
+// caller's stream; nothing here allocates device memory.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/recsa.h"
+#include "common.cuh"
+
+namespace recsa {
+template <typename T, int D>
+cudaError_t launch_build_level(const TreeParams&, int, long long, int, long long, cudaStream_t);
+template <typename T, int D>
+cudaError_t launch_append_one(const TreeParams&, const void*, const void*, cudaStream_t);
+template <typename T, int D>
+cudaError_t launch_copy_tokens(const TreeParams&, const void*, const void*, int, cudaStream_t);
+cudaError_t launch_set_lengths(const TreeParams&, const long long*, cudaStream_t);
+cudaError_t launch_bump_lengths(const TreeParams&, long long, cudaStream_t);
+template <typename T, int D, int G>
+cudaError_t launch_decode(const TreeParams&, const void*, void*, int*, long long*, cudaStream_t);
+template <typename T, int D, int G>
+cudaError_t launch_dense(const void*, const void*, const void*, void*, int, long long, long long, float*,
+                         cudaStream_t);
+int dense_splits(long long units, long long L);
+}  // namespace recsa
+
+using namespace recsa;
+
+struct recsa_ctx {
+    recsa_config cfg;
+    TreeParams p;
+    std::vector<long long> len;  // host mirror of every sequence's length
+    long long* len_stage;        // device [B] staging for recsa_build_tree
+    int G;
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+recsa_status fail(recsa_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return s;
+}
+
+recsa_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(RECSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+long long span_sat(int b, int j) {
+    long long s = 1;
+    for (int i = 0; i < j; i++) {
+        if (s > (1LL << 61) / b) return 1LL << 61;
+        s *= b;
+    }
+    return s;
+}
+
+// Top level over L >= 1 tokens (first level with at most b nodes).
+int levels_for(long long L, int b) {
+    long long n = L;
+    int j = 0;
+    do {
+        n = (n + b - 1) / b;
+        j++;
+    } while (n > b);
+    return j;
+}
+
+recsa_status check_config(const recsa_config* c) {
+    if (!c) return fail(RECSA_ERR_INVALID_ARG, "config is NULL");
+    if (c->batch < 1 || c->n_kv_heads < 1) return fail(RECSA_ERR_INVALID_ARG, "batch and n_kv_heads must be >= 1");
+    if (c->n_q_heads < c->n_kv_heads || c->n_q_heads % c->n_kv_heads)
+        return fail(RECSA_ERR_INVALID_ARG, "n_q_heads must be a multiple of n_kv_heads");
+    int G = c->n_q_heads / c->n_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return fail(RECSA_ERR_UNSUPPORTED, "group size %d not in {1,2,4,8}", G);
+    if (c->head_dim != 64 && c->head_dim != 128) return fail(RECSA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+    if (c->branching < 2 || c->branching > 256) return fail(RECSA_ERR_INVALID_ARG, "branching must be in [2, 256]");
+    if (c->k < 1 || c->k > 64) return fail(RECSA_ERR_INVALID_ARG, "k must be in [1, 64]");
+    if ((long long)c->k * c->branching > 4096) return fail(RECSA_ERR_INVALID_ARG, "k * branching must be <= 4096");
+    if (c->capacity < 1 || c->capacity > (1LL << 31)) return fail(RECSA_ERR_INVALID_ARG, "capacity out of range");
+    if (c->max_chunk < 0 || c->max_chunk > 65536) return fail(RECSA_ERR_INVALID_ARG, "max_chunk out of range");
+    if (!(c->rope_base > 1.0)) return fail(RECSA_ERR_INVALID_ARG, "rope_base must be > 1");
+    if (c->dtype != RECSA_F32 && c->dtype != RECSA_BF16) return fail(RECSA_ERR_INVALID_ARG, "unknown dtype");
+    return RECSA_OK;
+}
+
+struct Layout {
+    int J_cap, npos;
+    long long rows[MAXJ + 1];
+    size_t off_K[MAXJ + 1], off_V[MAXJ + 1], off_VS[MAXJ + 1], off_PK[MAXJ + 1], off_PV[MAXJ + 1];
+    size_t off_Wt, off_rope, off_len, off_err, off_stage, total;
+};
+
+Layout layout_for(const recsa_config* c) {
+    Layout l{};
+    const size_t es = c->dtype == RECSA_BF16 ? 2 : 4;
+    const size_t units = (size_t)c->batch * c->n_kv_heads, D = c->head_dim;
+    l.J_cap = levels_for(c->capacity, c->branching);
+    long long maxc = (long long)c->k * c->branching;
+    if (maxc < c->branching) maxc = c->branching;
+    l.npos = (int)(maxc + c->max_chunk);
+    size_t o = 0;
+    l.rows[0] = c->capacity;
+    for (int j = 1; j <= l.J_cap; j++) {
+        l.rows[j] = (c->capacity + span_sat(c->branching, j) - 1) / span_sat(c->branching, j);
+        size_t n = units * (size_t)l.rows[j] * D;
+        l.off_K[j] = o; o = align256(o + n * es);
+        l.off_V[j] = o; o = align256(o + n * es);
+        l.off_VS[j] = o; o = align256(o + n * 4);
+        l.off_PK[j] = o; o = align256(o + units * D * 4);
+        l.off_PV[j] = o; o = align256(o + units * D * 4);
+    }
+    l.off_Wt = o; o = align256(o + D * D * 4);
+    l.off_rope = o; o = align256(o + (size_t)l.npos * (D / 2) * 8);
+    l.off_len = o; o = align256(o + units * 8);
+    l.off_err = o; o = align256(o + 4);
+    l.off_stage = o; o = align256(o + (size_t)c->batch * 8);
+    l.total = o;
+    return l;
+}
+
+__global__ void pooler_transpose_kernel(const void* w, int bf16, int D, float* wt) {
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= D * D) return;
+    int r = i / D, c = i % D;
+    float x = bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(w)[i])
+                   : reinterpret_cast<const float*>(w)[i];
+    wt[c * D + r] = x;
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+}  // namespace
+
+#define DISPATCH_TD(dtype, D, ...)                                                        \
+    do {                                                                                  \
+        if ((dtype) == RECSA_BF16) {                                                      \
+            using T = __nv_bfloat16;                                                      \
+            if ((D) == 64) { constexpr int DD = 64; __VA_ARGS__; }                        \
+            else { constexpr int DD = 128; __VA_ARGS__; }                                 \
+        } else {                                                                          \
+            using T = float;                                                              \
+            if ((D) == 64) { constexpr int DD = 64; __VA_ARGS__; }                        \
+            else { constexpr int DD = 128; __VA_ARGS__; }                                 \
+        }                                                                                 \
+    } while (0)
+
+#define DISPATCH_G(G, ...)                                                                \
+    do {                                                                                  \
+        switch (G) {                                                                      \
+            case 1: { constexpr int GG = 1; __VA_ARGS__; } break;                         \
+            case 2: { constexpr int GG = 2; __VA_ARGS__; } break;                         \
+            case 4: { constexpr int GG = 4; __VA_ARGS__; } break;                         \
+            default: { constexpr int GG = 8; __VA_ARGS__; } break;                        \
+        }                                                                                 \
+    } while (0)
+
+extern "C" {
+
+const char* recsa_last_error(void) { return g_err.c_str(); }
+
+size_t recsa_workspace_bytes(const recsa_config* cfg) {
+    if (check_config(cfg) != RECSA_OK) return 0;
+    return layout_for(cfg).total;
+}
+
+recsa_status recsa_init(recsa_ctx** out, const recsa_config* cfg, void* k_cache, void* v_cache, void* workspace,
+                        size_t workspace_bytes, const void* pooler_w, recsa_stream_t stream) {
+    if (!out) return fail(RECSA_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    recsa_status st = check_config(cfg);
+    if (st != RECSA_OK) return st;
+    if (!k_cache || !v_cache || !workspace || !pooler_w) return fail(RECSA_ERR_INVALID_ARG, "NULL buffer");
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return fail(RECSA_ERR_INVALID_ARG, "cache not 16-byte aligned");
+    if (!aligned(workspace, 256)) return fail(RECSA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+    Layout l = layout_for(cfg);
+    if (workspace_bytes < l.total)
+        return fail(RECSA_ERR_CAPACITY, "workspace has %zu bytes, needs %zu", workspace_bytes, l.total);
+
+    recsa_ctx* c = new recsa_ctx();
+    c->cfg = *cfg;
+    c->G = cfg->n_q_heads / cfg->n_kv_heads;
+    c->len.assign(cfg->batch, 0);
+    TreeParams& p = c->p;
+    memset(&p, 0, sizeof p);
+    const int D = cfg->head_dim;
+    char* ws = static_cast<char*>(workspace);
+    p.B = cfg->batch; p.H = cfg->n_kv_heads; p.G = c->G; p.D = D; p.b = cfg->branching; p.k = cfg->k;
+    p.J_cap = l.J_cap; p.npos = l.npos; p.cap = cfg->capacity;
+    p.K[0] = k_cache; p.V[0] = v_cache;
+    for (int j = 0; j <= MAXJ; j++) p.span[j] = span_sat(cfg->branching, j);
+    p.rows[0] = cfg->capacity;
+    for (int j = 1; j <= l.J_cap; j++) {
+        p.rows[j] = l.rows[j];
+        p.K[j] = ws + l.off_K[j];
+        p.V[j] = ws + l.off_V[j];
+        p.VS[j] = reinterpret_cast<float*>(ws + l.off_VS[j]);
+        p.PK[j] = reinterpret_cast<float*>(ws + l.off_PK[j]);
+        p.PV[j] = reinterpret_cast<float*>(ws + l.off_PV[j]);
+    }
+    p.Wt = reinterpret_cast<float*>(ws + l.off_Wt);
+    p.rope = reinterpret_cast<float2*>(ws + l.off_rope);
+    p.len = reinterpret_cast<long long*>(ws + l.off_len);
+    p.err = reinterpret_cast<int*>(ws + l.off_err);
+    p.scale = (float)(1.0 / std::sqrt((double)D));
+    c->len_stage = reinterpret_cast<long long*>(ws + l.off_stage);
+
+    // RoPE table, fp64 on the host: (cos, sin)(pos * base^(-2i/d))
+    std::vector<float2> tab((size_t)l.npos * (D / 2));
+    for (int pos = 0; pos < l.npos; pos++)
+        for (int i = 0; i < D / 2; i++) {
+            double th = std::pow(cfg->rope_base, -2.0 * i / D);
+            tab[(size_t)pos * (D / 2) + i] = make_float2((float)std::cos(pos * th), (float)std::sin(pos * th));
+        }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync((void*)p.rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(p.len, 0, (size_t)p.B * p.H * 8, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(p.err, 0, 4, s);
+    if (e == cudaSuccess) {
+        pooler_transpose_kernel<<<(D * D + 255) / 256, 256, 0, s>>>(pooler_w, cfg->dtype == RECSA_BF16, D,
+                                                                     const_cast<float*>(p.Wt));
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) {
+        delete c;
+        return cuda_fail(e, "recsa_init");
+    }
+    *out = c;
+    return RECSA_OK;
+}
+
+void recsa_destroy(recsa_ctx* ctx) { delete ctx; }
+
+recsa_status recsa_build_tree(recsa_ctx* ctx, const long long* lengths, recsa_stream_t stream) {
+    if (!ctx || !lengths) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    const recsa_config& c = ctx->cfg;
+    long long maxL = 0;
+    for (int b = 0; b < c.batch; b++) {
+        if (lengths[b] < 0 || lengths[b] > c.capacity)
+            return fail(RECSA_ERR_CAPACITY, "length %lld of sequence %d outside [0, %lld]", lengths[b], b, c.capacity);
+        maxL = lengths[b] > maxL ? lengths[b] : maxL;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(ctx->len_stage, lengths, (size_t)c.batch * 8, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = launch_set_lengths(ctx->p, ctx->len_stage, s);
+    for (int j = 1; j <= ctx->p.J_cap && e == cudaSuccess; j++) {
+        long long nodes = (maxL + ctx->p.span[j] - 1) / ctx->p.span[j];
+        if (nodes == 0) continue;
+        DISPATCH_TD(c.dtype, c.head_dim, e = launch_build_level<T, DD>(ctx->p, j, 0, 0, nodes, s));
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_build_tree");
+    for (int b = 0; b < c.batch; b++) ctx->len[b] = lengths[b];
+    return RECSA_OK;
+}
+
+recsa_status recsa_append(recsa_ctx* ctx, const void* k_new, const void* v_new, int n, recsa_stream_t stream) {
+    if (!ctx || !k_new || !v_new) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    if (n < 1) return fail(RECSA_ERR_INVALID_ARG, "n must be >= 1");
+    if (!aligned(k_new, 16) || !aligned(v_new, 16)) return fail(RECSA_ERR_INVALID_ARG, "k_new/v_new not 16-byte aligned");
+    const recsa_config& c = ctx->cfg;
+    long long maxL = 0, minL = c.capacity;
+    for (int b = 0; b < c.batch; b++) {
+        if (ctx->len[b] + n > c.capacity)
+            return fail(RECSA_ERR_CAPACITY, "sequence %d: %lld + %d tokens exceed capacity %lld", b, ctx->len[b], n,
+                        c.capacity);
+        maxL = ctx->len[b] > maxL ? ctx->len[b] : maxL;
+        minL = ctx->len[b] < minL ? ctx->len[b] : minL;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (n == 1) {
+        DISPATCH_TD(c.dtype, c.head_dim, e = launch_append_one<T, DD>(ctx->p, k_new, v_new, s));
+    } else {
+        DISPATCH_TD(c.dtype, c.head_dim, e = launch_copy_tokens<T, DD>(ctx->p, k_new, v_new, n, s));
+        for (int j = 1; j <= ctx->p.J_cap && e == cudaSuccess; j++) {
+            const long long sp = ctx->p.span[j];
+            long long nodes = (maxL + n + sp - 1) / sp - minL / sp;
+            if (nodes < 1) nodes = 1;
+            DISPATCH_TD(c.dtype, c.head_dim, e = launch_build_level<T, DD>(ctx->p, j, n, 1, nodes, s));
+        }
+        if (e == cudaSuccess) e = launch_bump_lengths(ctx->p, n, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_append");
+    for (int b = 0; b < c.batch; b++) ctx->len[b] += n;
+    return RECSA_OK;
+}
+
+recsa_status recsa_decode(recsa_ctx* ctx, const void* q, void* out, int* sel_out, long long* rows_out,
+                          recsa_stream_t stream) {
+    if (!ctx || !q || !out) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    const recsa_config& c = ctx->cfg;
+    for (int b = 0; b < c.batch; b++)
+        if (ctx->len[b] < 1) return fail(RECSA_ERR_INVALID_ARG, "sequence %d holds no tokens", b);
+    if (!aligned(q, 16) || !aligned(out, 16)) return fail(RECSA_ERR_INVALID_ARG, "q/out not 16-byte aligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    DISPATCH_TD(c.dtype, c.head_dim,
+                DISPATCH_G(ctx->G, e = launch_decode<T, DD, GG>(ctx->p, q, out, sel_out, rows_out, s)));
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_decode");
+    return RECSA_OK;
+}
+
+size_t recsa_prefill_scratch_bytes(const recsa_config* cfg, int C) {
+    (void)cfg; (void)C;
+    return 0;
+}
+
+recsa_status recsa_prefill(recsa_ctx* ctx, const void* q, const void* k, const void* v, int C, void* out,
+                           int* sel_out, void* scratch, size_t scratch_bytes, recsa_stream_t stream) {
+    (void)ctx; (void)q; (void)k; (void)v; (void)C; (void)out; (void)sel_out; (void)scratch; (void)scratch_bytes;
+    (void)stream;
+    return fail(RECSA_ERR_UNSUPPORTED, "prefill is not built yet");
+}
+
+recsa_status recsa_get_lengths(const recsa_ctx* ctx, long long* lengths) {
+    if (!ctx || !lengths) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    for (int b = 0; b < ctx->cfg.batch; b++) lengths[b] = ctx->len[b];
+    return RECSA_OK;
+}
+
+recsa_status recsa_tree_shape(const recsa_ctx* ctx, int* j_cap, long long* rows) {
+    if (!ctx || !j_cap) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    *j_cap = ctx->p.J_cap;
+    if (rows)
+        for (int j = 0; j <= ctx->p.J_cap; j++) rows[j] = ctx->p.rows[j];
+    return RECSA_OK;
+}
+
+recsa_status recsa_level_arrays(const recsa_ctx* ctx, int level, void** keys, void** values, float** value_sums) {
+    if (!ctx) return fail(RECSA_ERR_INVALID_ARG, "NULL context");
+    if (level < 1 || level > ctx->p.J_cap) return fail(RECSA_ERR_INVALID_ARG, "level %d outside [1, %d]", level,
+                                                       ctx->p.J_cap);
+    if (keys) *keys = ctx->p.K[level];
+    if (values) *values = ctx->p.V[level];
+    if (value_sums) *value_sums = ctx->p.VS[level];
+    return RECSA_OK;
+}
+
+recsa_status recsa_check_device(recsa_ctx* ctx, recsa_stream_t stream) {
+    if (!ctx) return fail(RECSA_ERR_INVALID_ARG, "NULL context");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_check_device");
+    int word = 0;
+    e = cudaMemcpy(&word, ctx->p.err, 4, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(ctx->p.err, 0, 4);
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_check_device");
+    if (word) return fail(RECSA_ERR_DEVICE, "device error word 0x%x (1: length, 2: shape, 4: timeout)", word);
+    return RECSA_OK;
+}
+
+size_t recsa_dense_decode_scratch_bytes(int batch, int n_q_heads, int head_dim) {
+    if (batch < 1 || n_q_heads < 1 || head_dim < 1) return 0;
+    return (size_t)batch * n_q_heads * 256 * (head_dim + 2) * sizeof(float);
+}
+
+recsa_status recsa_dense_decode(const void* k_cache, const void* v_cache, const void* q, void* out, int batch,
+                                int n_kv_heads, int n_q_heads, int head_dim, long long length, long long l_stride,
+                                recsa_dtype dtype, void* scratch, size_t scratch_bytes, recsa_stream_t stream) {
+    if (!k_cache || !v_cache || !q || !out || !scratch) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    if (batch < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return fail(RECSA_ERR_INVALID_ARG, "bad head counts");
+    int G = n_q_heads / n_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return fail(RECSA_ERR_UNSUPPORTED, "group size %d", G);
+    if (head_dim != 64 && head_dim != 128) return fail(RECSA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+    if (length < 1 || l_stride < length) return fail(RECSA_ERR_INVALID_ARG, "bad length / stride");
+    if (scratch_bytes < recsa_dense_decode_scratch_bytes(batch, n_q_heads, head_dim))
+        return fail(RECSA_ERR_CAPACITY, "scratch too small");
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 16))
+        return fail(RECSA_ERR_INVALID_ARG, "buffers not 16-byte aligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    const int units = batch * n_kv_heads;
+    DISPATCH_TD(dtype, head_dim,
+                DISPATCH_G(G, e = launch_dense<T, DD, GG>(k_cache, v_cache, q, out, units, length, l_stride,
+                                                         static_cast<float*>(scratch), s)));
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_dense_decode");
+    return RECSA_OK;
+}
+
+}  // extern "C"

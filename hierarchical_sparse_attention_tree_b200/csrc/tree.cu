@@ -1,0 +1,299 @@
+// Tree build and append kernels.
+//
+// "RecSA ... builds a tree over the KV cache in which each node summarizes its
+// subtree with one key and one mean-pooled value. The keys come from one
+// pooler per layer, shared by all levels" (abstract, paraphrased); node value
+// = mean of every token value in the subtree ("Core Idea", mean pooling).
+//
+// Arithmetic contract, shared by every path that writes a node so that a tree
+// grown token by token is bit-identical to one built at once:
+//   value sum  VS_j[m] = (((0 + s_0) + s_1) + ...) over the children in order,
+//              s_c = token value (j = 1) or VS_{j-1}[c] (j >= 2), fp32;
+//   value      V_j[m]  = round(VS_j[m] / tokens(m));
+//   key        K_j[m]  = round(W * (((0 + k_0) + k_1) + ... ) / children(m)),
+//              k_c = stored child key; the product is an fmaf chain over the
+//              input coordinate c = 0..d-1 starting from 0;
+//   right edge PK_j, PV_j = the same running sums over every child of the
+//              last node but its last child, so an append only adds the
+//              completed child and the new last child.
+#include "common.cuh"
+
+namespace recsa {
+
+// ------------------------------------------------------------- lengths
+
+__global__ void set_lengths_kernel(long long* len, const long long* src, int B, int H) {
+    int u = blockIdx.x * blockDim.x + threadIdx.x;
+    if (u < B * H) len[u] = src[u / H];
+}
+
+__global__ void bump_lengths_kernel(long long* len, int n_units, long long n) {
+    int u = blockIdx.x * blockDim.x + threadIdx.x;
+    if (u < n_units) len[u] += n;
+}
+
+// ------------------------------------------------------------ copy rows
+
+// Copies n new tokens [B][n][H][D] into the cache after each unit's tokens.
+template <typename T, int D>
+__global__ void copy_tokens_kernel(TreeParams p, const T* __restrict__ k_new, const T* __restrict__ v_new, int n) {
+    constexpr int VEC = 16 / sizeof(T);
+    constexpr int PER_ROW = D / VEC;
+    long long units = (long long)p.B * p.H;
+    long long total = units * n * PER_ROW;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        int piece = (int)(i % PER_ROW);
+        long long r = i / PER_ROW;      // (b, t, h)
+        int h = (int)(r % p.H);
+        long long t = (r / p.H) % n;
+        int b = (int)(r / ((long long)p.H * n));
+        long long u = (long long)b * p.H + h;
+        long long L = p.len[u];
+        if (L + t >= p.cap) { flag_error(p.err, ERR_LENGTH); continue; }
+        const uint4* ks = reinterpret_cast<const uint4*>(k_new + (r * D)) + piece;
+        const uint4* vs = reinterpret_cast<const uint4*>(v_new + (r * D)) + piece;
+        T* kd = reinterpret_cast<T*>(p.K[0]) + (u * p.cap + L + t) * D;
+        T* vd = reinterpret_cast<T*>(p.V[0]) + (u * p.cap + L + t) * D;
+        reinterpret_cast<uint4*>(kd)[piece] = *ks;
+        reinterpret_cast<uint4*>(vd)[piece] = *vs;
+    }
+}
+
+// ---------------------------------------------------------- build level
+
+// One warp per node of level j (unit = blockIdx.y). Recomputes nodes
+// m >= m0 of the tree over L' = len[u] + add tokens, where m0 = 0 for a full
+// build and len[u] / b^j when `add` new tokens were just copied in.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) build_level_kernel(TreeParams p, int j, long long add, int from_len) {
+    constexpr int DPL = D / 32;  // columns per lane, contiguous
+    extern __shared__ float smem[];
+    float* Wt = smem;                    // [D][D]
+    float* km = smem + D * D;            // [warps][D]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    for (int i = threadIdx.x; i < D * D / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(Wt)[i] = reinterpret_cast<const float4*>(p.Wt)[i];
+    __syncthreads();
+
+    const long long u = blockIdx.y;
+    const long long L = p.len[u] + add;
+    const long long n_j = level_rows(p, j, L);
+    const long long n_prev = level_rows(p, j - 1, L);
+    const long long m0 = from_len ? p.len[u] / p.span[j] : 0;
+    const long long m = m0 + (long long)blockIdx.x * nwarps + warp;
+    if (m >= n_j) return;
+    if (n_j > p.rows[j] || L > p.cap) {
+        if (lane == 0) flag_error(p.err, ERR_SHAPE);
+        return;
+    }
+
+    const long long c_lo = m * p.b;
+    const long long c_hi = min(c_lo + (long long)p.b, n_prev);
+    const bool right_edge = (m == n_j - 1);
+    const T* Kc = reinterpret_cast<const T*>(p.K[j - 1]) + (u * p.rows[j - 1]) * D + lane * DPL;
+    const T* Vc = reinterpret_cast<const T*>(p.V[0]) + (u * p.cap) * D + lane * DPL;  // j == 1
+    const float* Sc = (j >= 2) ? p.VS[j - 1] + (u * p.rows[j - 1]) * D + lane * DPL : nullptr;
+
+    float ks[DPL], vs[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; e++) { ks[e] = 0.f; vs[e] = 0.f; }
+
+    constexpr int U = 8;
+    for (long long c0 = c_lo; c0 < c_hi; c0 += U) {
+        float kb[U][DPL], vb[U][DPL];
+#pragma unroll
+        for (int i = 0; i < U; i++) {
+            long long c = c0 + i;
+            if (c < c_hi) {
+                load_vec<T, DPL>(Kc + c * D, kb[i]);
+                if (j == 1)
+                    load_vec<T, DPL>(Vc + c * D, vb[i]);
+                else
+                    load_vec<float, DPL>(Sc + c * D, vb[i]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < U; i++) {
+            long long c = c0 + i;
+            if (c < c_hi) {
+                if (right_edge && c == c_hi - 1) {
+                    float* pk = p.PK[j] + u * D + lane * DPL;
+                    float* pv = p.PV[j] + u * D + lane * DPL;
+#pragma unroll
+                    for (int e = 0; e < DPL; e++) { pk[e] = ks[e]; pv[e] = vs[e]; }
+                }
+#pragma unroll
+                for (int e = 0; e < DPL; e++) { ks[e] = ks[e] + kb[i][e]; vs[e] = vs[e] + vb[i][e]; }
+            }
+        }
+    }
+
+    const long long t_lo = m * p.span[j];
+    const long long cnt = min(t_lo + p.span[j], L) - t_lo;
+    const float fcnt = (float)cnt, fnc = (float)(c_hi - c_lo);
+    float* vs_out = p.VS[j] + (u * p.rows[j] + m) * D + lane * DPL;
+    T* v_out = reinterpret_cast<T*>(p.V[j]) + (u * p.rows[j] + m) * D + lane * DPL;
+    float vm[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; e++) { vs_out[e] = vs[e]; vm[e] = __fdiv_rn(vs[e], fcnt); }
+    store_vec<T, DPL>(v_out, vm);
+
+    float* kmw = km + warp * D;
+#pragma unroll
+    for (int e = 0; e < DPL; e++) kmw[lane * DPL + e] = __fdiv_rn(ks[e], fnc);
+    __syncwarp();
+    float y[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; e++) y[e] = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < D; c++) {
+        const float x = kmw[c];
+        float w[DPL];
+#pragma unroll
+        for (int e = 0; e < DPL; e++) w[e] = Wt[c * D + lane * DPL + e];
+#pragma unroll
+        for (int e = 0; e < DPL; e++) y[e] = fmaf(w[e], x, y[e]);
+    }
+    T* k_out = reinterpret_cast<T*>(p.K[j]) + (u * p.rows[j] + m) * D + lane * DPL;
+    store_vec<T, DPL>(k_out, y);
+}
+
+// ----------------------------------------------------------- append one
+
+// Appends one token per unit and refreshes the right edge of every level.
+// One CTA of D threads per unit; thread t owns coordinate t.
+template <typename T, int D>
+__global__ void __launch_bounds__(D) append_one_kernel(TreeParams p, const T* __restrict__ k_new,
+                                                       const T* __restrict__ v_new) {
+    extern __shared__ float smem[];
+    float* Wt = smem;           // [D][D]
+    float* km = smem + D * D;   // [D]
+    const int t = threadIdx.x;
+    const long long u = blockIdx.x;
+    const int bseq = (int)(u / p.H), h = (int)(u % p.H);
+    const long long P = p.len[u];  // position of the new token
+    if (P >= p.cap) {
+        if (t == 0) flag_error(p.err, ERR_LENGTH);
+        return;
+    }
+    for (int i = t; i < D * D / 4; i += D)
+        reinterpret_cast<float4*>(Wt)[i] = reinterpret_cast<const float4*>(p.Wt)[i];
+
+    const long long src = ((long long)bseq * p.H + h) * D + t;  // [B][1][H][D]
+    const T kn = k_new[src], vn = v_new[src];
+    T* Kt = reinterpret_cast<T*>(p.K[0]) + u * p.cap * D;
+    T* Vt = reinterpret_cast<T*>(p.V[0]) + u * p.cap * D;
+    Kt[P * D + t] = kn;
+    Vt[P * D + t] = vn;
+
+    float kcur = to_f(kn), vcur = to_f(vn);                       // new last child of level j-1
+    float kold = P > 0 ? to_f(Kt[(P - 1) * D + t]) : 0.f;         // completed child (token P-1)
+    float vold = P > 0 ? to_f(Vt[(P - 1) * D + t]) : 0.f;
+    __syncthreads();
+
+    for (int j = 1; j <= p.J_cap; j++) {
+        const long long sj = p.span[j], sjm = p.span[j - 1];
+        const long long m = P / sj;
+        const bool new_node = (P % sj) == 0;
+        const bool child_done = (P % sjm) == 0;  // level j-1 started a new node at P
+        float* pkp = p.PK[j] + u * D + t;
+        float* pvp = p.PV[j] + u * D + t;
+        float pk, pv;
+        if (new_node) {
+            pk = 0.f; pv = 0.f;
+            *pkp = pk; *pvp = pv;
+        } else {
+            pk = *pkp; pv = *pvp;
+            if (child_done) {
+                pk = pk + kold; pv = pv + vold;
+                *pkp = pk; *pvp = pv;
+            }
+        }
+        const float ks = pk + kcur, vsum = pv + vcur;
+        const long long cnt = P + 1 - m * sj;
+        const long long nc = P / sjm - m * p.b + 1;
+        const long long row = u * p.rows[j] + m;
+        p.VS[j][row * D + t] = vsum;
+        reinterpret_cast<T*>(p.V[j])[row * D + t] = from_f<T>(__fdiv_rn(vsum, (float)cnt));
+        km[t] = __fdiv_rn(ks, (float)nc);
+        __syncthreads();
+        float y = 0.f;
+#pragma unroll 8
+        for (int c = 0; c < D; c++) y = fmaf(Wt[c * D + t], km[c], y);
+        const T ky = from_f<T>(y);
+        reinterpret_cast<T*>(p.K[j])[row * D + t] = ky;
+        // inputs of level j + 1
+        if ((P % sj) == 0 && m > 0) {  // node m - 1 of level j completed at the previous token
+            const long long prow = u * p.rows[j] + m - 1;
+            kold = to_f(reinterpret_cast<const T*>(p.K[j])[prow * D + t]);
+            vold = p.VS[j][prow * D + t];
+        }
+        kcur = to_f(ky);
+        vcur = vsum;
+        __syncthreads();
+    }
+    if (t == 0) p.len[u] = P + 1;
+}
+
+// --------------------------------------------------------------- launch
+
+template <typename T, int D>
+cudaError_t launch_build_level(const TreeParams& p, int j, long long add, int from_len, long long max_nodes,
+                               cudaStream_t s) {
+    const int threads = 256, wpb = threads / 32;
+    size_t smem = (size_t)(D * D + wpb * D) * sizeof(float);
+    auto kern = build_level_kernel<T, D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    long long gx = (max_nodes + wpb - 1) / wpb;
+    if (gx < 1) gx = 1;
+    dim3 grid((unsigned)gx, (unsigned)(p.B * p.H));
+    kern<<<grid, threads, smem, s>>>(p, j, add, from_len);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_append_one(const TreeParams& p, const void* k_new, const void* v_new, cudaStream_t s) {
+    size_t smem = (size_t)(D * D + D) * sizeof(float);
+    auto kern = append_one_kernel<T, D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<p.B * p.H, D, smem, s>>>(p, reinterpret_cast<const T*>(k_new), reinterpret_cast<const T*>(v_new));
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_copy_tokens(const TreeParams& p, const void* k_new, const void* v_new, int n, cudaStream_t s) {
+    long long total = (long long)p.B * p.H * n * (D * sizeof(T) / 16);
+    long long blocks = (total + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    copy_tokens_kernel<T, D><<<(unsigned)blocks, 256, 0, s>>>(p, reinterpret_cast<const T*>(k_new),
+                                                               reinterpret_cast<const T*>(v_new), n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_set_lengths(const TreeParams& p, const long long* dev_src, cudaStream_t s) {
+    int n = p.B * p.H;
+    set_lengths_kernel<<<(n + 255) / 256, 256, 0, s>>>(p.len, dev_src, p.B, p.H);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bump_lengths(const TreeParams& p, long long n, cudaStream_t s) {
+    int units = p.B * p.H;
+    bump_lengths_kernel<<<(units + 255) / 256, 256, 0, s>>>(p.len, units, n);
+    return cudaGetLastError();
+}
+
+#define RECSA_INST_TREE(T, D)                                                                                   \
+    template cudaError_t launch_build_level<T, D>(const TreeParams&, int, long long, int, long long,           \
+                                                  cudaStream_t);                                               \
+    template cudaError_t launch_append_one<T, D>(const TreeParams&, const void*, const void*, cudaStream_t);   \
+    template cudaError_t launch_copy_tokens<T, D>(const TreeParams&, const void*, const void*, int, cudaStream_t);
+RECSA_INST_TREE(float, 64)
+RECSA_INST_TREE(float, 128)
+RECSA_INST_TREE(__nv_bfloat16, 64)
+RECSA_INST_TREE(__nv_bfloat16, 128)
+
+}  // namespace recsa

@@ -1,0 +1,68 @@
+"""RecsaLayer: allocates the KV cache and workspace with PyTorch and drives
+one recsa_ctx through the C ABI. Marshalling only; the work runs in
+librecsa.so."""
+from __future__ import annotations
+
+import torch
+
+from . import recsa as _r
+
+
+class RecsaLayer:
+    def __init__(self, batch, n_kv_heads, n_q_heads, head_dim, branching, k, capacity, pooler_w: torch.Tensor,
+                 dtype=torch.bfloat16, rope_base=1e6, max_chunk=0, device="cuda", stream=None):
+        self.cfg = _r.make_config(batch, n_kv_heads, n_q_heads, head_dim, branching, k, capacity, dtype, rope_base,
+                                  max_chunk)
+        self.dtype, self.device = dtype, torch.device(device)
+        self.k_cache = torch.zeros(batch, n_kv_heads, capacity, head_dim, dtype=dtype, device=device)
+        self.v_cache = torch.zeros_like(self.k_cache)
+        self.workspace = torch.zeros(_r.workspace_bytes(self.cfg), dtype=torch.uint8, device=device)
+        w = pooler_w.to(device=device, dtype=dtype).contiguous()
+        self.ctx = _r.Context(self.cfg, self.k_cache, self.v_cache, self.workspace, w, stream)
+        torch.cuda.current_stream(self.device).synchronize() if stream is None else stream.synchronize()
+        self._scratch = None
+
+    @property
+    def G(self) -> int:
+        return self.cfg.n_q_heads // self.cfg.n_kv_heads
+
+    def load(self, K: torch.Tensor, V: torch.Tensor, lengths, stream=None):
+        """Copy tokens [B][H][L][d] into the cache and build the tree over
+        the first lengths[b] tokens of each sequence."""
+        L = K.shape[2]
+        self.k_cache[:, :, :L].copy_(K, non_blocking=True)
+        self.v_cache[:, :, :L].copy_(V, non_blocking=True)
+        self.ctx.build_tree(lengths, stream)
+
+    def append(self, k_new, v_new, stream=None):
+        self.ctx.append(k_new, v_new, stream)
+
+    def decode(self, q, out=None, sel_out=None, rows_out=None, stream=None):
+        if out is None:
+            out = torch.empty_like(q)
+        self.ctx.decode(q, out, sel_out, rows_out, stream)
+        return out
+
+    def prefill(self, q, k, v, out=None, sel_out=None, stream=None):
+        if out is None:
+            out = torch.empty_like(q)
+        need = self.ctx.prefill_scratch_bytes(q.shape[1])
+        if self._scratch is None or self._scratch.numel() < need:
+            self._scratch = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
+        self.ctx.prefill(q, k, v, out, sel_out, self._scratch, stream)
+        return out
+
+    def lengths(self):
+        return self.ctx.lengths()
+
+    def level(self, j):
+        return self.ctx.level(j)
+
+    def tree_shape(self):
+        return self.ctx.tree_shape()
+
+    def check(self, stream=None):
+        self.ctx.check_device(stream)
+
+    def close(self):
+        self.ctx.close()

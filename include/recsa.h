@@ -1,0 +1,156 @@
+/*
+ * recsa.h — C ABI of librecsa.so, RecSA (Recursive Sparse Attention) tree
+ * sparse attention for one attention layer on an NVIDIA B200 (sm_100a).
+ *
+ * The method ("Recursive Sparse Attention: Million-Token Length
+ * Extrapolation at Logarithmic Cost", arXiv 2611.07232, abstract; the
+ * kongchang.com RecSA article, "Core Idea" and "Position Encoding"):
+ *   - a tree is kept over each (sequence, KV head) slice of the KV cache; the
+ *     bottom level is the exact tokens, node m of level j covers children
+ *     [m b, (m+1) b) of level j-1 and tokens [m b^j, (m+1) b^j);
+ *   - a node's value is the exact mean of its subtree's token values; its key
+ *     is one per-layer pooler W (d x d, y = W x) applied to the mean of its
+ *     children's stored keys;
+ *   - the top level J is the first level with at most b nodes; a query scores
+ *     every top-level node, keeps the k best (ranked by the sum of its G query
+ *     heads' logits, ties to the smaller node id), scores the children of the
+ *     kept nodes, and so on down to the tokens;
+ *   - every scored-but-not-kept node enters one shared softmax as a summary
+ *     (its key's logit, its mean value); the tokens under the kept level-1
+ *     nodes enter exactly;
+ *   - each entry is RoPE-rotated (rotate-half, theta_i = base^(-2i/d)) at its
+ *     index among its level's candidates (ascending node order), and the query
+ *     of a level with n candidates sits at index n-1; logits are scaled by
+ *     1/sqrt(d).
+ *
+ * Memory. The caller owns all device memory: the KV cache, the workspace
+ * (tree levels, running sums, RoPE table, pooler copy, lengths) and every
+ * input and output buffer. The library never allocates device memory and
+ * never synchronises the device except in recsa_check_device.
+ *
+ * Layouts (row-major, element type = config.dtype unless stated):
+ *   cache      K, V [B][H_kv][capacity][d]   keys stored before RoPE
+ *   decode     q, out [B][H_q][d]            query head h reads KV head h / G
+ *   append     k_new, v_new [B][n][H_kv][d]
+ *   prefill    q, out [B][C][H_q][d]; k, v [B][C][H_kv][d]
+ *
+ * Streams. Every call that launches work is asynchronous on the given
+ * stream (a cudaStream_t; NULL = legacy default stream). Argument errors are
+ * detected on the host, return a status and launch nothing;
+ * recsa_last_error() then describes the error (thread-local string).
+ */
+#ifndef RECSA_H
+#define RECSA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* recsa_stream_t; /* same type as cudaStream_t */
+typedef struct recsa_ctx recsa_ctx;
+
+typedef enum {
+    RECSA_OK = 0,
+    RECSA_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or config   */
+    RECSA_ERR_CAPACITY = 2,    /* would exceed capacity or the workspace    */
+    RECSA_ERR_UNSUPPORTED = 3, /* valid but not built (e.g. head_dim 96)   */
+    RECSA_ERR_CUDA = 4,        /* a CUDA runtime call failed                */
+    RECSA_ERR_DEVICE = 5       /* a kernel reported an inconsistent state   */
+} recsa_status;
+
+typedef enum { RECSA_F32 = 0, RECSA_BF16 = 1 } recsa_dtype;
+
+typedef struct {
+    int batch;          /* B independent sequences, >= 1                      */
+    int n_kv_heads;     /* H_kv >= 1                                          */
+    int n_q_heads;      /* H_q = G * H_kv, G in {1, 2, 4, 8}                  */
+    int head_dim;       /* d in {64, 128}                                     */
+    int branching;      /* b in [2, 256]                                      */
+    int k;              /* kept nodes per level, 1 <= k <= 64, k * b <= 4096  */
+    long long capacity; /* maximum tokens per sequence, >= 1                  */
+    int max_chunk;      /* largest prefill chunk C (0: prefill not used)      */
+    double rope_base;   /* RoPE base, > 1                                     */
+    recsa_dtype dtype;  /* storage and I/O type of cache, nodes, q, out       */
+} recsa_config;
+
+/* Bytes of device workspace recsa_init needs for this configuration (0 if
+ * the configuration is invalid; recsa_last_error says why). */
+size_t recsa_workspace_bytes(const recsa_config* cfg);
+
+/* Creates a context. k_cache / v_cache: the caller's cache buffers (layout
+ * above), borrowed for the context's lifetime. workspace: >=
+ * recsa_workspace_bytes(cfg) bytes of device memory, 256-byte aligned, owned
+ * by the context until recsa_destroy. pooler_w: device pointer to W [d][d]
+ * (row-major, y = W x) in cfg->dtype; copied into the workspace on `stream`,
+ * so it may be freed once that stream has passed this call. All sequence
+ * lengths start at 0. On error *out is left NULL. */
+recsa_status recsa_init(recsa_ctx** out, const recsa_config* cfg, void* k_cache, void* v_cache, void* workspace,
+                        size_t workspace_bytes, const void* pooler_w, recsa_stream_t stream);
+
+/* Sets sequence b's length to lengths[b] (host array of B entries, each in
+ * [0, capacity]) and builds every tree level from the tokens already in the
+ * cache ("builds a tree over the KV cache", abstract). */
+recsa_status recsa_build_tree(recsa_ctx* ctx, const long long* lengths, recsa_stream_t stream);
+
+/* Appends n >= 1 tokens to every sequence: copies k_new / v_new
+ * ([B][n][H_kv][d], device) into the cache after each sequence's current
+ * tokens, then brings every node whose subtree gained tokens up to date
+ * (right-edge nodes stay exact means; keys are recomputed by the pooler).
+ * RECSA_ERR_CAPACITY (nothing launched) if any sequence would exceed the
+ * capacity. */
+recsa_status recsa_append(recsa_ctx* ctx, const void* k_new, const void* v_new, int n, recsa_stream_t stream);
+
+/* One decode query per sequence (per-level top-k descent, shared softmax and
+ * candidate-index RoPE: abstract; "Core Idea"; "Position Encoding").
+ * q [B][H_q][d] (device) is the query of the last cached position: append
+ * the current token first; the query descends the tree over every cached
+ * token. out [B][H_q][d] (device). sel_out (nullable, device int32 [B][H_kv][J_cap][k]): the kept
+ * node ids of level j in row j-1, ascending, -1 padded (levels above the
+ * current top level are all -1). rows_out (nullable, device int64
+ * [B][H_kv][2]): K rows and V rows (= softmax entries) read per KV head.
+ * Every sequence must hold at least one token. */
+recsa_status recsa_decode(recsa_ctx* ctx, const void* q, void* out, int* sel_out, long long* rows_out,
+                          recsa_stream_t stream);
+
+/* Chunked causal prefill of C tokens per sequence (1 <= C <= max_chunk):
+ * token t of the chunk attends the tree over the sequence's cached tokens
+ * [0, s) plus the chunk's own tokens s..t exactly; those follow the level-0
+ * candidates in the RoPE index order. q [B][C][H_q][d], k, v
+ * [B][C][H_kv][d], out [B][C][H_q][d] (device). sel_out (nullable, device
+ * int32 [B][C][H_kv][J_cap][k]) as in recsa_decode. scratch: device memory
+ * of recsa_prefill_scratch_bytes(cfg, C) bytes, 256-byte aligned. The chunk
+ * is not appended: call recsa_append(k, v, C) afterwards. */
+size_t recsa_prefill_scratch_bytes(const recsa_config* cfg, int C);
+recsa_status recsa_prefill(recsa_ctx* ctx, const void* q, const void* k, const void* v, int C, void* out,
+                           int* sel_out, void* scratch, size_t scratch_bytes, recsa_stream_t stream);
+
+/* Host-side view of the state, for tests and tools. */
+recsa_status recsa_get_lengths(const recsa_ctx* ctx, long long* lengths /* host [B] */);
+/* J_cap (levels kept) and, for j = 1..J_cap, rows[j] = node rows per unit. */
+recsa_status recsa_tree_shape(const recsa_ctx* ctx, int* j_cap, long long* rows /* host [J_cap + 1] */);
+/* Device pointers of level j (1..J_cap): keys and values [B][H_kv][rows[j]][d]
+ * in cfg->dtype, and the fp32 value sums [B][H_kv][rows[j]][d]. */
+recsa_status recsa_level_arrays(const recsa_ctx* ctx, int level, void** keys, void** values, float** value_sums);
+
+/* Waits for `stream`, then reads and clears the device error word:
+ * RECSA_ERR_DEVICE if a kernel flagged an inconsistent state. */
+recsa_status recsa_check_device(recsa_ctx* ctx, recsa_stream_t stream);
+
+const char* recsa_last_error(void);
+void recsa_destroy(recsa_ctx* ctx);
+
+/* Comparator, not part of the method: dense GQA flash-decode of one query
+ * per sequence over every cached token, keys used as stored (no RoPE).
+ * k_cache, v_cache [B][H_kv][L_stride][d], q, out [B][H_q][d], bf16 or fp32.
+ * scratch: recsa_dense_decode_scratch_bytes(...) bytes of device memory. */
+size_t recsa_dense_decode_scratch_bytes(int batch, int n_q_heads, int head_dim);
+recsa_status recsa_dense_decode(const void* k_cache, const void* v_cache, const void* q, void* out, int batch,
+                                int n_kv_heads, int n_q_heads, int head_dim, long long length, long long l_stride,
+                                recsa_dtype dtype, void* scratch, size_t scratch_bytes, recsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -168,3 +168,31 @@ def plain(seed: int, a: int, shape, mean=0.0, scale=1.0, bf16=False) -> np.ndarr
     out = _alloc(shape, bf16)
     _load().synth_plain(seed, a, out.size, mean, scale, int(bf16), _ptr(out))
     return out
+
+
+def cache_arrays(w, length: int, nthreads=None, seq_offset: int = 0, out=None):
+    """Keys and values [B][H][length][d] of a workload (np.int16 bf16 bits or
+    float32) and each sequence's run table. Sequence b uses generator
+    sequence id seq_offset + b. `out` = (K, V) preallocated arrays, optional."""
+    B, H, d = w.batch, w.n_kv_heads, w.head_dim
+    K, V = out if out is not None else (_alloc((B, H, length, d), w.bf16), _alloc((B, H, length, d), w.bf16))
+    run_tables = []
+    for b in range(B):
+        s = seq_offset + b
+        rs = runs(w.seed, s, length, w.run_min, w.run_max)
+        run_tables.append(rs)
+        keys(w.seed, s, H, d, w.centroids, w.sigma_noise, rs, 0, length, w.bf16, out=K[b], head_stride=length * d,
+             nthreads=nthreads)
+        values(w.seed, s, H, d, 0, length, w.bf16, out=V[b], head_stride=length * d, nthreads=nthreads)
+    return K, V, run_tables
+
+
+def decode_queries(w, run_tables, step: int, length: int, seq_offset: int = 0):
+    """Decode queries [B][H*G][d] for `step` with `length` cached tokens."""
+    qs = [decode_query(w.seed, seq_offset + b, step, length, w.n_kv_heads, w.group, w.head_dim, w.centroids,
+                       w.sigma_noise, run_tables[b], w.bf16)[0] for b in range(w.batch)]
+    return np.stack(qs)
+
+
+def workload_pooler(w):
+    return pooler(w.seed, w.head_dim, w.bf16)

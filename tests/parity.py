@@ -1,0 +1,94 @@
+"""Helpers that compare the CUDA path with the fp64 oracle (tests only)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import synth
+
+NEAR_TIE = 1e-4  # oracle margin S_(k) - S_(k+1) below which a query is a near tie
+
+
+def to_dev(a: np.ndarray, bf16: bool, device="cuda") -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if bf16:
+        t = t.view(torch.bfloat16)
+    return t.to(device)
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def storage_of(bf16: bool) -> int:
+    return oracle.STORE_BF16 if bf16 else oracle.STORE_F32
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    a = np.abs(x)
+    a = np.where(a < 2.0 ** -126, 2.0 ** -126, a)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+def compare_nodes(gpu: np.ndarray, ref: np.ndarray, bf16: bool):
+    """Returns (ok, n_off_by_one_ulp). bf16: at most 1 ulp of the larger
+    magnitude; fp32: |diff| <= 1e-5 + 1e-5 |ref|."""
+    if bf16:
+        ulp = bf16_ulp(np.maximum(np.abs(gpu), np.abs(ref)))
+        diff = np.abs(gpu - ref)
+        return bool((diff <= ulp * 1.0000001).all()), int((diff > 0).sum())
+    ok = np.abs(gpu - ref) <= 1e-5 + 1e-5 * np.abs(ref)
+    return bool(ok.all()), int((~ok).sum())
+
+
+def unit_tokens(K: np.ndarray, b: int, h: int, L: int):
+    return K[b, h, :L]
+
+
+def gpu_tree_unit(layer, b: int, h: int, J: int, L: int):
+    """GPU node arrays of one unit, levels 1..J, as fp64 numpy (rows < n_j)."""
+    Ks, Vs = [None], [None]
+    for j in range(1, J + 1):
+        n = -(-L // layer.cfg.branching ** j)
+        kj, vj, _ = layer.level(j)
+        Ks.append(to_f64(kj[b, h, :n]))
+        Vs.append(to_f64(vj[b, h, :n]))
+    return Ks, Vs
+
+
+def oracle_query(tree_K, tree_V, K, V, b, h, L, q_unit, w, Kloc=None, Vloc=None):
+    """q_unit: [G][d] float32."""
+    return oracle.query(tree_K, tree_V, K[b, h], V[b, h], L, q_unit, w.head_dim, w.branching, w.k, w.group,
+                        w.rope_base, Kloc, Vloc)
+
+
+def q_unit(q: np.ndarray, b: int, h: int, G: int) -> np.ndarray:
+    """Query heads of KV head h of sequence b, as float32 [G][d]."""
+    return synth.as_f32(np.ascontiguousarray(q[b, h * G:(h + 1) * G]))
+
+
+def check_decode(gpu_out, gpu_sel, gpu_rows, ref, b, h, G, tol, report):
+    """Compares one unit's decode with an oracle result; near ties are counted
+    and skipped."""
+    if len(ref["margin"]) and ref["margin"].min() < NEAR_TIE:
+        report["near_ties"] += 1
+        return
+    J = ref["J"]
+    for j in range(1, J + 1):
+        got = [x for x in gpu_sel[b, h, j - 1].tolist() if x >= 0]
+        want = [x for x in ref["sel"][j - 1].tolist() if x >= 0]
+        if got != want:
+            report["sel_mismatch"] += 1
+            report.setdefault("first_mismatch", (b, h, j, got, want))
+            return
+    assert (gpu_sel[b, h, J:] == -1).all()
+    err = np.abs(gpu_out[b, h * G:(h + 1) * G] - ref["out"]).max()
+    report["max_abs"] = max(report["max_abs"], float(err))
+    assert err <= tol, (b, h, err)
+    assert tuple(gpu_rows[b, h]) == (ref["k_rows"], ref["v_rows"]), (gpu_rows[b, h], ref["k_rows"], ref["v_rows"])
+    report["checked"] += 1
+
+
+def new_report():
+    return {"checked": 0, "near_ties": 0, "sel_mismatch": 0, "max_abs": 0.0}

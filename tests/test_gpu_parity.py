@@ -1,0 +1,320 @@
+"""CUDA path vs the fp64 oracle, through the C ABI (needs a B200).
+
+Bars: selections bit-exact except near ties (oracle margin < 1e-4, counted);
+outputs within max-abs 1e-4 (fp32) / 2e-2 (bf16 I/O, fp32 accumulation);
+node arrays within 1e-5 relative (fp32) / 1 ulp (bf16); rows read equal.
+"staged" runs the oracle's descent over the GPU's stored node arrays (read
+as data), so selection is checked independently of 1-ulp node rounding;
+"free" runs the oracle on its own tree.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from hierarchical_sparse_attention_tree_b200 import RecsaError, RecsaLayer
+from hierarchical_sparse_attention_tree_b200 import recsa as R
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+W_TINY = synth.WORKLOADS["tiny_f32"]
+
+
+def small(**kw):
+    base = dict(name="small", batch=1, n_kv_heads=1, group=4, head_dim=128, branching=8, k=3, length=1000,
+                bf16=True, centroids=16, run_min=16, run_max=64)
+    base.update(kw)
+    return synth.Workload(**base)
+
+
+def make_layer(w, capacity, max_chunk=0):
+    W = synth.workload_pooler(w)
+    return RecsaLayer(w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim, w.branching, w.k, capacity,
+                      parity.to_dev(W, w.bf16), dtype=torch.bfloat16 if w.bf16 else torch.float32,
+                      rope_base=w.rope_base, max_chunk=max_chunk), W
+
+
+def per_seq_queries(w, runs, step, lengths):
+    return np.stack([synth.decode_query(w.seed, b, step, lengths[b], w.n_kv_heads, w.group, w.head_dim, w.centroids,
+                                        w.sigma_noise, runs[b], w.bf16)[0] for b in range(w.batch)])
+
+
+def run_decode(layer, w, q_np):
+    B, H, G, D = w.batch, w.n_kv_heads, w.group, w.head_dim
+    J_cap, _ = layer.tree_shape()
+    q = parity.to_dev(q_np, w.bf16)
+    sel = torch.full((B, H, J_cap, w.k), -7, dtype=torch.int32, device="cuda")
+    rows = torch.zeros((B, H, 2), dtype=torch.int64, device="cuda")
+    out = layer.decode(q, sel_out=sel, rows_out=rows)
+    torch.cuda.synchronize()
+    layer.check()
+    return parity.to_f64(out), sel.cpu().numpy(), rows.cpu().numpy()
+
+
+def check_units(layer, w, K, V, Wp, lengths, q_np, gout, gsel, grows, units=None, staged=True, free=True,
+                free_exact=None):
+    G = w.group
+    tol = 2e-2 if w.bf16 else 1e-4
+    storage = parity.storage_of(w.bf16)
+    reports = {"staged": parity.new_report(), "free": parity.new_report()}
+    units = units or [(b, h) for b in range(w.batch) for h in range(w.n_kv_heads)]
+    for b, h in units:
+        L = lengths[b]
+        J, _ = oracle.levels(L, w.branching)
+        qu = parity.q_unit(q_np, b, h, G)
+        if staged:
+            tK, tV = parity.gpu_tree_unit(layer, b, h, J, L)
+            ref = parity.oracle_query(tK, tV, K, V, b, h, L, qu, w)
+            parity.check_decode(gout, gsel, grows, ref, b, h, G, tol, reports["staged"])
+        if free:
+            tree = oracle.build_tree(K[b, h], V[b, h], L, w.head_dim, w.branching, synth.as_f32(Wp), storage)
+            ref = oracle.query_tree(tree, K[b, h], V[b, h], qu, w.k, G, w.rope_base)
+            rep = reports["free"]
+            before = rep["sel_mismatch"]
+            try:
+                parity.check_decode(gout, gsel, grows, ref, b, h, G, tol, rep)
+            except AssertionError:
+                if free_exact:
+                    raise
+                rep["sel_mismatch"] += 1
+            if free_exact and rep["sel_mismatch"] != before:
+                raise AssertionError(rep)
+    st = reports["staged"]
+    if staged:
+        assert st["sel_mismatch"] == 0, st
+        assert st["checked"] > 0 or st["near_ties"] > 0
+    return reports
+
+
+def check_nodes(layer, w, K, V, Wp, lengths, units=None):
+    """GPU node arrays vs the oracle's, every kept level."""
+    storage = parity.storage_of(w.bf16)
+    J_cap, _ = layer.tree_shape()
+    units = units or [(b, h) for b in range(w.batch) for h in range(w.n_kv_heads)]
+    off = 0
+    for b, h in units:
+        L = lengths[b]
+        if L == 0:
+            continue
+        tree = oracle.Tree(w.head_dim, w.branching, L, storage, J_keep=J_cap).build(K[b, h], V[b, h], L,
+                                                                                     synth.as_f32(Wp))
+        for j in range(1, J_cap + 1):
+            n = -(-L // w.branching ** j)
+            kj, vj, sj = layer.level(j)
+            okk, nk = parity.compare_nodes(parity.to_f64(kj[b, h, :n]), tree.K[j][:n], w.bf16)
+            okv, nv = parity.compare_nodes(parity.to_f64(vj[b, h, :n]), tree.V[j][:n], w.bf16)
+            assert okk and okv, (b, h, j, nk, nv)
+            off += nk + nv
+    return off
+
+
+# ---------------------------------------------------------------- tiny fp32
+
+
+def test_tiny_f32_build_and_decode():
+    """The tiny fp32 workload: L=4096, one KV head, G=4, d=64, b=16, k=4
+    (levels 4096 -> 256 -> 16), 8 decode queries against a fixed cache."""
+    w = W_TINY
+    K, V, runs = synth.cache_arrays(w, w.length)
+    layer, Wp = make_layer(w, w.length)
+    layer.load(parity.to_dev(K, False), parity.to_dev(V, False), [w.length])
+    assert layer.tree_shape()[0] == 2
+    check_nodes(layer, w, K, V, Wp, [w.length])
+    total = parity.new_report()
+    for s in range(w.queries):
+        q = per_seq_queries(w, runs, s, [w.length])
+        gout, gsel, grows = run_decode(layer, w, q)
+        rep = check_units(layer, w, K, V, Wp, [w.length], q, gout, gsel, grows, free_exact=True)
+        for key in ("checked", "near_ties"):
+            total[key] += rep["staged"][key]
+        assert grows[0, 0, 0] <= w.k * w.branching * 3
+    assert total["checked"] >= 6, total
+
+
+# -------------------------------------------------- bf16, several units
+
+
+@pytest.mark.parametrize("D,G", [(128, 4), (64, 2), (128, 1), (64, 8)])
+def test_bf16_ragged_batch(D, G):
+    w = small(batch=3, n_kv_heads=2, group=G, head_dim=D, branching=8, k=3)
+    lengths = [1, 517, 3001]
+    K, V, runs = synth.cache_arrays(w, max(lengths))
+    layer, Wp = make_layer(w, 4096)
+    layer.load(parity.to_dev(K, True), parity.to_dev(V, True), lengths)
+    check_nodes(layer, w, K, V, Wp, lengths)
+    for s in range(3):
+        q = per_seq_queries(w, runs, s, lengths)
+        gout, gsel, grows = run_decode(layer, w, q)
+        check_units(layer, w, K, V, Wp, lengths, q, gout, gsel, grows)
+
+
+def test_f32_d128_matches_free_oracle():
+    w = small(batch=2, n_kv_heads=2, group=4, head_dim=128, branching=16, k=4, bf16=False)
+    lengths = [4100, 700]
+    K, V, runs = synth.cache_arrays(w, max(lengths))
+    layer, Wp = make_layer(w, 8192)
+    layer.load(parity.to_dev(K, False), parity.to_dev(V, False), lengths)
+    check_nodes(layer, w, K, V, Wp, lengths)
+    for s in range(3):
+        q = per_seq_queries(w, runs, s, lengths)
+        gout, gsel, grows = run_decode(layer, w, q)
+        check_units(layer, w, K, V, Wp, lengths, q, gout, gsel, grows, free_exact=True)
+
+
+@pytest.mark.parametrize("L", [1, 2, 7, 8, 9, 63, 64, 65, 511, 512, 513])
+def test_edge_lengths(L):
+    """Single token, exactly b and b^2 tokens, one past (a new level)."""
+    w = small(batch=1, n_kv_heads=1, group=4, head_dim=64, branching=8, k=2, bf16=False)
+    K, V, runs = synth.cache_arrays(w, L)
+    layer, Wp = make_layer(w, 600)
+    layer.load(parity.to_dev(K, False), parity.to_dev(V, False), [L])
+    check_nodes(layer, w, K, V, Wp, [L])
+    q = per_seq_queries(w, runs, 0, [L])
+    gout, gsel, grows = run_decode(layer, w, q)
+    check_units(layer, w, K, V, Wp, [L], q, gout, gsel, grows, free_exact=True)
+
+
+def test_dense_equivalence_on_gpu():
+    """k covering every level keeps everything: the GPU output equals dense
+    causal RoPE attention (the oracle reaches the same case)."""
+    w = small(batch=1, n_kv_heads=2, group=4, head_dim=64, branching=16, k=64, bf16=False)
+    L = 1000
+    K, V, runs = synth.cache_arrays(w, L)
+    layer, Wp = make_layer(w, L)
+    layer.load(parity.to_dev(K, False), parity.to_dev(V, False), [L])
+    q = per_seq_queries(w, runs, 0, [L])
+    gout, gsel, grows = run_decode(layer, w, q)
+    assert (grows[0, :, 1] == L).all()  # every token enters the softmax
+    check_units(layer, w, K, V, Wp, [L], q, gout, gsel, grows, free_exact=True)
+
+
+# ---------------------------------------------------------------- append
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_append_matches_rebuild_bitwise(bf16):
+    """Token-by-token and chunked appends leave exactly the node arrays a
+    fresh build over the same tokens produces."""
+    w = small(batch=2, n_kv_heads=2, group=2, head_dim=64, branching=4, k=2, bf16=bf16)
+    start = [30, 61]
+    plan = [1] * 40 + [7, 1, 64, 3, 1, 16]
+    total = sum(plan)
+    cap = max(start) + total
+    K, V, runs = synth.cache_arrays(w, cap)
+    Kd, Vd = parity.to_dev(K, bf16), parity.to_dev(V, bf16)
+    inc, Wp = make_layer(w, cap)
+    K0, V0 = Kd.clone(), Vd.clone()
+    for b in range(w.batch):  # the cache holds only the first start[b] tokens
+        K0[b, :, start[b]:] = 0
+        V0[b, :, start[b]:] = 0
+    inc.load(K0, V0, start)
+    # the appended tokens come from the generator: sequence b, positions start[b] + ...
+    pos = list(start)
+    for n in plan:
+        kn = torch.stack([Kd[b, :, pos[b]:pos[b] + n] for b in range(w.batch)]).permute(0, 2, 1, 3).contiguous()
+        vn = torch.stack([Vd[b, :, pos[b]:pos[b] + n] for b in range(w.batch)]).permute(0, 2, 1, 3).contiguous()
+        inc.append(kn, vn)
+        pos = [p + n for p in pos]
+        full, _ = make_layer(w, cap)
+        full.load(Kd, Vd, pos)
+        torch.cuda.synchronize()
+        J_cap, rows = inc.tree_shape()
+        for j in range(1, J_cap + 1):
+            for a, b_ in zip(inc.level(j), full.level(j)):
+                for s in range(w.batch):
+                    n_j = -(-pos[s] // w.branching ** j)
+                    assert torch.equal(a[s, :, :n_j], b_[s, :, :n_j]), (n, j, s)
+        full.close()
+    assert inc.lengths() == pos
+    inc.check()
+    for b in range(w.batch):  # the appended rows landed after each sequence's tokens
+        assert torch.equal(inc.k_cache[b, :, :pos[b]], Kd[b, :, :pos[b]])
+        assert torch.equal(inc.v_cache[b, :, :pos[b]], Vd[b, :, :pos[b]])
+    check_nodes(inc, w, K, V, Wp, pos)
+    q = per_seq_queries(w, runs, 0, pos)
+    gout, gsel, grows = run_decode(inc, w, q)
+    check_units(inc, w, K, V, Wp, pos, q, gout, gsel, grows, free_exact=not bf16)
+
+
+def test_capacity_and_argument_errors():
+    w = small(batch=1, n_kv_heads=1, group=4, head_dim=64, branching=4, k=2, bf16=False)
+    K, V, _ = synth.cache_arrays(w, 20)
+    layer, _ = make_layer(w, 20)
+    with pytest.raises(RecsaError) as e:
+        layer.decode(torch.zeros(1, 4, 64, device="cuda"))
+    assert e.value.status == R.ERR_INVALID_ARG  # no tokens yet
+    layer.load(parity.to_dev(K, False), parity.to_dev(V, False), [18])
+    kn = torch.zeros(1, 3, 1, 64, device="cuda")
+    with pytest.raises(RecsaError) as e:
+        layer.append(kn, kn)
+    assert e.value.status == R.ERR_CAPACITY
+    assert layer.lengths() == [18]
+    with pytest.raises(RecsaError) as e:
+        layer.ctx.build_tree([21])
+    assert e.value.status == R.ERR_CAPACITY
+    layer.check()
+
+
+# ------------------------------------------------------- full-size decode
+
+
+def _full_size(name, steps, units):
+    w = synth.WORKLOADS[name]
+    L0 = w.length
+    cap = L0 + steps
+    K, V, runs = synth.cache_arrays(w, cap)
+    layer, Wp = make_layer(w, cap)
+    Kd, Vd = parity.to_dev(K, True), parity.to_dev(V, True)
+    layer.load(Kd, Vd, [L0] * w.batch)
+    check_nodes(layer, w, K, V, Wp, [L0] * w.batch, units=units[:1])
+    lengths = [L0] * w.batch
+    staged, free = parity.new_report(), parity.new_report()
+    for s in range(steps):
+        kn = Kd[:, :, lengths[0]:lengths[0] + 1].permute(0, 2, 1, 3).contiguous()
+        vn = Vd[:, :, lengths[0]:lengths[0] + 1].permute(0, 2, 1, 3).contiguous()
+        layer.append(kn, vn)
+        lengths = [x + 1 for x in lengths]
+        q = per_seq_queries(w, runs, s, lengths)
+        gout, gsel, grows = run_decode(layer, w, q)
+        rep = check_units(layer, w, K, V, Wp, lengths, q, gout, gsel, grows, units=units)
+        for key in ("checked", "near_ties", "sel_mismatch"):
+            staged[key] += rep["staged"][key]
+            free[key] += rep["free"][key]
+    check_nodes(layer, w, K, V, Wp, lengths, units=units[:1])
+    print(f"{name}: staged {staged} free {free}")
+    assert staged["checked"] >= len(units) * steps // 2
+    return staged, free
+
+
+def test_decode_131k_sampled():
+    """Qwen3-4B-shaped layer at L=131072 (b=64, k=16): build, then
+    append + decode steps; sampled KV heads checked against the oracle."""
+    _full_size("decode_131k", 3, [(0, 0), (0, 5)])
+
+
+def test_decode_524k_batch4_sampled():
+    """The 524K, batch-4 decode workload in the benchmark's launch shape."""
+    _full_size("decode_524k_b4", 2, [(0, 0), (1, 3), (3, 7)])
+
+
+# ----------------------------------------------------- dense comparator
+
+
+@pytest.mark.parametrize("dtype,D,G,L", [(torch.bfloat16, 128, 4, 70000), (torch.float32, 64, 2, 999),
+                                         (torch.bfloat16, 64, 8, 5)])
+def test_dense_decode_comparator(dtype, D, G, L):
+    B, H = 2, 3
+    g = torch.Generator(device="cuda").manual_seed(0)
+    Kc = torch.randn(B, H, L + 3, D, device="cuda", generator=g).to(dtype)
+    Vc = torch.randn(B, H, L + 3, D, device="cuda", generator=g).to(dtype)
+    q = torch.randn(B, H * G, D, device="cuda", generator=g).to(dtype)
+    out = torch.empty_like(q)
+    scratch = torch.empty(R.dense_decode_scratch_bytes(B, H * G, D), dtype=torch.uint8, device="cuda")
+    R.dense_decode(Kc, Vc, q, out, L, scratch)
+    qf = q.float().view(B, H, G, D)
+    s = torch.einsum("bhgd,bhtd->bhgt", qf, Kc[:, :, :L].float()) / D ** 0.5
+    ref = torch.einsum("bhgt,bhtd->bhgd", torch.softmax(s, -1), Vc[:, :, :L].float()).reshape(B, H * G, D)
+    tol = 2e-2 if dtype == torch.bfloat16 else 1e-4
+    assert (out.float() - ref).abs().max().item() <= tol

@@ -1,0 +1,61 @@
+"""The C-ABI library loads on a CPU-only host, exports every symbol its
+header declares, and rejects bad arguments on the host before touching a
+device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hierarchical_sparse_attention_tree_b200 import recsa as R
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "recsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(recsa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol():
+    lib = R.lib()
+    names = declared_symbols()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(R.EXPORTS) == names
+
+
+def test_workspace_sizes():
+    cfg = R.make_config(4, 8, 32, 128, 64, 16, 524288 + 512)
+    n = R.workspace_bytes(cfg)
+    # three levels of bf16 keys/values plus fp32 value sums: a few percent of the 8.6 GB cache
+    assert 0.25e9 < n < 0.3e9
+    tiny = R.make_config(1, 1, 4, 64, 16, 4, 4096, dtype=__import__("torch").float32)
+    assert R.workspace_bytes(tiny) > 2 * 256 * 64 * 4
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("head_dim", 96, R.ERR_UNSUPPORTED), ("branching", 1, R.ERR_INVALID_ARG), ("k", 0, R.ERR_INVALID_ARG),
+    ("n_q_heads", 12, R.ERR_INVALID_ARG), ("n_q_heads", 24, R.ERR_UNSUPPORTED), ("capacity", 0, R.ERR_INVALID_ARG),
+    ("rope_base", 1.0, R.ERR_INVALID_ARG), ("k", 65, R.ERR_INVALID_ARG),
+])
+def test_bad_config_rejected(field, value, status):
+    cfg = R.make_config(1, 8, 32, 128, 64, 16, 1024)
+    setattr(cfg, field, value)
+    assert R.lib().recsa_workspace_bytes(ctypes.byref(cfg)) == 0
+    assert R.lib().recsa_last_error()
+    h = ctypes.c_void_p()
+    st = R.lib().recsa_init(ctypes.byref(h), ctypes.byref(cfg), None, None, None, 0, None, None)
+    assert st == status and not h.value
+
+
+def test_null_buffers_rejected():
+    cfg = R.make_config(1, 8, 32, 128, 64, 16, 1024)
+    h = ctypes.c_void_p()
+    assert R.lib().recsa_init(ctypes.byref(h), ctypes.byref(cfg), None, None, None, 0, None, None) == R.ERR_INVALID_ARG
+    assert b"NULL" in R.lib().recsa_last_error()
+    assert R.lib().recsa_build_tree(None, None, None) == R.ERR_INVALID_ARG
+    assert R.lib().recsa_decode(None, None, None, None, None, None) == R.ERR_INVALID_ARG
+    assert R.lib().recsa_dense_decode_scratch_bytes(4, 32, 128) == 4 * 32 * 256 * 130 * 4
