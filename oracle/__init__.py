@@ -55,6 +55,8 @@ def _load():
             lib.orc_round.argtypes = [dbl, i32]
             lib.orc_build.restype = i32
             lib.orc_build.argtypes = [vp, vp, i32, i64, i32, i32, vp, i32, i64, i32, vp, vp]
+            lib.orc_pool_level.restype = i32
+            lib.orc_pool_level.argtypes = [vp, i64, i32, i32, vp, i32, vp]
             lib.orc_query.restype = i32
             lib.orc_query.argtypes = [i32, i32, i32, i32, dbl, i64, vp, vp, vp, vp, i32, vp, vp, i64, vp, vp, vp, vp,
                                       vp]
@@ -78,6 +80,18 @@ def levels(T: int, b: int):
 
 def round_store(x: float, storage: int) -> float:
     return _load().orc_round(x, storage)
+
+
+def pool_level(child_keys, b: int, W, storage: int) -> np.ndarray:
+    """Keys of the level above, pooled from the given child keys (rows as
+    stored): the pooler applied to the mean of each node's children."""
+    ck = np.ascontiguousarray(child_keys, dtype=np.float64)
+    n, d = ck.shape
+    Wf = np.ascontiguousarray(W, dtype=np.float32)
+    out = np.zeros((-(-n // b), d))
+    if _load().orc_pool_level(ck.ctypes.data, n, d, b, Wf.ctypes.data, storage, out.ctypes.data) != 0:
+        raise ValueError("bad arguments")
+    return out
 
 
 def _ptr_array(arrs):

@@ -110,6 +110,16 @@ static long long ipow_sat(int b, int j) {
 
 /* --------------------------------------------------------------- tree */
 
+/* The pooler (R1): y = W x for the mean x of a node's children's keys,
+ * rounded to the storage type. */
+static void pool_mean(const double* mean, int d, const float* W, int storage, double* out) {
+    for (int r = 0; r < d; r++) {
+        double y = 0.0;
+        for (int c = 0; c < d; c++) y += (double)W[r * d + c] * mean[c];
+        out[r] = orc_round(y, storage);
+    }
+}
+
 int orc_build(const void* Ktok, const void* Vtok, int tok_dtype, long long T, int d, int b, const float* W,
               int storage, long long t_from, int J_keep, double* const* Knode, double* const* Vnode) {
     long long n[ORC_MAXLEV + 1];
@@ -138,15 +148,30 @@ int orc_build(const void* Ktok, const void* Vtok, int tok_dtype, long long T, in
                     s += (j == 1) ? tok_at(Ktok, tok_dtype, c * d + i) : Knode[j - 1][c * d + i];
                 mean[i] = s / (double)(c_hi - c_lo);
             }
-            for (int r = 0; r < d; r++) {
-                double y = 0.0;
-                for (int c = 0; c < d; c++) y += (double)W[r * d + c] * mean[c];
-                Knode[j][m * d + r] = orc_round(y, storage);
-            }
+            pool_mean(mean, d, W, storage, Knode[j] + m * d);
         }
     }
     free(mean);
     return Jb;
+}
+
+int orc_pool_level(const double* child_keys, long long n_children, int d, int b, const float* W, int storage,
+                   double* out) {
+    if (n_children < 1 || d < 1 || b < 2) return -1;
+    double* mean = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!mean) return -1;
+    long long n = (n_children + b - 1) / b;
+    for (long long m = 0; m < n; m++) {
+        long long c_lo = m * b, c_hi = (m + 1) * b < n_children ? (m + 1) * b : n_children;
+        for (int i = 0; i < d; i++) {
+            double s = 0.0;
+            for (long long c = c_lo; c < c_hi; c++) s += child_keys[c * d + i];
+            mean[i] = s / (double)(c_hi - c_lo);
+        }
+        pool_mean(mean, d, W, storage, out + m * d);
+    }
+    free(mean);
+    return 0;
 }
 
 /* --------------------------------------------------------------- RoPE */

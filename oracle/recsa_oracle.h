@@ -43,6 +43,12 @@ double orc_round(double x, int storage);
 int orc_build(const void* Ktok, const void* Vtok, int tok_dtype, long long T, int d, int b, const float* W,
               int storage, long long t_from, int J_keep, double* const* Knode, double* const* Vnode);
 
+/* Keys of the level above n_children given child keys (fp64 rows, as
+ * stored): row m = round(W * mean of children [m b, min((m+1) b, n))).
+ * out holds ceil(n_children / b) rows. Returns 0, or -1 on bad arguments. */
+int orc_pool_level(const double* child_keys, long long n_children, int d, int b, const float* W, int storage,
+                   double* out);
+
 /* One query of one unit (a KV head and its G query heads) against the tree
  * over tokens [0, T) (Knode/Vnode levels 1..J(T)) and the level-0 tokens,
  * followed by nloc local tokens (a prefill chunk's own causal tokens; 0 for

@@ -89,24 +89,30 @@ def check_units(layer, w, K, V, Wp, lengths, q_np, gout, gsel, grows, units=None
 
 
 def check_nodes(layer, w, K, V, Wp, lengths, units=None):
-    """GPU node arrays vs the oracle's, every kept level."""
+    """GPU node arrays vs the oracle, every kept level. Values: the oracle's
+    exact subtree means, rounded once. Keys: the oracle's pooler applied to
+    the mean of the children as the GPU stored them (level 1: the tokens), so
+    a 1-ulp rounding difference one level down is not compounded."""
     storage = parity.storage_of(w.bf16)
     J_cap, _ = layer.tree_shape()
     units = units or [(b, h) for b in range(w.batch) for h in range(w.n_kv_heads)]
+    Wf = synth.as_f32(Wp)
     off = 0
     for b, h in units:
         L = lengths[b]
         if L == 0:
             continue
-        tree = oracle.Tree(w.head_dim, w.branching, L, storage, J_keep=J_cap).build(K[b, h], V[b, h], L,
-                                                                                     synth.as_f32(Wp))
+        tree = oracle.Tree(w.head_dim, w.branching, L, storage, J_keep=J_cap).build(K[b, h], V[b, h], L, Wf)
+        below = synth.as_f32(K[b, h, :L]).astype(np.float64)
         for j in range(1, J_cap + 1):
             n = -(-L // w.branching ** j)
             kj, vj, sj = layer.level(j)
-            okk, nk = parity.compare_nodes(parity.to_f64(kj[b, h, :n]), tree.K[j][:n], w.bf16)
+            gk = parity.to_f64(kj[b, h, :n])
+            okk, nk = parity.compare_nodes(gk, oracle.pool_level(below, w.branching, Wf, storage), w.bf16)
             okv, nv = parity.compare_nodes(parity.to_f64(vj[b, h, :n]), tree.V[j][:n], w.bf16)
             assert okk and okv, (b, h, j, nk, nv)
             off += nk + nv
+            below = gk
     return off
 
 

@@ -309,3 +309,16 @@ def test_decode_equals_chunk_form_when_nothing_dropped():
     dec = oracle.query_tree(tree, K, V, q, k=k, G=G, rope_base=1e6)
     pre = oracle.query([None], [None], K[:0], V[:0], 0, q, d, b, k, G, 1e6, Kloc=K, Vloc=V)
     np.testing.assert_allclose(dec["out"], pre["out"], atol=1e-12)
+
+
+def test_pool_level_matches_build():
+    """Pooling a level from given child keys reproduces the build's keys."""
+    T, b, d = 700, 5, 8
+    K, V, W = _rand(34, (T, d)), _rand(35, (T, d)), _rand(36, (d, d))
+    for storage in (F64, oracle.STORE_BF16):
+        tree = oracle.build_tree(K, V, T, d, b, W, storage)
+        J, n = oracle.levels(T, b)
+        np.testing.assert_array_equal(oracle.pool_level(K.astype(np.float64), b, W, storage), tree.K[1][:n[1]])
+        for j in range(2, J + 1):
+            np.testing.assert_array_equal(oracle.pool_level(tree.K[j - 1][:n[j - 1]], b, W, storage),
+                                          tree.K[j][:n[j]])
