@@ -63,7 +63,8 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_kernel(TreeParams p, Decod
     unsigned long long* skey = topbuf + 2 * KMAX;                                  // [my_max]
     long long* par = reinterpret_cast<long long*>(skey + a.my_max);                // [KMAX]
     long long* chosen = par + KMAX;                                                // [KMAX]
-    float* cm = reinterpret_cast<float*>(chosen + KMAX);                           // [G]
+    long long* picked = chosen + KMAX;                                             // [KMAX]
+    float* cm = reinterpret_cast<float*>(picked + KMAX);                           // [G]
     float* cl = cm + G;                                                            // [G]
     float* cacc = cl + G;                                                          // [G][D]
     float* wm = cacc + G * D;                                                      // [W][G]
@@ -247,21 +248,20 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_kernel(TreeParams p, Decod
                     }
                     for (int x = 0; x < nm; x++)
                         if (mine[x] == best) mine[x] = 0;
-                    if (lane == 0) chosen[r] = key_id(best);
+                    if (lane == 0) picked[r] = key_id(best);
                     __syncwarp();
                 }
-                // ascending node order
-                long long id = lane < kk ? chosen[lane] : 0;
-                __syncwarp();
-                if (lane < kk) {
+                // ascending node order (ids are distinct: rank = number of smaller ids)
+                for (int x = lane; x < kk; x += 32) {
+                    const long long id = picked[x];
                     int pos = 0;
-                    for (int r = 0; r < kk; r++) pos += (chosen[r] < id);
-                    __syncwarp(__activemask());
+                    for (int r = 0; r < kk; r++) pos += (picked[r] < id);
                     chosen[pos] = id;
                 }
                 __syncwarp();
-                if (rank == 0 && a.sel_out && lane < p.k) {
-                    a.sel_out[(u * p.J_cap + (j - 1)) * p.k + lane] = lane < kk ? (int)chosen[lane] : -1;
+                if (rank == 0 && a.sel_out) {
+                    for (int x = lane; x < p.k; x += 32)
+                        a.sel_out[(u * p.J_cap + (j - 1)) * p.k + x] = x < kk ? (int)chosen[x] : -1;
                 }
             }
             __syncthreads();
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_kernel(TreeParams p, Decod
 }
 
 size_t decode_smem_bytes(int D, int G, int my_max) {
-    size_t s = 2 * KMAX * 8 + (size_t)my_max * 8 + 2 * KMAX * 8;
+    size_t s = 2 * KMAX * 8 + (size_t)my_max * 8 + 3 * KMAX * 8;
     s += (size_t)(2 * G + G * D + 2 * DEC_WARPS * G + DEC_WARPS * G * D + G * my_max) * 4;
     return s;
 }

@@ -41,11 +41,15 @@ __global__ void __launch_bounds__(DN_THREADS) dense_partial_kernel(const T* __re
     }
     const T* Ku = K + u * ld * D + gl * EPL;
     const T* Vu = V + u * ld * D + gl * EPL;
-    for (long long tb = t0 + grp; tb < t1; tb += (long long)NG * U) {
+    // Warp-uniform loop: every lane of a warp runs the same iterations (the
+    // shuffles below need all 32 lanes); rows past t1 are masked, not skipped.
+    constexpr int NW = DN_THREADS / 32;
+    const int warp = tid >> 5, gi = (tid & 31) / LPR;
+    for (long long base = t0 + (long long)warp * RPW; base < t1; base += (long long)NW * RPW * U) {
         float kr[U][EPL] = {}, vr[U][EPL] = {};
 #pragma unroll
         for (int i = 0; i < U; i++) {
-            const long long t = tb + (long long)i * NG;
+            const long long t = base + gi + (long long)i * NW * RPW;
             if (t < t1) {
                 load_vec<T, EPL>(Ku + t * D, kr[i]);
                 load_vec<T, EPL>(Vu + t * D, vr[i]);
@@ -53,7 +57,7 @@ __global__ void __launch_bounds__(DN_THREADS) dense_partial_kernel(const T* __re
         }
 #pragma unroll
         for (int i = 0; i < U; i++) {
-            const long long t = tb + (long long)i * NG;
+            const long long t = base + gi + (long long)i * NW * RPW;
             float lg[G];
 #pragma unroll
             for (int g = 0; g < G; g++) {

@@ -104,12 +104,15 @@ def check_nodes(layer, w, K, V, Wp, lengths, units=None):
             continue
         tree = oracle.Tree(w.head_dim, w.branching, L, storage, J_keep=J_cap).build(K[b, h], V[b, h], L, Wf)
         below = synth.as_f32(K[b, h, :L]).astype(np.float64)
+        vtok = synth.as_f32(V[b, h, :L])
         for j in range(1, J_cap + 1):
             n = -(-L // w.branching ** j)
             kj, vj, sj = layer.level(j)
             gk = parity.to_f64(kj[b, h, :n])
-            okk, nk = parity.compare_nodes(gk, oracle.pool_level(below, w.branching, Wf, storage), w.bf16)
-            okv, nv = parity.compare_nodes(parity.to_f64(vj[b, h, :n]), tree.V[j][:n], w.bf16)
+            okk, nk = parity.compare_nodes(gk, oracle.pool_level(below, w.branching, Wf, storage), w.bf16,
+                                           atol=parity.pooled_key_bound(below, w.branching, Wf))
+            okv, nv = parity.compare_nodes(parity.to_f64(vj[b, h, :n]), tree.V[j][:n], w.bf16,
+                                           atol=parity.mean_value_bound(vtok, w.branching ** j))
             assert okk and okv, (b, h, j, nk, nv)
             off += nk + nv
             below = gk
