@@ -21,7 +21,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -49,6 +48,7 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU-baseline sample")
+    ap.add_argument("--settle-s", type=float, default=0.3, help="decode-only launches before timing (clock sampling)")
     return ap.parse_args()
 
 
@@ -80,55 +80,51 @@ def kernel_traffic(kernel: str):
 
 
 class ClockSampler:
-    """nvidia-smi samples every 200 ms while the timed region runs."""
+    """Polls NVML every 10 ms (SM clock, max SM clock, throttle reasons) from
+    a thread while the timed region runs."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, device_index: int):
-        self.lines = []
-        self.proc = None
+        self.sm, self.reasons, self.max_sm = [], set(), None
+        self.stop_flag = threading.Event()
+        self.err = None
         try:
-            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
-            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except Exception:
-            self.proc = None
+            import pynvml
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.nv = pynvml
+            self.max_sm = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+        except Exception as e:  # no NVML: report why
+            self.err = str(e)
+            self.t = None
+
+    def _poll(self):
+        while not self.stop_flag.is_set():
+            try:
+                self.sm.append(float(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception as e:
+                self.err = str(e)
+                return
+            time.sleep(0.01)
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
+        if self.t is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        self.stop_flag.set()
         self.t.join(timeout=2)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.sm) if self.sm else None, "sm_max_mhz": self.max_sm,
+                "reasons": sorted(self.reasons), "samples": len(self.sm)}
 
 
 def dist_setup(n_gpus: int):
@@ -320,9 +316,16 @@ def main():
         s_idx += 1
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_)]
     torch.cuda.synchronize(dev)
+    # clock sampling starts with ~0.3 s of decode-only launches (the tree is not
+    # changed), so the samples see this load; then the timed region
+    clocks = ClockSampler(dev.index)
+    t_settle = time.perf_counter()
+    while time.perf_counter() - t_settle < args.settle_s:
+        for _ in range(32):
+            layer.decode(q_d[s_idx], out)
+        torch.cuda.synchronize(dev)
     barrier(world, local)
     torch.cuda.synchronize(dev)
-    clocks = ClockSampler(dev.index)
     t_wall = time.perf_counter()
     for i in range(K_):
         flush.fill_(float(s_idx))

@@ -49,5 +49,6 @@ WORKLOADS = {
     "decode_524k_b4": Workload(name="decode_524k_b4", batch=4, length=524288, decode_steps=256, **_QWEN),
     "prefill_131k": Workload(name="prefill_131k", batch=1, length=131072, chunk=4096, **_QWEN),
     "decode_2m": Workload(name="decode_2m", batch=1, length=2097152, decode_steps=128, **_QWEN),
+    "decode_524k_b1": Workload(name="decode_524k_b1", batch=1, length=524288, decode_steps=256, **_QWEN),
     "prefill_524k": Workload(name="prefill_524k", batch=1, length=524288, chunk=4096, **_QWEN),
 }
