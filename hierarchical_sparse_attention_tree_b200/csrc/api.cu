@@ -23,9 +23,11 @@ cudaError_t launch_bump_lengths(const TreeParams&, long long, cudaStream_t);
 template <typename T, int D, int G>
 cudaError_t launch_decode(const TreeParams&, const void*, void*, int*, long long*, cudaStream_t);
 template <typename T, int D, int G>
-cudaError_t launch_dense(const void*, const void*, const void*, void*, int, long long, long long, float*,
+cudaError_t launch_dense(const void*, const void*, const void*, void*, int, long long, long long, float*, int,
                          cudaStream_t);
 int dense_splits(long long units, long long L);
+size_t dense_static_scratch_bytes();
+cudaError_t dense_static_scratch(float** out);
 }  // namespace recsa
 
 using namespace recsa;
@@ -384,8 +386,39 @@ recsa_status recsa_dense_decode(const void* k_cache, const void* v_cache, const 
     const int units = batch * n_kv_heads;
     DISPATCH_TD(dtype, head_dim,
                 DISPATCH_G(G, e = launch_dense<T, DD, GG>(k_cache, v_cache, q, out, units, length, l_stride,
-                                                         static_cast<float*>(scratch), s)));
+                                                         static_cast<float*>(scratch), 256, s)));
     if (e != cudaSuccess) return cuda_fail(e, "recsa_dense_decode");
+    return RECSA_OK;
+}
+
+recsa_status recsa_dense_decode_static(const void* k_cache, const void* v_cache, const void* q, void* out, int batch,
+                                       int n_kv_heads, int n_q_heads, int head_dim, long long length,
+                                       long long l_stride, recsa_dtype dtype, recsa_stream_t stream) {
+    if (!k_cache || !v_cache || !q || !out) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    if (batch < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return fail(RECSA_ERR_INVALID_ARG, "bad head counts");
+    int G = n_q_heads / n_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return fail(RECSA_ERR_UNSUPPORTED, "group size %d", G);
+    if (head_dim != 64 && head_dim != 128) return fail(RECSA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+    if (dtype != RECSA_F32 && dtype != RECSA_BF16) return fail(RECSA_ERR_INVALID_ARG, "unknown dtype");
+    if (length < 1 || l_stride < length) return fail(RECSA_ERR_INVALID_ARG, "bad length / stride");
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 16))
+        return fail(RECSA_ERR_INVALID_ARG, "buffers not 16-byte aligned");
+    const int units = batch * n_kv_heads;
+    const size_t per_split = (size_t)units * G * (head_dim + 2) * sizeof(float);
+    const size_t limit = dense_static_scratch_bytes();
+    if (per_split > limit)
+        return fail(RECSA_ERR_CAPACITY,
+                    "batch * n_q_heads = %d needs %zu bytes of scratch per split; the fixed scratch holds %zu bytes",
+                    batch * n_q_heads, per_split, limit);
+    const int max_splits = (int)(limit / per_split);
+    float* scratch = nullptr;
+    cudaError_t e = dense_static_scratch(&scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_dense_decode_static: scratch address");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    DISPATCH_TD(dtype, head_dim,
+                DISPATCH_G(G, e = launch_dense<T, DD, GG>(k_cache, v_cache, q, out, units, length, l_stride, scratch,
+                                                         max_splits < 256 ? max_splits : 256, s)));
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_dense_decode_static");
     return RECSA_OK;
 }
 

@@ -6,6 +6,8 @@
 // Split-KV: CTA (s, u) streams tokens [s*chunk, (s+1)*chunk) of unit u with
 // 16-byte loads, keeps an online softmax per row group, and writes a partial
 // (max, sum, acc) that a second kernel merges.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace recsa {
@@ -137,10 +139,41 @@ int dense_splits(long long units, long long L) {
     return (int)(s < 1 ? 1 : s);
 }
 
+// Fixed-size device scratch for recsa_dense_decode_static: 8 MiB, held by
+// every device that loads the library until the process exits. Host code
+// must not pass the symbol itself to a kernel (on the host it names a
+// stand-in, not device memory); dense_static_scratch() looks up its device
+// address once per device.
+constexpr size_t DN_STATIC_BYTES = size_t(8) << 20;
+static __device__ __align__(256) float g_dense_static_scratch[DN_STATIC_BYTES / sizeof(float)];
+
+size_t dense_static_scratch_bytes() { return DN_STATIC_BYTES; }
+
+cudaError_t dense_static_scratch(float** out) {
+    static std::mutex mu;
+    static void* addr[256] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_dense_static_scratch);  // with `dev` current
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *out = static_cast<float*>(addr[dev]);
+    return cudaSuccess;
+}
+
+// max_splits bounds the split count so the partials fit the scratch given.
 template <typename T, int D, int G>
 cudaError_t launch_dense(const void* K, const void* V, const void* q, void* out, int units, long long L, long long ld,
-                         float* scratch, cudaStream_t st) {
-    const int splits = dense_splits(units, L);
+                         float* scratch, int max_splits, cudaStream_t st) {
+    int splits = dense_splits(units, L);
+    if (splits > max_splits) splits = max_splits;
+    if (splits < 1) return cudaErrorInvalidValue;
     dim3 grid(splits, units);
     dense_partial_kernel<T, D, G><<<grid, DN_THREADS, 0, st>>>(
         reinterpret_cast<const T*>(K), reinterpret_cast<const T*>(V), reinterpret_cast<const T*>(q), scratch, L, ld,
@@ -153,7 +186,7 @@ cudaError_t launch_dense(const void* K, const void* V, const void* q, void* out,
 
 #define RECSA_INST_DN(T, D, G)                                                                                   \
     template cudaError_t launch_dense<T, D, G>(const void*, const void*, const void*, void*, int, long long,     \
-                                               long long, float*, cudaStream_t);
+                                               long long, float*, int, cudaStream_t);
 #define RECSA_INST_DN_G(T, D) RECSA_INST_DN(T, D, 1) RECSA_INST_DN(T, D, 2) RECSA_INST_DN(T, D, 4) RECSA_INST_DN(T, D, 8)
 RECSA_INST_DN_G(float, 64)
 RECSA_INST_DN_G(float, 128)

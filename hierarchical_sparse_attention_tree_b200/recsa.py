@@ -22,7 +22,7 @@ EXPORTS = [
     "recsa_workspace_bytes", "recsa_init", "recsa_build_tree", "recsa_append", "recsa_decode",
     "recsa_prefill_scratch_bytes", "recsa_prefill", "recsa_get_lengths", "recsa_tree_shape", "recsa_level_arrays",
     "recsa_check_device", "recsa_last_error", "recsa_destroy", "recsa_dense_decode_scratch_bytes",
-    "recsa_dense_decode",
+    "recsa_dense_decode", "recsa_dense_decode_static",
 ]
 
 
@@ -67,6 +67,7 @@ def lib():
             "recsa_destroy": (None, [vp]),
             "recsa_dense_decode_scratch_bytes": (sz, [i32, i32, i32]),
             "recsa_dense_decode": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i64, i64, i32, vp, sz, vp]),
+            "recsa_dense_decode_static": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i64, i64, i32, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -207,3 +208,12 @@ def dense_decode(k_cache, v_cache, q, out, length, scratch, stream=None):
     _check(lib().recsa_dense_decode(_ptr(k_cache), _ptr(v_cache), _ptr(q), _ptr(out), B, H, Hq, D, length, Ls,
                                     dtype_code(k_cache.dtype), _ptr(scratch),
                                     scratch.numel() * scratch.element_size(), _stream(stream)))
+
+
+def dense_decode_static(k_cache, v_cache, q, out, length, stream=None):
+    """recsa_dense_decode without a scratch argument: for callers that cannot
+    allocate device memory (the library's fixed 8 MiB device array is used)."""
+    B, H, Ls, D = k_cache.shape
+    Hq = q.shape[1]
+    _check(lib().recsa_dense_decode_static(_ptr(k_cache), _ptr(v_cache), _ptr(q), _ptr(out), B, H, Hq, D, length, Ls,
+                                           dtype_code(k_cache.dtype), _stream(stream)))

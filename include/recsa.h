@@ -25,8 +25,10 @@
  *
  * Memory. The caller owns all device memory: the KV cache, the workspace
  * (tree levels, running sums, RoPE table, pooler copy, lengths) and every
- * input and output buffer. The library never allocates device memory and
- * never synchronises the device except in recsa_check_device.
+ * input and output buffer. The library makes no allocation call and never
+ * synchronises the device except in recsa_check_device. The one piece of
+ * device memory it owns is a fixed 8 MiB array used only by
+ * recsa_dense_decode_static (see there).
  *
  * Layouts (row-major, element type = config.dtype unless stated):
  *   cache      K, V [B][H_kv][capacity][d]   keys stored before RoPE
@@ -149,6 +151,26 @@ size_t recsa_dense_decode_scratch_bytes(int batch, int n_q_heads, int head_dim);
 recsa_status recsa_dense_decode(const void* k_cache, const void* v_cache, const void* q, void* out, int batch,
                                 int n_kv_heads, int n_q_heads, int head_dim, long long length, long long l_stride,
                                 recsa_dtype dtype, void* scratch, size_t scratch_bytes, recsa_stream_t stream);
+
+/* The dense comparator above, for callers that cannot allocate device
+ * memory: they hold only their input and output buffers (for example a
+ * plugin whose host application owns all device memory, or a path where
+ * allocation is forbidden after start-up), so they cannot provide `scratch`.
+ * The paper has no counterpart; this is a property of the library.
+ * Instead of a caller buffer, the partial results go to a fixed 8 MiB array
+ * in device memory that every GPU which loads the library holds until the
+ * process exits. Same arguments and results as recsa_dense_decode, minus the
+ * scratch; nothing is allocated and nothing needs clearing (every partial is
+ * written before it is read). Limit: batch * n_q_heads * (head_dim + 2) * 4
+ * bytes must fit in 8 MiB (batch * n_q_heads <= 16131 at head_dim 128);
+ * larger calls return RECSA_ERR_CAPACITY and launch nothing; the split count
+ * shrinks to fit. The first call on each device looks up the array's device
+ * address (with that device current), so make it before any stream capture.
+ * All calls share the one array: calls whose kernels overlap on a device
+ * (for example on two streams) race and corrupt each other's results. */
+recsa_status recsa_dense_decode_static(const void* k_cache, const void* v_cache, const void* q, void* out, int batch,
+                                       int n_kv_heads, int n_q_heads, int head_dim, long long length,
+                                       long long l_stride, recsa_dtype dtype, recsa_stream_t stream);
 
 #ifdef __cplusplus
 }
