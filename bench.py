@@ -253,7 +253,7 @@ def main():
     B, H, Hq, D = w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim
     L0 = w.length
     W_, K_ = args.warmup, args.steps
-    n_total = 2 * (W_ + K_) + 1
+    n_total = 2 * (W_ + K_) + 9
     cap = L0 + n_total
     seq_off = rank * B
     bf = torch.bfloat16
@@ -298,23 +298,23 @@ def main():
         nprev = -(-L0 // w.branching ** (j - 1))
         build_bytes += B * H * (nprev * D * (es + 4) + nj * D * (2 * es + 4))
 
-    # ---- device-resident decode steps: warm-up, then K timed steps
-    def step(s, ev=None, rows_slot=None):
+    # ---- device-resident decode steps: warm-up, then K timed steps. One
+    # step = append one token per sequence + one decode query per sequence,
+    # bracketed by two events (the decode may overlap the append's tail).
+    def step(s, ev=None):
         if ev is not None:
             ev[0].record(stream)
         layer.append(kn_d[s], vn_d[s])
+        layer.decode(q_d[s], out)
         if ev is not None:
             ev[1].record(stream)
-        layer.decode(q_d[s], out, rows_out=rows_slot)
-        if ev is not None:
-            ev[2].record(stream)
 
     s_idx = 0
     for _ in range(W_):
         flush.fill_(float(s_idx))
         step(s_idx)
         s_idx += 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_)]
     torch.cuda.synchronize(dev)
     # clock sampling starts with ~0.3 s of decode-only launches (the tree is not
     # changed), so the samples see this load; then the timed region
@@ -329,7 +329,7 @@ def main():
     t_wall = time.perf_counter()
     for i in range(K_):
         flush.fill_(float(s_idx))
-        step(s_idx, evs[i], rows[i])
+        step(s_idx, evs[i])
         s_idx += 1
     torch.cuda.synchronize(dev)
     wall_s = time.perf_counter() - t_wall
@@ -337,11 +337,31 @@ def main():
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
     layer.check()
-    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
-    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    app_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     total_s = max_over_ranks(sum(step_ms) / 1e3, world)
     value = world * B * K_ / total_s
+
+    # ---- the decode kernel alone (roofline): K launches on the current tree,
+    # L2 flushed before each, events around each launch on its stream
+    dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_)]
+    for i in range(K_):
+        flush.fill_(3.0)
+        dev_ev[i][0].record(stream)
+        layer.decode(q_d[i % n_total], out, rows_out=rows[i])
+        dev_ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    layer.check()
+    dec_ms = [e[0].elapsed_time(e[1]) for e in dev_ev]
+    # append alone, for the record (appends K more tokens)
+    app_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(8)]
+    for i in range(8):
+        flush.fill_(4.0)
+        app_ev[i][0].record(stream)
+        layer.append(kn_d[s_idx], vn_d[s_idx])
+        app_ev[i][1].record(stream)
+        s_idx += 1
+    torch.cuda.synchronize(dev)
+    app_ms = [e[0].elapsed_time(e[1]) for e in app_ev]
 
     rows_np = rows.cpu().numpy()
     dec_bytes = int(rows_np.sum()) * D * es + K_ * 2 * B * Hq * D * es  # gathered K/V rows + q + out
@@ -437,7 +457,7 @@ def main():
                          "unit": "GB/s", "frac": achieved / hbm, "peak_source": peak_src,
                          "traffic": kernel_traffic("decode_kernel"),
                          "algorithmic_bytes_per_launch": dec_bytes_per_launch, "launch_ms": dec_avg_s * 1e3},
-            "append_ms": sum(app_ms) / K_, "decode_ms": sum(dec_ms) / K_,
+            "append_ms": sum(app_ms) / len(app_ms), "decode_ms": sum(dec_ms) / K_,
             "rows_per_query": {"k_rows": float(rows_np[..., 0].mean()), "v_rows": float(rows_np[..., 1].mean())},
             "build_tree": {"ms": build_ms, "gbs": build_bytes / (build_ms / 1e3) / 1e9,
                            "frac_hbm": build_bytes / (build_ms / 1e3) / 1e9 / hbm},

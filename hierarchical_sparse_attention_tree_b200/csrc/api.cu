@@ -91,7 +91,7 @@ recsa_status check_config(const recsa_config* c) {
     if (c->branching < 2 || c->branching > 256) return fail(RECSA_ERR_INVALID_ARG, "branching must be in [2, 256]");
     if (c->k < 1 || c->k > 64) return fail(RECSA_ERR_INVALID_ARG, "k must be in [1, 64]");
     if ((long long)c->k * c->branching > 4096) return fail(RECSA_ERR_INVALID_ARG, "k * branching must be <= 4096");
-    if (c->capacity < 1 || c->capacity > (1LL << 31)) return fail(RECSA_ERR_INVALID_ARG, "capacity out of range");
+    if (c->capacity < 1 || c->capacity >= (1LL << 31)) return fail(RECSA_ERR_INVALID_ARG, "capacity out of range");
     if (c->max_chunk < 0 || c->max_chunk > 65536) return fail(RECSA_ERR_INVALID_ARG, "max_chunk out of range");
     if (!(c->rope_base > 1.0)) return fail(RECSA_ERR_INVALID_ARG, "rope_base must be > 1");
     if (c->dtype != RECSA_F32 && c->dtype != RECSA_BF16) return fail(RECSA_ERR_INVALID_ARG, "unknown dtype");
@@ -124,8 +124,8 @@ Layout layout_for(const recsa_config* c) {
         l.off_PK[j] = o; o = align256(o + units * D * 4);
         l.off_PV[j] = o; o = align256(o + units * D * 4);
     }
-    l.off_Wt = o; o = align256(o + D * D * 4);
-    l.off_rope = o; o = align256(o + (size_t)l.npos * (D / 2) * 8);
+    l.off_Wt = o; o = align256(o + D * D * es);
+    l.off_rope = o; o = align256(o + (size_t)l.npos * 3 * (D / 2) * 4);
     l.off_len = o; o = align256(o + units * 8);
     l.off_err = o; o = align256(o + 4);
     l.off_stage = o; o = align256(o + (size_t)c->batch * 8);
@@ -133,13 +133,15 @@ Layout layout_for(const recsa_config* c) {
     return l;
 }
 
-__global__ void pooler_transpose_kernel(const void* w, int bf16, int D, float* wt) {
+// Wt[c][r] = W[r][c], same element type (a copy, no rounding).
+__global__ void pooler_transpose_kernel(const void* w, int bf16, int D, void* wt) {
     int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= D * D) return;
     int r = i / D, c = i % D;
-    float x = bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(w)[i])
-                   : reinterpret_cast<const float*>(w)[i];
-    wt[c * D + r] = x;
+    if (bf16)
+        reinterpret_cast<__nv_bfloat16*>(wt)[c * D + r] = reinterpret_cast<const __nv_bfloat16*>(w)[i];
+    else
+        reinterpret_cast<float*>(wt)[c * D + r] = reinterpret_cast<const float*>(w)[i];
 }
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
@@ -212,27 +214,32 @@ recsa_status recsa_init(recsa_ctx** out, const recsa_config* cfg, void* k_cache,
         p.PK[j] = reinterpret_cast<float*>(ws + l.off_PK[j]);
         p.PV[j] = reinterpret_cast<float*>(ws + l.off_PV[j]);
     }
-    p.Wt = reinterpret_cast<float*>(ws + l.off_Wt);
-    p.rope = reinterpret_cast<float2*>(ws + l.off_rope);
+    p.Wt = ws + l.off_Wt;
+    p.rope = reinterpret_cast<float*>(ws + l.off_rope);
     p.len = reinterpret_cast<long long*>(ws + l.off_len);
     p.err = reinterpret_cast<int*>(ws + l.off_err);
     p.scale = (float)(1.0 / std::sqrt((double)D));
     c->len_stage = reinterpret_cast<long long*>(ws + l.off_stage);
 
-    // RoPE table, fp64 on the host: (cos, sin)(pos * base^(-2i/d))
-    std::vector<float2> tab((size_t)l.npos * (D / 2));
+    // RoPE table, fp64 on the host: row pos = [cos | sin | -sin](pos * base^(-2i/d)), i < d/2
+    const int HD = D / 2;
+    std::vector<float> tab((size_t)l.npos * 3 * HD);
     for (int pos = 0; pos < l.npos; pos++)
-        for (int i = 0; i < D / 2; i++) {
-            double th = std::pow(cfg->rope_base, -2.0 * i / D);
-            tab[(size_t)pos * (D / 2) + i] = make_float2((float)std::cos(pos * th), (float)std::sin(pos * th));
+        for (int i = 0; i < HD; i++) {
+            const double th = std::pow(cfg->rope_base, -2.0 * i / D);
+            const float c = (float)std::cos(pos * th), sn = (float)std::sin(pos * th);
+            float* row = tab.data() + (size_t)pos * 3 * HD;
+            row[i] = c;
+            row[HD + i] = sn;
+            row[2 * HD + i] = -sn;
         }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync((void*)p.rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice, s);
+    cudaError_t e = cudaMemcpyAsync((void*)p.rope, tab.data(), tab.size() * sizeof(float), cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(p.len, 0, (size_t)p.B * p.H * 8, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(p.err, 0, 4, s);
     if (e == cudaSuccess) {
         pooler_transpose_kernel<<<(D * D + 255) / 256, 256, 0, s>>>(pooler_w, cfg->dtype == RECSA_BF16, D,
-                                                                     const_cast<float*>(p.Wt));
+                                                                     const_cast<void*>(p.Wt));
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) {

@@ -29,8 +29,8 @@ struct TreeParams {
     float* VS[MAXJ + 1];       // fp32 value sums [B*H][rows[j]][D] (j >= 1)
     float* PK[MAXJ + 1];       // right-edge key prefix sums [B*H][D] (j >= 1)
     float* PV[MAXJ + 1];       // right-edge value prefix sums [B*H][D] (j >= 1)
-    const float* Wt;           // pooler, transposed: Wt[c * D + r] = W[r][c]
-    const float2* rope;        // [npos][D/2] = (cos, sin)(p * theta_i)
+    const void* Wt;            // pooler, transposed, storage type: Wt[c * D + r] = W[r][c]
+    const float* rope;         // [npos][3][D/2]: cos, sin, -sin of (p * theta_i), theta_i = base^(-2i/d)
     long long* len;            // [B*H] tokens held by each unit
     int* err;                  // device error word
     float scale;               // 1 / sqrt(D)
@@ -123,5 +123,166 @@ __device__ __forceinline__ int top_level(const TreeParams& p, long long L) {
 }
 
 __device__ __forceinline__ void flag_error(int* err, int bits) { atomicOr(err, bits); }
+
+}  // namespace recsa
+
+// ---------------------------------------------------------------------
+// mbarrier + 1D bulk async copy (global -> this CTA's shared memory).
+// PTX ISA: mbarrier.*, cp.async.bulk.shared::cluster.global.mbarrier::
+// complete_tx::bytes. Addresses 16-byte aligned, sizes multiples of 16.
+
+namespace recsa {
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Arrive once and add `bytes` to the transaction count of the current phase.
+// Relaxed: the barrier only counts the copy's bytes; it orders none of this
+// thread's earlier memory operations (so it does not wait for them).
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.relaxed.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for phase `parity` of `bar` to complete, for at most ~2^31 clock
+// cycles (about a second). Returns false on timeout (the caller flags an
+// error and carries on without using the data; it never exits early, so
+// cluster barriers stay balanced).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > (1LL << 31)) return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+}  // namespace recsa
+
+namespace recsa {
+
+// Orders this thread's earlier generic-proxy accesses to shared memory before
+// later async-proxy (bulk copy) writes to it.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// The two halves of this lane's PPL rotation pairs, (x_i, x_{i+D/2}) for
+// i = lane*PPL + e, as floats.
+template <typename T, int PPL, int HD>
+__device__ __forceinline__ void load_pairs(const T* row, int lane, float* a, float* b);
+
+template <>
+__device__ __forceinline__ void load_pairs<__nv_bfloat16, 2, 64>(const __nv_bfloat16* row, int lane, float* a,
+                                                                  float* b) {
+    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(row + lane * 2);
+    const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(row + 64 + lane * 2);
+    a[0] = __low2float(x); a[1] = __high2float(x);
+    b[0] = __low2float(y); b[1] = __high2float(y);
+}
+template <>
+__device__ __forceinline__ void load_pairs<__nv_bfloat16, 1, 32>(const __nv_bfloat16* row, int lane, float* a,
+                                                                  float* b) {
+    a[0] = __bfloat162float(row[lane]);
+    b[0] = __bfloat162float(row[32 + lane]);
+}
+template <>
+__device__ __forceinline__ void load_pairs<float, 2, 64>(const float* row, int lane, float* a, float* b) {
+    const float2 x = *reinterpret_cast<const float2*>(row + lane * 2);
+    const float2 y = *reinterpret_cast<const float2*>(row + 64 + lane * 2);
+    a[0] = x.x; a[1] = x.y;
+    b[0] = y.x; b[1] = y.y;
+}
+template <>
+__device__ __forceinline__ void load_pairs<float, 1, 32>(const float* row, int lane, float* a, float* b) {
+    a[0] = row[lane];
+    b[0] = row[32 + lane];
+}
+
+
+}  // namespace recsa
+
+
+namespace recsa {
+
+
+// Elements [i0, i0 + N) and [HD + i0, HD + i0 + N) of a row, as floats
+// (N = 4 or 8; 8- or 16-byte aligned vector loads).
+template <typename T, int N>
+__device__ __forceinline__ void load_half_rows(const T* row, int i0, int HD, float* a, float* b) {
+    load_vec<T, N>(row + i0, a);
+    load_vec<T, N>(row + HD + i0, b);
+}
+
+}  // namespace recsa
+
+namespace recsa {
+
+// Packed fp32 arithmetic (two independent IEEE fp32 operations per
+// instruction, round to nearest even): same results as two fmaf / fmul.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(*reinterpret_cast<unsigned long long*>(&d))
+        : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)),
+          "l"(*reinterpret_cast<unsigned long long*>(&c)));
+    return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;"
+        : "=l"(*reinterpret_cast<unsigned long long*>(&d))
+        : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)));
+    return d;
+}
+
+// N consecutive floats of a RoPE table block (16-byte loads), as float2 pairs.
+template <int N>
+__device__ __forceinline__ void load_tab2(const float* p, float2* out) {
+#pragma unroll
+    for (int x = 0; x < N / 4; x++) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(p) + x);
+        out[2 * x] = make_float2(v.x, v.y);
+        out[2 * x + 1] = make_float2(v.z, v.w);
+    }
+}
+
+// N consecutive elements of a row as float2 pairs (N = 4 or 8).
+template <typename T, int N>
+__device__ __forceinline__ void load_row2(const T* row, float2* out) {
+    float f[N];
+    load_vec<T, N>(row, f);
+#pragma unroll
+    for (int x = 0; x < N / 2; x++) out[x] = make_float2(f[2 * x], f[2 * x + 1]);
+}
 
 }  // namespace recsa
