@@ -71,7 +71,7 @@ def kernel_traffic(kernel: str):
     try:
         with open(path) as f:
             d = json.load(f)[kernel]
-        src = open(os.path.join(ROOT, d["source"]), "rb").read()
+        src = b"".join(open(os.path.join(ROOT, f), "rb").read() for f in d["sources"])
         if hashlib.sha256(src).hexdigest()[:16] != d["source_sha"]:
             return None
         return d["bytes_per_launch"]
