@@ -26,6 +26,13 @@ template <typename T, int D, int G>
 cudaError_t launch_dense(const void*, const void*, const void*, void*, int, long long, long long, float*, int,
                          cudaStream_t);
 int dense_splits(long long units, long long L);
+template <int D>
+cudaError_t launch_prefill_local(const TreeParams&, const void*, const void*, const void*, float*, int, int, int, int,
+                                 cudaStream_t);
+template <typename T, int D, int G>
+cudaError_t launch_prefill_tree(const TreeParams&, const void*, void*, const float*, int*, int, int, int,
+                                cudaStream_t);
+size_t prefill_tree_smem_bytes(int D, int G, int elem, int k, int b);
 size_t dense_static_scratch_bytes();
 cudaError_t dense_static_scratch(float** out);
 }  // namespace recsa
@@ -322,15 +329,48 @@ recsa_status recsa_decode(recsa_ctx* ctx, const void* q, void* out, int* sel_out
 }
 
 size_t recsa_prefill_scratch_bytes(const recsa_config* cfg, int C) {
-    (void)cfg; (void)C;
-    return 0;
+    if (check_config(cfg) != RECSA_OK || C < 1) return 0;
+    return (size_t)cfg->batch * C * cfg->n_q_heads * (cfg->head_dim + 2) * sizeof(float);
 }
 
 recsa_status recsa_prefill(recsa_ctx* ctx, const void* q, const void* k, const void* v, int C, void* out,
                            int* sel_out, void* scratch, size_t scratch_bytes, recsa_stream_t stream) {
-    (void)ctx; (void)q; (void)k; (void)v; (void)C; (void)out; (void)sel_out; (void)scratch; (void)scratch_bytes;
-    (void)stream;
-    return fail(RECSA_ERR_UNSUPPORTED, "prefill is not built yet");
+    if (!ctx || !q || !k || !v || !out || !scratch) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    const recsa_config& c = ctx->cfg;
+    if (c.dtype != RECSA_BF16) return fail(RECSA_ERR_UNSUPPORTED, "prefill is built for bf16 storage only");
+    if (C < 1 || C > c.max_chunk) return fail(RECSA_ERR_INVALID_ARG, "chunk %d outside [1, max_chunk=%d]", C, c.max_chunk);
+    for (int b = 0; b < c.batch; b++)
+        if (ctx->len[b] + C > c.capacity)
+            return fail(RECSA_ERR_CAPACITY, "sequence %d: %lld + %d tokens exceed capacity %lld", b, ctx->len[b], C,
+                        c.capacity);
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+        return fail(RECSA_ERR_INVALID_ARG, "q/k/v/out not 16-byte aligned");
+    if (!aligned(scratch, 256)) return fail(RECSA_ERR_INVALID_ARG, "scratch not 256-byte aligned");
+    const size_t need = recsa_prefill_scratch_bytes(&c, C);
+    if (scratch_bytes < need) return fail(RECSA_ERR_CAPACITY, "scratch has %zu bytes, needs %zu", scratch_bytes, need);
+    if (prefill_tree_smem_bytes(c.head_dim, ctx->G, 2, c.k, c.branching) > 227 * 1024)
+        return fail(RECSA_ERR_UNSUPPORTED, "k * branching too large for the prefill kernel's shared memory");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float* state = static_cast<float*>(scratch);
+    cudaError_t e;
+    if (c.head_dim == 64)
+        e = launch_prefill_local<64>(ctx->p, q, k, v, state, c.batch, C, c.n_q_heads, c.n_kv_heads, s);
+    else
+        e = launch_prefill_local<128>(ctx->p, q, k, v, state, c.batch, C, c.n_q_heads, c.n_kv_heads, s);
+    if (e == cudaSuccess) {
+        using T = __nv_bfloat16;
+        if (c.head_dim == 64) {
+            constexpr int DD = 64;
+            DISPATCH_G(ctx->G, e = launch_prefill_tree<T, DD, GG>(ctx->p, q, out, state, sel_out, c.batch, C,
+                                                                  c.n_q_heads, s));
+        } else {
+            constexpr int DD = 128;
+            DISPATCH_G(ctx->G, e = launch_prefill_tree<T, DD, GG>(ctx->p, q, out, state, sel_out, c.batch, C,
+                                                                  c.n_q_heads, s));
+        }
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_prefill");
+    return RECSA_OK;
 }
 
 recsa_status recsa_get_lengths(const recsa_ctx* ctx, long long* lengths) {

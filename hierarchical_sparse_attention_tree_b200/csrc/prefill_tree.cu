@@ -1,0 +1,482 @@
+// Prefill, tree part: one CTA per (chunk token, KV head).
+//
+// Token t of a chunk [s, s+C) attends the tree over the s tokens cached
+// before the chunk (RecSA abstract: per-level selection of at most k
+// candidates, summaries of the unselected candidates in one softmax with the
+// exact tokens, candidate-index RoPE), then the chunk's own tokens s..t,
+// which follow the level-0 candidates: the query sits at index n0 + (t - s)
+// among n0 kept tokens plus the chunk prefix. The chunk-local part (causal
+// attention inside the chunk) has already been computed as a softmax state
+// per (token, query head); this kernel runs the descent, accumulates the
+// tree's entries into a second state and merges the two.
+//
+// Per level, the candidates (children of the kept parents, ascending) are
+// brought into shared memory TILE rows at a time with bulk async copies and
+// scored in fp32 on CUDA cores (the selection must match the fp64 reference
+// exactly); the top k come from a bitonic sort of the packed (score, id)
+// keys; the value rows of the candidates not kept are then streamed for the
+// softmax. Level-0 candidates are scored and accumulated tile by tile.
+#include "common.cuh"
+
+namespace recsa {
+
+constexpr int PT_THREADS = 256;
+constexpr int PT_WARPS = PT_THREADS / 32;
+constexpr int PT_TILE = 128;
+constexpr int PT_KMAX = 64;
+constexpr int PT_CPT = 4;  // output columns per thread in the softmax-value product
+
+struct PrefillTreeArgs {
+    const void* q;       // [B][C][Hq][D]
+    void* out;           // [B][C][Hq][D]
+    const float* state;  // [B][C][Hq][D + 2] local part: unnormalised acc, max, sum
+    int* sel_out;        // nullable [B][C][H][J_cap][k]
+    int C, Hq;
+    int maxc;            // most candidates a level can have
+    int sortn;           // power of two >= maxc
+};
+
+struct PtSmem {
+    uint64_t bar[2];
+    unsigned long long thresh;
+    int par[PT_KMAX], chosen[PT_KMAX];
+    int nlev[MAXJ + 1];
+    float red[PT_WARPS][8];
+    float M[8];
+};
+
+// [tiles: K | V (2 * TILE * D * elem), later the entry-group partials][PtSmem]
+// [key u64 maxc][skey u64 sortn][qf G*D][lg G*maxc][pbuf TILE*G][cacc G*D][cl G]
+__host__ __device__ inline size_t prefill_tree_smem(int D, int G, int elem, int maxc, int sortn) {
+    size_t tiles = 2 * (size_t)PT_TILE * D * elem;
+    const size_t eg = (size_t)(PT_THREADS / (D / PT_CPT)) * G * D * 4;
+    if (eg > tiles) tiles = eg;
+    tiles = (tiles + 127) & ~(size_t)127;
+    return tiles + sizeof(PtSmem) + (size_t)maxc * 8 + (size_t)sortn * 8 +
+           (size_t)(G * D + G * maxc + PT_TILE * G + G * D + G) * 4;
+}
+__host__ __device__ inline size_t prefill_tree_tiles(int D, int G, int elem) {
+    size_t tiles = 2 * (size_t)PT_TILE * D * elem;
+    const size_t eg = (size_t)(PT_THREADS / (D / PT_CPT)) * G * D * 4;
+    if (eg > tiles) tiles = eg;
+    return (tiles + 127) & ~(size_t)127;
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams p, PrefillTreeArgs a) {
+    constexpr int HD = D / 2;
+    constexpr int PL = 4;
+    constexpr int P2 = PL / 2;
+    constexpr int LPC = HD / PL;
+    constexpr int CPW = 32 / LPC;
+    static_assert(G <= LPC && 32 % LPC == 0 && G <= 8, "scoring layout");
+    constexpr int NCC = D / PT_CPT, NEG = PT_THREADS / NCC;
+    constexpr int W = PT_WARPS;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = blockIdx.x;            // token of the chunk
+    const long long u = blockIdx.y;      // (sequence, KV head)
+    const int bseq = (int)(u / p.H), h = (int)(u % p.H);
+    const int b = p.b, MC = a.maxc;
+
+    extern __shared__ __align__(128) unsigned char smem_pt[];
+    const size_t tiles_bytes = prefill_tree_tiles(D, G, (int)sizeof(T));
+    T* Kt = reinterpret_cast<T*>(smem_pt);
+    T* Vt = Kt + (size_t)PT_TILE * D;
+    float* egacc = reinterpret_cast<float*>(smem_pt);
+    PtSmem* sm = reinterpret_cast<PtSmem*>(smem_pt + tiles_bytes);
+    unsigned long long* key = reinterpret_cast<unsigned long long*>(sm + 1);
+    unsigned long long* skey = key + MC;
+    float* qf = reinterpret_cast<float*>(skey + a.sortn);
+    float* lg = qf + G * D;           // [G][MC]
+    float* pbuf = lg + G * MC;        // [TILE][G]
+    float* cacc = pbuf + PT_TILE * G;
+    float* cl = cacc + G * D;
+
+    if (tid == 0) {
+        mbar_init(&sm->bar[0], 1);
+        mbar_init(&sm->bar[1], 1);
+        fence_mbar_init();
+    }
+    if (tid < 8) sm->M[tid] = -INFINITY;
+    {
+        const T* qg = reinterpret_cast<const T*>(a.q) + (((size_t)bseq * a.C + t) * a.Hq + h * G) * D;
+        for (int i = tid; i < G * D; i += PT_THREADS) qf[i] = to_f(qg[i]);
+    }
+    const long long Sraw = p.len[u];  // tokens in the tree (the chunk starts here)
+    const bool bad_len = (Sraw < 0 || Sraw + a.C > p.cap);
+    const int S = bad_len ? 0 : (int)Sraw;
+    bool bad = bad_len;
+    if (tid == 0) {
+        if (bad_len) flag_error(p.err, ERR_LENGTH);
+        int n = S;
+        sm->nlev[0] = n;
+        for (int j = 1; j <= p.J_cap; j++) {
+            n = (n + b - 1) / b;
+            sm->nlev[j] = n;
+        }
+    }
+    __syncthreads();
+
+    const int cc = tid % NCC, eg = tid / NCC;
+    float2 acc[G][PT_CPT / 2];
+    float lpart[G];
+#pragma unroll
+    for (int g = 0; g < G; g++) {
+        lpart[g] = 0.f;
+#pragma unroll
+        for (int c = 0; c < PT_CPT / 2; c++) acc[g][c] = make_float2(0.f, 0.f);
+    }
+    uint32_t phase[2] = {0u, 0u};
+
+    // thread 0: rows [r0, r1) of level j's candidate list (children of sm->par)
+    auto issue = [&](int which, int j, int r0, int r1) {
+        T* dst = which == 0 ? Kt : Vt;
+        const T* base = reinterpret_cast<const T*>(which == 0 ? p.K[j] : p.V[j]) + (u * p.rows[j]) * D;
+        const int n_j = sm->nlev[j];
+        const int pr = r0 / b, o0 = r0 - pr * b;
+        uint32_t total = 0;
+        for (int r = r0, q = pr, o = o0; r < r1; q++, o = 0) {
+            const int n = min(b - o, r1 - r);
+            const int id0 = sm->par[q] * b + o;
+            if (id0 >= 0 && id0 + n <= n_j) total += (uint32_t)(n * D * sizeof(T));
+            r += n;
+        }
+        fence_proxy_async_shared();
+        mbar_arrive_expect_tx(&sm->bar[which], total);
+        for (int r = r0, q = pr, o = o0; r < r1; q++, o = 0) {
+            const int n = min(b - o, r1 - r);
+            const int id0 = sm->par[q] * b + o;
+            if (id0 >= 0 && id0 + n <= n_j)
+                bulk_g2s(dst + (size_t)(r - r0) * D, base + (size_t)id0 * D, (uint32_t)(n * D * sizeof(T)),
+                         &sm->bar[which]);
+            else
+                flag_error(p.err, ERR_SHAPE);
+            r += n;
+        }
+    };
+    auto wait_tile = [&](int which) {
+        if (!mbar_wait(&sm->bar[which], phase[which])) {
+            if (lane == 0) flag_error(p.err, ERR_TIMEOUT);
+            bad = true;
+        }
+        phase[which] ^= 1u;
+    };
+    auto ncand_of = [&](int j, int npar) -> int {
+        const int n_j = sm->nlev[j];
+        const int last = sm->par[npar - 1];
+        if (last < 0 || last * b >= n_j) return 0;
+        return (npar - 1) * b + min(b, n_j - last * b);
+    };
+
+    // Scores of tile rows [0, nmy) = candidate ranks [r0, r0 + nmy) with the
+    // query at index P: key rotated by (rank mod b), query by P - b*(rank / b).
+    auto score_tile = [&](int r0, int nmy, int P, bool want_keys) {
+        const int grp = lane / LPC, gl = lane % LPC;
+        const int chunk = (nmy + W - 1) / W;
+        const int w_lo = warp * chunk, w_hi = min(nmy, w_lo + chunk);
+        float2 qa2[G][P2], qb2[G][P2];
+        int rcur = -1;
+        for (int base = w_lo; base < w_hi; base += CPW) {
+            const int i = base + grp;
+            float v[G];
+#pragma unroll
+            for (int g = 0; g < G; g++) v[g] = 0.f;
+            if (i < w_hi) {
+                const int rnk = r0 + i, r = rnk / b, o = rnk - r * b;
+                if (r != rcur) {
+                    const float* row = p.rope + (size_t)(P - r * b) * 3 * HD + gl * PL;
+                    float2 c2[P2], s2[P2], n2[P2];
+                    load_tab2<PL>(row, c2);
+                    load_tab2<PL>(row + HD, s2);
+                    load_tab2<PL>(row + 2 * HD, n2);
+#pragma unroll
+                    for (int g = 0; g < G; g++)
+#pragma unroll
+                        for (int x = 0; x < P2; x++) {
+                            const float2 xa = make_float2(qf[g * D + gl * PL + 2 * x], qf[g * D + gl * PL + 2 * x + 1]);
+                            const float2 xb = make_float2(qf[g * D + HD + gl * PL + 2 * x],
+                                                          qf[g * D + HD + gl * PL + 2 * x + 1]);
+                            qa2[g][x] = ffma2(xa, c2[x], fmul2(xb, n2[x]));
+                            qb2[g][x] = ffma2(xb, c2[x], fmul2(xa, s2[x]));
+                        }
+                    rcur = r;
+                }
+                const float* row = p.rope + (size_t)o * 3 * HD + gl * PL;
+                float2 c2[P2], s2[P2], n2[P2], ka[P2], kb[P2];
+                load_tab2<PL>(row, c2);
+                load_tab2<PL>(row + HD, s2);
+                load_tab2<PL>(row + 2 * HD, n2);
+                load_row2<T, PL>(Kt + (size_t)i * D + gl * PL, ka);
+                load_row2<T, PL>(Kt + (size_t)i * D + HD + gl * PL, kb);
+                float2 v2[G];
+#pragma unroll
+                for (int g = 0; g < G; g++) v2[g] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int x = 0; x < P2; x++) {
+                    const float2 ra = ffma2(ka[x], c2[x], fmul2(kb[x], n2[x]));
+                    const float2 rb = ffma2(kb[x], c2[x], fmul2(ka[x], s2[x]));
+#pragma unroll
+                    for (int g = 0; g < G; g++) v2[g] = ffma2(qa2[g][x], ra, ffma2(qb2[g][x], rb, v2[g]));
+                }
+#pragma unroll
+                for (int g = 0; g < G; g++) v[g] = v2[g].x + v2[g].y;
+            }
+            int cnt = G, hh = 0, tbits = 0;
+#pragma unroll
+            for (int sft = LPC / 2; sft >= 1; sft >>= 1) {
+                if (cnt > 1) {
+                    const int half = cnt / 2;
+                    const bool hi = (gl & sft) != 0;
+#pragma unroll
+                    for (int x = 0; x < G / 2; x++) {
+                        if (x < half) {
+                            const float send = hi ? v[x] : v[x + half];
+                            const float keep = hi ? v[x + half] : v[x];
+                            v[x] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+                        }
+                    }
+                    hh += hi ? half : 0;
+                    tbits |= sft;
+                    cnt = half;
+                } else {
+                    v[0] += __shfl_xor_sync(0xffffffffu, v[0], sft);
+                }
+            }
+            const float logit = v[0] * p.scale;
+            float Ssum = logit;
+#pragma unroll
+            for (int sft = LPC / 2; sft >= 1; sft >>= 1)
+                if (tbits & sft) Ssum += __shfl_xor_sync(0xffffffffu, Ssum, sft);
+            if (i < w_hi && (gl & ~tbits) == 0) {
+                lg[hh * MC + r0 + i] = logit;
+                if (hh == 0 && want_keys) {
+                    const int rnk = r0 + i, q = rnk / b;
+                    key[r0 + i] = sel_key(Ssum, sm->par[q] * b + (rnk - q * b));
+                }
+            }
+        }
+    };
+
+    // Entries of tile rows [0, nmy) (ranks r0..) join the CTA's softmax:
+    // all of them (tokens) or the candidates not kept (key < threshold).
+    auto accumulate = [&](int r0, int nmy, bool tokens) {
+        float mx[G];
+#pragma unroll
+        for (int g = 0; g < G; g++) mx[g] = -INFINITY;
+        for (int e = tid; e < nmy; e += PT_THREADS) {
+            if (tokens || key[r0 + e] < sm->thresh)
+#pragma unroll
+                for (int g = 0; g < G; g++) mx[g] = fmaxf(mx[g], lg[g * MC + r0 + e]);
+        }
+#pragma unroll
+        for (int g = 0; g < G; g++) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], o));
+            if (lane == 0) sm->red[warp][g] = mx[g];
+        }
+        __syncthreads();
+        float Mn[G], alpha[G];
+#pragma unroll
+        for (int g = 0; g < G; g++) {
+            float m = sm->M[g];
+            const float mold = m;
+#pragma unroll
+            for (int w = 0; w < W; w++) m = fmaxf(m, sm->red[w][g]);
+            Mn[g] = m;
+            alpha[g] = (m == -INFINITY) ? 1.f : (mold == -INFINITY ? 0.f : expf(mold - m));
+            lpart[g] *= alpha[g];
+        }
+        for (int e = tid; e < nmy; e += PT_THREADS) {
+            const bool valid = tokens || key[r0 + e] < sm->thresh;
+#pragma unroll
+            for (int g = 0; g < G; g++) {
+                const float pe = valid ? expf(lg[g * MC + r0 + e] - Mn[g]) : 0.f;
+                pbuf[e * G + g] = pe;
+                lpart[g] += pe;
+            }
+        }
+        __syncthreads();
+        if (tid < G) sm->M[tid] = Mn[tid];
+#pragma unroll
+        for (int g = 0; g < G; g++)
+#pragma unroll
+            for (int c = 0; c < PT_CPT / 2; c++) acc[g][c] = fmul2(acc[g][c], make_float2(alpha[g], alpha[g]));
+#pragma unroll 2
+        for (int e = eg; e < nmy; e += NEG) {
+            float2 vv[PT_CPT / 2];
+            load_row2<T, PT_CPT>(Vt + (size_t)e * D + cc * PT_CPT, vv);
+#pragma unroll
+            for (int g = 0; g < G; g++) {
+                const float pe = pbuf[e * G + g];
+                const float2 pp = make_float2(pe, pe);
+#pragma unroll
+                for (int c = 0; c < PT_CPT / 2; c++) acc[g][c] = ffma2(pp, vv[c], acc[g][c]);
+            }
+        }
+    };
+
+    int J = 0;
+    if (!bad_len && S > 0) {
+        J = 1;
+        while (J < p.J_cap && sm->nlev[J] > b) J++;  // top level of the tree over S tokens
+        int j = J, npar = 1;
+        if (tid == 0) sm->par[0] = 0;
+        __syncthreads();
+        int* selrow = a.sel_out ? a.sel_out + (((size_t)bseq * a.C + t) * p.H + h) * p.J_cap * p.k : nullptr;
+        for (; j >= 1; j--) {
+            const int ncand = ncand_of(j, npar);
+            if (ncand < 1) {
+                if (tid == 0) flag_error(p.err, ERR_SHAPE);
+                bad = true;
+                break;
+            }
+            const int kk = min(p.k, ncand);
+            if (ncand > p.k) {
+                // score every candidate, tile by tile
+                for (int r0 = 0; r0 < ncand; r0 += PT_TILE) {
+                    const int nmy = min(PT_TILE, ncand - r0);
+                    if (tid == 0) issue(0, j, r0, r0 + nmy);
+                    wait_tile(0);
+                    score_tile(r0, nmy, ncand - 1, true);
+                    __syncthreads();
+                }
+                // top kk by a descending bitonic sort of the packed keys
+                for (int i = tid; i < a.sortn; i += PT_THREADS) skey[i] = i < ncand ? key[i] : 0ull;
+                __syncthreads();
+                for (int k2 = 2; k2 <= a.sortn; k2 <<= 1)
+                    for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
+                        for (int i = tid; i < a.sortn; i += PT_THREADS) {
+                            const int ixj = i ^ j2;
+                            if (ixj > i) {
+                                const unsigned long long x = skey[i], y = skey[ixj];
+                                const bool desc = (i & k2) == 0;
+                                if (desc ? (x < y) : (x > y)) {
+                                    skey[i] = y;
+                                    skey[ixj] = x;
+                                }
+                            }
+                        }
+                        __syncthreads();
+                    }
+                if (tid < kk) {
+                    const int id = (int)key_id(skey[tid]);
+                    int pos = 0;
+                    for (int r = 0; r < kk; r++) pos += (int)key_id(skey[r]) < id;
+                    sm->chosen[pos] = id;
+                }
+                if (tid == 0) sm->thresh = skey[kk - 1];
+                __syncthreads();
+                // summaries of the candidates not kept
+                for (int r0 = 0; r0 < ncand; r0 += PT_TILE) {
+                    const int nmy = min(PT_TILE, ncand - r0);
+                    if (tid == 0) issue(1, j, r0, r0 + nmy);
+                    wait_tile(1);
+                    accumulate(r0, nmy, false);
+                    __syncthreads();
+                }
+            } else {  // keeps every candidate: nothing to read or score
+                if (tid < ncand) sm->chosen[tid] = sm->par[tid / b] * b + tid % b;
+                __syncthreads();
+            }
+            if (selrow)
+                for (int x = tid; x < p.k; x += PT_THREADS) selrow[(j - 1) * p.k + x] = x < kk ? sm->chosen[x] : -1;
+            if (tid < kk) sm->par[tid] = sm->chosen[tid];
+            npar = kk;
+            __syncthreads();
+        }
+        // level 0: the tokens under the kept level-1 nodes, then (in index
+        // order) the chunk's own tokens, already in the local state
+        const int n0 = bad ? 0 : ncand_of(0, npar);
+        const int P0 = n0 + t;
+        for (int r0 = 0; r0 < n0; r0 += PT_TILE) {
+            const int nmy = min(PT_TILE, n0 - r0);
+            if (tid == 0) {
+                issue(0, 0, r0, r0 + nmy);
+                issue(1, 0, r0, r0 + nmy);
+            }
+            wait_tile(0);
+            score_tile(r0, nmy, P0, false);
+            __syncthreads();
+            wait_tile(1);
+            accumulate(r0, nmy, true);
+            __syncthreads();
+        }
+    }
+    if (a.sel_out) {
+        int* selrow = a.sel_out + (((size_t)bseq * a.C + t) * p.H + h) * p.J_cap * p.k;
+        for (int i = tid; i < (p.J_cap - J) * p.k; i += PT_THREADS) selrow[J * p.k + i] = -1;
+    }
+
+    // CTA state of the tree entries (egacc overlays the tiles)
+    __syncthreads();
+#pragma unroll
+    for (int g = 0; g < G; g++) {
+#pragma unroll
+        for (int c = 0; c < PT_CPT / 2; c++) {
+            egacc[(eg * G + g) * D + cc * PT_CPT + 2 * c] = acc[g][c].x;
+            egacc[(eg * G + g) * D + cc * PT_CPT + 2 * c + 1] = acc[g][c].y;
+        }
+        float s = lpart[g];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) sm->red[warp][g] = s;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < G * D; idx += PT_THREADS) {
+        float s = 0.f;
+#pragma unroll
+        for (int x = 0; x < NEG; x++) s += egacc[x * G * D + idx];
+        cacc[idx] = s;
+    }
+    if (tid < G) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < W; w++) s += sm->red[w][tid];
+        cl[tid] = s;
+    }
+    __syncthreads();
+    // merge with the chunk-local state and write the output
+    for (int idx = tid; idx < G * D; idx += PT_THREADS) {
+        const int g = idx / D, e = idx % D;
+        const float* st = a.state + (((size_t)bseq * a.C + t) * a.Hq + h * G + g) * (D + 2);
+        const float ml = st[D], ll = st[D + 1], mt = sm->M[g];
+        const float M = fmaxf(ml, mt);
+        const float ft = (mt == -INFINITY) ? 0.f : expf(mt - M);
+        const float fl = (ml == -INFINITY) ? 0.f : expf(ml - M);
+        const float num = cacc[idx] * ft + st[e] * fl;
+        const float den = cl[g] * ft + ll * fl;
+        T* outp = reinterpret_cast<T*>(a.out) + (((size_t)bseq * a.C + t) * a.Hq + h * G + g) * D;
+        outp[e] = from_f<T>(bad ? 0.f : num / den);
+    }
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_prefill_tree(const TreeParams& p, const void* q, void* out, const float* state, int* sel_out,
+                                int B, int C, int Hq, cudaStream_t s) {
+    PrefillTreeArgs a{q, out, state, sel_out, C, Hq, 0, 1};
+    a.maxc = p.k * p.b > p.b ? p.k * p.b : p.b;
+    while (a.sortn < a.maxc) a.sortn <<= 1;
+    const size_t smem = prefill_tree_smem(D, G, (int)sizeof(T), a.maxc, a.sortn);
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
+    auto kern = prefill_tree_kernel<T, D, G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    dim3 grid(C, B * p.H);
+    kern<<<grid, PT_THREADS, smem, s>>>(p, a);
+    return cudaGetLastError();
+}
+
+size_t prefill_tree_smem_bytes(int D, int G, int elem, int k, int b) {
+    int maxc = k * b > b ? k * b : b, sortn = 1;
+    while (sortn < maxc) sortn <<= 1;
+    return prefill_tree_smem(D, G, elem, maxc, sortn);
+}
+
+#define RECSA_INST_PT(T, D, G)                                                                                   \
+    template cudaError_t launch_prefill_tree<T, D, G>(const TreeParams&, const void*, void*, const float*, int*, \
+                                                      int, int, int, cudaStream_t);
+#define RECSA_INST_PT_G(T, D) RECSA_INST_PT(T, D, 1) RECSA_INST_PT(T, D, 2) RECSA_INST_PT(T, D, 4) RECSA_INST_PT(T, D, 8)
+RECSA_INST_PT_G(__nv_bfloat16, 64)
+RECSA_INST_PT_G(__nv_bfloat16, 128)
+
+}  // namespace recsa

@@ -283,6 +283,8 @@ static void pq_rows(void* p, long long lo, long long hi) {
     pq_args* a = (pq_args*)p;
     uint64_t bn = synth_stream(a->seed, TAG_PQ_NOISE, (uint64_t)a->seq);
     int Hq = a->H * a->G;
+    double* cent = (double*)malloc(sizeof(double) * (size_t)a->H * (size_t)a->d);
+    long long cent_run = -1;
     for (long long r = lo; r < hi; r++) { /* r indexes (t - t0) */
         long long t = a->t0 + r;
         long long L0 = 0, H0 = a->n_runs - 1;
@@ -293,16 +295,26 @@ static void pq_rows(void* p, long long lo, long long hi) {
             else
                 H0 = mid - 1;
         }
+        if (L0 != cent_run) { /* centroids of this run, every KV head */
+            for (int h = 0; h < a->H; h++) {
+                long long m = run_centroid(a->seed, a->seq, L0, a->H, h, a->M);
+                for (int i = 0; i < a->d; i++) cent[h * a->d + i] = centroid_coord(a->seed, a->H, h, m, a->M, a->d, i);
+            }
+            cent_run = L0;
+        }
         for (int g = 0; g < Hq; g++) {
             int h = g / a->G;
-            long long m = run_centroid(a->seed, a->seq, L0, a->H, h, a->M);
-            for (int i = 0; i < a->d; i++) {
-                double x = centroid_coord(a->seed, a->H, h, m, a->M, a->d, i) +
-                           a->sigma * synth_normal_at(bn, ((uint64_t)t << 24) + (uint64_t)g * (uint64_t)a->d + (uint64_t)i);
-                store(a->out, a->out_bf16, (r * Hq + g) * (int64_t)a->d + i, x);
+            uint64_t ctr = ((uint64_t)t << 24) + (uint64_t)g * (uint64_t)a->d;
+            for (int i = 0; i < a->d; i += 2) {
+                double c, sn;
+                normal_pair(bn, (ctr + (uint64_t)i) >> 1, &c, &sn);
+                store(a->out, a->out_bf16, (r * Hq + g) * (int64_t)a->d + i, cent[h * a->d + i] + a->sigma * c);
+                store(a->out, a->out_bf16, (r * Hq + g) * (int64_t)a->d + i + 1,
+                      cent[h * a->d + i + 1] + a->sigma * sn);
             }
         }
     }
+    free(cent);
 }
 
 /* Prefill queries for tokens [t0, t1) of sequence `seq`: out[(t-t0)][g][i]. */
