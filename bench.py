@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--prefill-workload", default="prefill_524k")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU-baseline sample")
     ap.add_argument("--settle-s", type=float, default=0.3, help="decode-only launches before timing (clock sampling)")
     return ap.parse_args()
@@ -229,6 +231,85 @@ def run_reference(args, w, world, rank):
                                        "right-edge node refresh + one query per KV head, fp64"},
             "e2e": {"value": v, "unit": "query-tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ prefill
+
+
+def measure_prefill(wname, dev, flush, hbm_gbs):
+    """Chunked prefill of one sequence: every chunk runs recsa_prefill then
+    recsa_append (the tree grows after each chunk). Returns the timings and a
+    dense causal prefill of the same length (torch SDPA) for comparison."""
+    from hierarchical_sparse_attention_tree_b200 import RecsaLayer
+
+    w = synth.WORKLOADS[wname]
+    B, H, Hq, D, C, Ltot = w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim, w.chunk, w.length
+    bf = torch.bfloat16
+    t0 = time.perf_counter()
+    K, V, runs = synth.cache_arrays(w, Ltot)
+    Q = [synth.prefill_queries(w.seed, b, 0, Ltot, H, w.group, D, w.centroids, w.sigma_noise, runs[b], True)
+         for b in range(B)]
+    Wp = synth.workload_pooler(w)
+    gen_s = time.perf_counter() - t0
+    layer = RecsaLayer(B, H, Hq, D, w.branching, w.k, Ltot, torch.from_numpy(Wp).view(bf).to(dev), dtype=bf,
+                       rope_base=w.rope_base, max_chunk=C, device=dev)
+    kd = torch.from_numpy(np.ascontiguousarray(K.transpose(0, 2, 1, 3))).view(bf).to(dev)  # [B][L][H][D]
+    vd = torch.from_numpy(np.ascontiguousarray(V.transpose(0, 2, 1, 3))).view(bf).to(dev)
+    qd = torch.stack([torch.from_numpy(x).view(bf) for x in Q]).to(dev)                      # [B][L][Hq][D]
+    del K, V, Q
+    out = torch.empty((B, C, Hq, D), dtype=bf, device=dev)
+    n_chunks = (Ltot + C - 1) // C
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_chunks)]
+    stream = torch.cuda.current_stream(dev)
+    # one warm-up chunk on a throw-away layer of the same shape
+    warm = RecsaLayer(B, H, Hq, D, w.branching, w.k, 2 * C, torch.from_numpy(Wp).view(bf).to(dev), dtype=bf,
+                      rope_base=w.rope_base, max_chunk=C, device=dev)
+    for s0 in (0, C):
+        warm.prefill(qd[:, s0:s0 + C].contiguous(), kd[:, s0:s0 + C].contiguous(), vd[:, s0:s0 + C].contiguous(), out)
+        warm.append(kd[:, s0:s0 + C].contiguous(), vd[:, s0:s0 + C].contiguous())
+    torch.cuda.synchronize(dev)
+    warm.close()
+    chunks = [(qd[:, s0:s0 + C].contiguous(), kd[:, s0:s0 + C].contiguous(), vd[:, s0:s0 + C].contiguous())
+              for s0 in range(0, Ltot, C)]
+    torch.cuda.synchronize(dev)
+    for i, (qc, kc, vc) in enumerate(chunks):
+        flush.fill_(5.0)
+        ev[i][0].record(stream)
+        layer.prefill(qc, kc, vc, out[:, :qc.shape[1]])
+        ev[i][1].record(stream)
+        layer.append(kc, vc)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    layer.check()
+    pre_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    app_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(pre_ms) + sum(app_ms)
+    del chunks
+    layer.close()
+    res = {"workload": wname, "tokens": B * Ltot, "chunk": C, "tok_s": B * Ltot / (total_ms / 1e3),
+           "ms_total": total_ms, "ms_per_chunk": total_ms / n_chunks, "build_share": sum(app_ms) / total_ms,
+           "prefill_ms_per_chunk": sum(pre_ms) / n_chunks, "append_ms_per_chunk": sum(app_ms) / n_chunks,
+           "input_gen_s": gen_s, "l2": "flushed before each chunk"}
+    # dense causal prefill of the same length (torch SDPA, GQA), one timed run after a warm-up
+    try:
+        qt = qd.transpose(1, 2)                   # [B][Hq][L][D]
+        kt = kd.transpose(1, 2)
+        vt = vd.transpose(1, 2)
+        sdpa = torch.nn.functional.scaled_dot_product_attention
+        sdpa(qt[:, :, :C], kt[:, :, :C], vt[:, :, :C], is_causal=True, enable_gqa=True)
+        torch.cuda.synchronize(dev)
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        sdpa(qt, kt, vt, is_causal=True, enable_gqa=True)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        dms = a_.elapsed_time(b_)
+        flops = 4.0 * B * Hq * D * Ltot * Ltot / 2
+        res["dense_sdpa"] = {"ms": dms, "tok_s": B * Ltot / (dms / 1e3), "tflops": flops / (dms / 1e3) / 1e12,
+                             "recsa_speedup": dms / total_ms}
+    except Exception as e:  # the comparator is optional
+        res["dense_sdpa"] = {"error": str(e)[:200]}
+    return res
 
 
 # -------------------------------------------------------------------- main
@@ -443,6 +524,10 @@ def main():
                "sample": f"{done} decode steps of sequence 0 of {B} (8 KV heads in parallel): refresh of the "
                          "nodes the new token touched + one query per KV head, fp64"}
 
+    prefill = None
+    if not args.no_prefill:
+        prefill = measure_prefill(args.prefill_workload, dev, flush, hbm)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "query-tok/s", "n_gpus": world, "steps": K_, "warmup": W_,
@@ -452,7 +537,7 @@ def main():
                        "head_dim": D, "branching": w.branching, "k": w.k,
                        "step": "recsa_append(1 token/seq) + recsa_decode(1 query/seq)",
                        "l2": "flushed between steps (256 MB write, outside the events)",
-                       "value_is": "decode query-tok/s; prefill not measured in this line"},
+                       "value_is": "decode query-tok/s; prefill tok/s under 'prefill'"},
             "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": achieved, "peak": hbm,
                          "unit": "GB/s", "frac": achieved / hbm, "peak_source": peak_src,
                          "traffic": kernel_traffic("decode_kernel"),
@@ -462,7 +547,7 @@ def main():
             "build_tree": {"ms": build_ms, "gbs": build_bytes / (build_ms / 1e3) / 1e9,
                            "frac_hbm": build_bytes / (build_ms / 1e3) / 1e9 / hbm},
             "e2e": e2e, "gpu_launches": 2 * K_, "clocks": clk, "dense_decode": dense, "cpu_baseline": cpu,
-            "wall_s_timed_loop": wall_s, "input_gen_s": gen_s,
+            "wall_s_timed_loop": wall_s, "input_gen_s": gen_s, "prefill": prefill,
         }
         print(json.dumps(line), flush=True)
     layer.close()
