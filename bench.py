@@ -334,7 +334,7 @@ def main():
     B, H, Hq, D = w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim
     L0 = w.length
     W_, K_ = args.warmup, args.steps
-    n_total = 2 * (W_ + K_) + 9
+    n_total = 2 * (W_ + K_) + 25
     cap = L0 + n_total
     seq_off = rank * B
     bf = torch.bfloat16
@@ -381,12 +381,11 @@ def main():
 
     # ---- device-resident decode steps: warm-up, then K timed steps. One
     # step = append one token per sequence + one decode query per sequence,
-    # bracketed by two events (the decode may overlap the append's tail).
-    def step(s, ev=None):
+    # one launch (recsa_append_decode), bracketed by two events.
+    def step(s, ev=None, rows_out=None):
         if ev is not None:
             ev[0].record(stream)
-        layer.append(kn_d[s], vn_d[s])
-        layer.decode(q_d[s], out)
+        layer.append_decode(kn_d[s], vn_d[s], q_d[s], out, rows_out=rows_out)
         if ev is not None:
             ev[1].record(stream)
 
@@ -410,7 +409,7 @@ def main():
     t_wall = time.perf_counter()
     for i in range(K_):
         flush.fill_(float(s_idx))
-        step(s_idx, evs[i])
+        step(s_idx, evs[i], rows[i])
         s_idx += 1
     torch.cuda.synchronize(dev)
     wall_s = time.perf_counter() - t_wall
@@ -421,18 +420,29 @@ def main():
     step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     total_s = max_over_ranks(sum(step_ms) / 1e3, world)
     value = world * B * K_ / total_s
+    rows_np = rows.cpu().numpy()  # K and V rows each fused step's descent read
 
-    # ---- the decode kernel alone (roofline): K launches on the current tree,
-    # L2 flushed before each, events around each launch on its stream
+    # ---- for the record: the decode kernel alone (K launches on the current
+    # tree), the append alone, and the step as two launches
     dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_)]
     for i in range(K_):
         flush.fill_(3.0)
         dev_ev[i][0].record(stream)
-        layer.decode(q_d[i % n_total], out, rows_out=rows[i])
+        layer.decode(q_d[i % n_total], out)
         dev_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     layer.check()
     dec_ms = [e[0].elapsed_time(e[1]) for e in dev_ev]
+    split_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(16)]
+    for i in range(16):
+        flush.fill_(5.0)
+        split_ev[i][0].record(stream)
+        layer.append(kn_d[s_idx], vn_d[s_idx])
+        layer.decode(q_d[s_idx], out)
+        split_ev[i][1].record(stream)
+        s_idx += 1
+    torch.cuda.synchronize(dev)
+    split_ms = [e[0].elapsed_time(e[1]) for e in split_ev]
     # append alone, for the record (appends K more tokens)
     app_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(8)]
     for i in range(8):
@@ -444,12 +454,17 @@ def main():
     torch.cuda.synchronize(dev)
     app_ms = [e[0].elapsed_time(e[1]) for e in app_ev]
 
-    rows_np = rows.cpu().numpy()
-    dec_bytes = int(rows_np.sum()) * D * es + K_ * 2 * B * Hq * D * es  # gathered K/V rows + q + out
+    # roofline of the fused step kernel: algorithmic bytes per launch = the
+    # gathered K/V rows + q + out, plus the append (new token row; per level
+    # the right-edge node K, V, fp32 value sum written and prefix sums read
+    # and written; the pooler once)
+    J_cap = layer.tree_shape()[0]
+    app_bytes = B * H * (2 * D * es + J_cap * D * (2 * es + 4 + 16)) + D * D * es
+    dec_bytes = int(rows_np.sum()) * D * es + K_ * (2 * B * Hq * D * es + app_bytes)
     dec_bytes_per_launch = dec_bytes / K_
     peaks, peak_src = measured_peaks()
     hbm = float(peaks["hbm_gbs"])
-    dec_avg_s = sum(dec_ms) / K_ / 1e3
+    dec_avg_s = sum(step_ms) / K_ / 1e3
     achieved = dec_bytes_per_launch / dec_avg_s / 1e9
 
     # ---- end to end through the public API: pinned host inputs in, output out
@@ -464,8 +479,7 @@ def main():
             qb.copy_(q_h[s], non_blocking=True)
             kb.copy_(kn_h[s], non_blocking=True)
             vb.copy_(vn_h[s], non_blocking=True)
-            layer.append(kb, vb)
-            layer.decode(qb, out)
+            layer.append_decode(kb, vb, qb, out)
             out_h.copy_(out, non_blocking=True)
             if ev is not None:
                 ev[1].record(stream)
@@ -535,7 +549,7 @@ def main():
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "L": L0, "batch_per_gpu": B, "n_q_heads": Hq, "n_kv_heads": H,
                        "head_dim": D, "branching": w.branching, "k": w.k,
-                       "step": "recsa_append(1 token/seq) + recsa_decode(1 query/seq)",
+                       "step": "recsa_append_decode: append 1 token/seq + 1 decode query/seq, one launch",
                        "l2": "flushed between steps (256 MB write, outside the events)",
                        "value_is": "decode query-tok/s; prefill tok/s under 'prefill'"},
             "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": achieved, "peak": hbm,
@@ -543,10 +557,11 @@ def main():
                          "traffic": kernel_traffic("decode_kernel"),
                          "algorithmic_bytes_per_launch": dec_bytes_per_launch, "launch_ms": dec_avg_s * 1e3},
             "append_ms": sum(app_ms) / len(app_ms), "decode_ms": sum(dec_ms) / K_,
+            "split_step_ms": sum(split_ms) / len(split_ms),
             "rows_per_query": {"k_rows": float(rows_np[..., 0].mean()), "v_rows": float(rows_np[..., 1].mean())},
             "build_tree": {"ms": build_ms, "gbs": build_bytes / (build_ms / 1e3) / 1e9,
                            "frac_hbm": build_bytes / (build_ms / 1e3) / 1e9 / hbm},
-            "e2e": e2e, "gpu_launches": 2 * K_, "clocks": clk, "dense_decode": dense, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": K_, "clocks": clk, "dense_decode": dense, "cpu_baseline": cpu,
             "wall_s_timed_loop": wall_s, "input_gen_s": gen_s, "prefill": prefill,
         }
         print(json.dumps(line), flush=True)

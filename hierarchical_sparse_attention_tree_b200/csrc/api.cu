@@ -21,7 +21,8 @@ cudaError_t launch_copy_tokens(const TreeParams&, const void*, const void*, int,
 cudaError_t launch_set_lengths(const TreeParams&, const long long*, cudaStream_t);
 cudaError_t launch_bump_lengths(const TreeParams&, long long, cudaStream_t);
 template <typename T, int D, int G>
-cudaError_t launch_decode(const TreeParams&, const void*, void*, int*, long long*, cudaStream_t);
+cudaError_t launch_decode(const TreeParams&, const void*, const void*, const void*, void*, int*, long long*,
+                          cudaStream_t);
 template <typename T, int D, int G>
 cudaError_t launch_dense(const void*, const void*, const void*, void*, int, long long, long long, float*, int,
                          cudaStream_t);
@@ -323,8 +324,27 @@ recsa_status recsa_decode(recsa_ctx* ctx, const void* q, void* out, int* sel_out
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
     DISPATCH_TD(c.dtype, c.head_dim,
-                DISPATCH_G(ctx->G, e = launch_decode<T, DD, GG>(ctx->p, q, out, sel_out, rows_out, s)));
+                DISPATCH_G(ctx->G, e = launch_decode<T, DD, GG>(ctx->p, nullptr, nullptr, q, out, sel_out, rows_out, s)));
     if (e != cudaSuccess) return cuda_fail(e, "recsa_decode");
+    return RECSA_OK;
+}
+
+recsa_status recsa_append_decode(recsa_ctx* ctx, const void* k_new, const void* v_new, const void* q, void* out,
+                                 int* sel_out, long long* rows_out, recsa_stream_t stream) {
+    if (!ctx || !k_new || !v_new || !q || !out) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(q, 16) || !aligned(out, 16))
+        return fail(RECSA_ERR_INVALID_ARG, "k_new/v_new/q/out not 16-byte aligned");
+    const recsa_config& c = ctx->cfg;
+    for (int b = 0; b < c.batch; b++)
+        if (ctx->len[b] + 1 > c.capacity)
+            return fail(RECSA_ERR_CAPACITY, "sequence %d: %lld + 1 tokens exceed capacity %lld", b, ctx->len[b],
+                        c.capacity);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    DISPATCH_TD(c.dtype, c.head_dim,
+                DISPATCH_G(ctx->G, e = launch_decode<T, DD, GG>(ctx->p, k_new, v_new, q, out, sel_out, rows_out, s)));
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_append_decode");
+    for (int b = 0; b < c.batch; b++) ctx->len[b] += 1;
     return RECSA_OK;
 }
 

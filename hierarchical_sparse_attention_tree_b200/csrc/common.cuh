@@ -195,6 +195,10 @@ namespace recsa {
 __device__ __forceinline__ void fence_proxy_async_shared() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Orders this thread's generic-proxy global accesses with async-proxy ones.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 // The two halves of this lane's PPL rotation pairs, (x_i, x_{i+D/2}) for
 // i = lane*PPL + e, as floats.
@@ -265,18 +269,24 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
     return d;
 }
 
-// N consecutive floats of a RoPE table block (16-byte loads), as float2 pairs.
+// N consecutive floats of a RoPE table block (N = 2: one 8-byte load; N a
+// multiple of 4: 16-byte loads), as float2 pairs.
 template <int N>
 __device__ __forceinline__ void load_tab2(const float* p, float2* out) {
+    static_assert(N == 2 || N % 4 == 0, "table load width");
+    if constexpr (N == 2) {
+        out[0] = __ldg(reinterpret_cast<const float2*>(p));
+    } else {
 #pragma unroll
-    for (int x = 0; x < N / 4; x++) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(p) + x);
-        out[2 * x] = make_float2(v.x, v.y);
-        out[2 * x + 1] = make_float2(v.z, v.w);
+        for (int x = 0; x < N / 4; x++) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(p) + x);
+            out[2 * x] = make_float2(v.x, v.y);
+            out[2 * x + 1] = make_float2(v.z, v.w);
+        }
     }
 }
 
-// N consecutive elements of a row as float2 pairs (N = 4 or 8).
+// N consecutive elements of a row as float2 pairs (N = 2, 4 or 8).
 template <typename T, int N>
 __device__ __forceinline__ void load_row2(const T* row, float2* out) {
     float f[N];

@@ -27,7 +27,9 @@
 // enters a logit), so the keys use b table rows however long the lists are.
 #include <cooperative_groups.h>
 
+#include "append.cuh"
 #include "common.cuh"
+#include "score.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -39,6 +41,8 @@ constexpr int DEC_CLUSTER = 8;
 constexpr int KMAX = 64;
 
 struct DecodeArgs {
+    const void* k_new;    // nullable [B][H][D]: append this token first (fused step)
+    const void* v_new;
     const void* q;
     void* out;
     int* sel_out;         // nullable [B*H][J_cap][k]
@@ -48,8 +52,8 @@ struct DecodeArgs {
 };
 
 struct DecSmem {
-    uint64_t bar[2];                     // [0]: key tile, [1]: value tile
-    unsigned long long topbuf[2][KMAX];  // local top-k lists (sorted), double-buffered by level parity
+    uint64_t bar[3];                     // [0]: key tile, [1]: value tile, [2]: pooler (append)
+    unsigned long long wl[DEC_WARPS][KMAX];  // per-warp top-k lists, sorted, zero padded
     unsigned long long picked[KMAX];     // global top-k keys, best first
     unsigned long long thresh;           // the k-th best key
     int par[KMAX];                       // kept parents of the current level, ascending
@@ -70,13 +74,17 @@ __host__ __device__ constexpr int dec_neg() { return DEC_THREADS / (D / CPT); }
 
 // Shared memory: [region0: K tile | V tile; at the end: entry-group partials,
 // then (rank 0) the cluster gather area][DecSmem][key: u64 MY][gkeys: u64
-// CS*KMAX][qf G*D][lg G*MY][pbuf MY*G][cacc G*D][cml 2G]
+// 2*CS*KMAX][qf G*D][lg MY*G (logits, then softmax weights)][cacc G*D][cml 2G]
 __host__ __device__ inline size_t decode_smem_tail(int D, int G, int MY) {
-    return sizeof(DecSmem) + (size_t)MY * 8 + (size_t)DEC_CLUSTER * KMAX * 8 +
-           (size_t)(G * D + G * MY + MY * G + G * D + 2 * G) * 4;
+    return sizeof(DecSmem) + (size_t)MY * 8 + (size_t)2 * DEC_CLUSTER * KMAX * 8 +
+           (size_t)(G * D + MY * G + G * D + 2 * G) * 4;
 }
-__host__ __device__ inline size_t decode_region0(int D, int G, int MY, int elem) {
-    const size_t tiles = 2 * (size_t)MY * D * elem;
+__host__ __device__ inline size_t decode_region0(int D, int G, int MY, int elem, int J_cap, bool fused) {
+    // the appending CTA of a fused step first holds the pooler and the
+    // append scratch here
+    const size_t app = fused ? (size_t)D * D * elem + append_scratch_floats(D, J_cap) * 4 : 0;
+    const size_t tiles0 = 2 * (size_t)MY * D * elem;
+    const size_t tiles = tiles0 > app ? tiles0 : app;
     const size_t eg = (size_t)(DEC_THREADS / (D / CPT)) * G * D * 4;
     const size_t eg_al = (eg + 127) & ~(size_t)127;
     const size_t gat = (size_t)DEC_CLUSTER * (G * D + 2 * G) * 4;
@@ -99,15 +107,50 @@ __device__ __forceinline__ int rank_among(const unsigned long long* key, int n, 
     return (r0 + r1) + (r2 + r3);
 }
 
+// Sorts one key per lane in descending order across the warp (bitonic network).
+__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
+#pragma unroll
+    for (int k2 = 2; k2 <= 32; k2 <<= 1)
+#pragma unroll
+        for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
+            const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j2);
+            const bool desc = (lane & k2) == 0, lower = (lane & j2) == 0;
+            x = (lower == desc) ? (x > y ? x : y) : (x < y ? x : y);
+        }
+    return x;
+}
+
+// Rank of key x among NL lists (list l at lists + l*stride, n keys each,
+// sorted descending, zero padded): the number of keys greater than x, by one
+// binary search per list, all lists advancing together. Keys are distinct.
+template <int NL>
+__device__ __forceinline__ int rank_in_lists(const unsigned long long* lists, int stride, int n,
+                                             unsigned long long x) {
+    int cnt[NL];
+#pragma unroll
+    for (int l = 0; l < NL; l++) cnt[l] = 0;
+#pragma unroll
+    for (int st = KMAX; st >= 1; st >>= 1) {
+        if (st > n) continue;  // uniform: n is the same in every thread
+        // every probe is a load at a valid index (clamped), so the NL loads of
+        // a round are independent of each other
+#pragma unroll
+        for (int l = 0; l < NL; l++) {
+            const int pos = cnt[l] + st;
+            const unsigned long long y = lists[l * stride + min(pos, n) - 1];
+            cnt[l] = (pos <= n && y > x) ? pos : cnt[l];
+        }
+    }
+    int r = 0;
+#pragma unroll
+    for (int l = 0; l < NL; l++) r += cnt[l];
+    return r;
+}
+
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, DecodeArgs a) {
-    constexpr int HD = D / 2;
-    constexpr int PL = 4;                 // rotation pairs per lane in scoring
-    constexpr int LPC = HD / PL;          // lanes per candidate in scoring
-    constexpr int CPW = 32 / LPC;         // candidates per warp step in scoring
-    static_assert(G <= LPC && 32 % LPC == 0 && G <= 8, "scoring layout");
     constexpr int NCC = dec_ncc<D>();     // column chunks in accumulation
     constexpr int NEG = dec_neg<D>();     // entry groups in accumulation
     constexpr int W = DEC_WARPS;
@@ -126,39 +169,52 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
     float* gat = reinterpret_cast<float*>(smem_raw + ((NEG * G * D * 4 + 127) & ~127));  // [CS][G*D + 2G]
     DecSmem* sm = reinterpret_cast<DecSmem*>(smem_raw + a.region0);
     unsigned long long* key = reinterpret_cast<unsigned long long*>(sm + 1);
-    unsigned long long* gkeys = key + MY;
-    float* qf = reinterpret_cast<float*>(gkeys + DEC_CLUSTER * KMAX);
-    float* lg = qf + G * D;    // [G][MY] logits
-    float* pbuf = lg + G * MY; // [MY][G] softmax weights
-    float* cacc = pbuf + MY * G;
+    unsigned long long* gkeys = key + MY;  // [2][CS][KMAX]: the CTAs' top-k lists, by level parity
+    float* qf = reinterpret_cast<float*>(gkeys + 2 * DEC_CLUSTER * KMAX);
+    float* lg = qf + G * D;    // [MY][G] logits, then softmax weights
+    float* cacc = lg + MY * G;
     float* cml = cacc + G * D;  // [G] max, [G] sum
 
     // set-up that does not read the tree (overlaps the previous kernel under
     // programmatic dependent launch)
+    // fused step: the last CTA of the cluster appends the token (its rows
+    // of the first scored level are the last ones, which the append changes)
+    const bool app = a.k_new != nullptr;
+    const bool appender = app && rank == CS - 1;
     if (tid == 0) {
         mbar_init(&sm->bar[0], 1);
         mbar_init(&sm->bar[1], 1);
+        mbar_init(&sm->bar[2], 1);
         fence_mbar_init();
+        if (appender) {  // the pooler is constant: fetch it before the dependency wait
+            mbar_arrive_expect_tx(&sm->bar[2], (uint32_t)(D * D * sizeof(T)));
+            bulk_g2s(smem_raw, p.Wt, (uint32_t)(D * D * sizeof(T)), &sm->bar[2]);
+        }
     }
+    asm volatile("griddepcontrol.launch_dependents;");
     if (tid < 8) sm->M[tid] = -INFINITY;
     grid_dependency_wait();  // from here on, every earlier kernel's writes are visible
+    const long long Lraw = p.len[u];  // both loads in flight together
     {
         const T* qg = reinterpret_cast<const T*>(a.q) + (u * G) * D;
-        for (int i = tid; i < G * D; i += DEC_THREADS) qf[i] = to_f(qg[i]);
-    }
-
-    const long long Lraw = p.len[u];
-    const bool bad_len = (Lraw <= 0 || Lraw > p.cap);
-    const int L = bad_len ? 0 : (int)Lraw;
-    bool bad = bad_len;
-    if (tid == 0) {
-        if (bad_len && rank == 0) flag_error(p.err, ERR_LENGTH);
-        int n = L;
-        sm->nlev[0] = n;
-        for (int j = 1; j <= p.J_cap; j++) {
-            n = (n + b - 1) / b;
-            sm->nlev[j] = n;
+        constexpr int QV = (G * D) / DEC_THREADS >= 4 ? 4 : 2;  // elements per thread and load
+        float f[QV];
+        for (int i = tid * QV; i < G * D; i += DEC_THREADS * QV) {
+            load_vec<T, QV>(qg + i, f);
+#pragma unroll
+            for (int x = 0; x < QV; x++) qf[i + x] = f[x];
         }
+    }
+    // after a fused append the tree holds one more token
+    const bool bad_len = app ? (Lraw < 0 || Lraw >= p.cap) : (Lraw <= 0 || Lraw > p.cap);
+    const int L = bad_len ? 0 : (int)Lraw + (app ? 1 : 0);
+    bool bad = bad_len;
+    bool appended = false;
+    if (tid == 0 && bad_len && rank == 0) flag_error(p.err, ERR_LENGTH);
+    if (tid <= p.J_cap) {  // n_j = ceil(L / b^j), the same as j nested ceilings
+        long long pw = 1;
+        for (int x = 0; x < tid && pw <= L; x++) pw *= b;
+        sm->nlev[tid] = (int)((L + pw - 1) / pw);
     }
     __syncthreads();
 
@@ -191,6 +247,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
             r += n;
         }
         fence_proxy_async_shared();
+        fence_proxy_async_global();  // global writes of a fused append seen by the bulk reads
         mbar_arrive_expect_tx(&sm->bar[which], total);
         for (int r = r0, q = pr, o = o0; r < r1; q++, o = 0) {
             const int n = min(b - o, r1 - r);
@@ -220,45 +277,37 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
 
     // One shared softmax over every level's entries: entries [0, nmy) of this
     // CTA join with weights exp(logit - running max); `tokens` = every entry
-    // counts, otherwise only candidates that were not kept.
+    // counts, otherwise only candidates that were not kept. The scoring pass
+    // has left each warp's largest logit per head in sm->red (over all rows,
+    // kept ones included: a bound on the entries that join, which is all the
+    // running maximum needs).
+    const int gt = tid % G;  // the head of this thread's weights (DEC_THREADS % G == 0)
     auto accumulate = [&](int nmy, bool tokens) {
-        float mx[G];
-#pragma unroll
-        for (int g = 0; g < G; g++) mx[g] = -INFINITY;
-        for (int e = tid; e < nmy; e += DEC_THREADS) {
-            if (tokens || key[e] < sm->thresh)
-#pragma unroll
-                for (int g = 0; g < G; g++) mx[g] = fmaxf(mx[g], lg[g * MY + e]);
-        }
-#pragma unroll
-        for (int g = 0; g < G; g++) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], o));
-            if (lane == 0) sm->red[warp][g] = mx[g];
-        }
-        __syncthreads();
-        float Mn[G], alpha[G];
+        float Mt = 0.f, Mown = 0.f, alpha[G];
 #pragma unroll
         for (int g = 0; g < G; g++) {
             float m = sm->M[g];
             const float mold = m;
 #pragma unroll
             for (int w = 0; w < W; w++) m = fmaxf(m, sm->red[w][g]);
-            Mn[g] = m;
             alpha[g] = (m == -INFINITY) ? 1.f : (mold == -INFINITY ? 0.f : expf(mold - m));
             lpart[g] *= alpha[g];
+            if (g == gt) Mt = m;
+            if (g == tid) Mown = m;
         }
-        for (int e = tid; e < nmy; e += DEC_THREADS) {
+        float lsum = 0.f;
+        for (int x = tid; x < nmy * G; x += DEC_THREADS) {
+            const int e = x / G;
             const bool valid = tokens || key[e] < sm->thresh;
-#pragma unroll
-            for (int g = 0; g < G; g++) {
-                const float pe = valid ? expf(lg[g * MY + e] - Mn[g]) : 0.f;
-                pbuf[e * G + g] = pe;
-                lpart[g] += pe;
-            }
+            const float pe = valid ? expf(lg[x] - Mt) : 0.f;
+            lg[x] = pe;
+            lsum += pe;
         }
-        __syncthreads();
-        if (tid < G) sm->M[tid] = Mn[tid];
+#pragma unroll
+        for (int g = 0; g < G; g++)
+            if (g == gt) lpart[g] += lsum;
+        __syncthreads();  // weights in place; every thread has read sm->M
+        if (tid < G) sm->M[tid] = Mown;
 #pragma unroll
         for (int g = 0; g < G; g++)
 #pragma unroll
@@ -269,7 +318,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
             load_row2<T, CPT>(Vt + (size_t)e * D + cc * CPT, v);
 #pragma unroll
             for (int g = 0; g < G; g++) {
-                const float pe = pbuf[e * G + g];
+                const float pe = lg[e * G + g];
                 const float2 pp = make_float2(pe, pe);
 #pragma unroll
                 for (int c = 0; c < CPT / 2; c++) acc[g][c] = ffma2(pp, v[c], acc[g][c]);
@@ -277,6 +326,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
         }
     };
 
+    if (appender && bad_len) {  // no append; the pooler copy must land before the area is reused
+        if (!mbar_wait(&sm->bar[2], 0) && tid == 0) flag_error(p.err, ERR_TIMEOUT);
+        __syncthreads();
+    }
     if (!bad_len) {
         int j = 1;
         while (j < p.J_cap && sm->nlev[j] > b) j++;  // top level
@@ -289,8 +342,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
             if (nc > p.k || nc < 1) break;
             if (tid < nc) sm->chosen[tid] = sm->par[tid / b] * b + tid % b;
             __syncthreads();
-            if (rank == 0 && a.sel_out)
-                for (int x = tid; x < p.k; x += DEC_THREADS)
+            if (rank == 0 && a.sel_out)  // not thread 0: it issues the copies
+                for (int x = tid - 32; x >= 0 && x < p.k; x += DEC_THREADS - 32)
                     a.sel_out[(u * p.J_cap + (j - 1)) * p.k + x] = x < nc ? sm->chosen[x] : -1;
             if (tid < nc) sm->par[tid] = sm->chosen[tid];
             npar = nc;
@@ -303,148 +356,147 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
             bad = true;
             if (tid == 0) flag_error(p.err, ERR_SHAPE);
         }
+        // contiguous row ranges counted from the end: the last CTA holds the
+        // last rows of every level
         int per = (ncand + CS - 1) / CS;
-        int r0 = min(ncand, rank * per), r1 = min(ncand, r0 + per);
-        if (tid == 0) {
+        int r0 = max(0, ncand - (CS - rank) * per), r1 = max(0, ncand - (CS - 1 - rank) * per);
+        if (app && ncand >= 1 && ncand - 1 <= (CS - 1) * MY) {
+            // fused step: the appending CTA takes only the right-edge row (it
+            // appends first), the others share the rest
+            const int per1 = (ncand - 1 + CS - 2) / (CS - 1);
+            r0 = rank == CS - 1 ? ncand - 1 : min(ncand - 1, rank * per1);
+            r1 = rank == CS - 1 ? ncand : min(ncand - 1, r0 + per1);
+        }
+        // Fused step. The appending CTA holds the last rows of this level,
+        // the only ones the append changes: its tiles are requested now, like
+        // every CTA's, into a place after the pooler and the append scratch
+        // (when they fit), and the refreshed right-edge row is written over
+        // the copied one once the tile has landed. The other CTAs read the
+        // right edge only after the first selection barrier, which this CTA
+        // reaches after the append.
+        // [pooler | append scratch | patch rows: key, value | first tiles]
+        auto patch_rows = [&]() {
+            return reinterpret_cast<T*>(
+                smem_raw + ((D * D * sizeof(T) + append_scratch_floats(D, p.J_cap) * 4 + 127) & ~(size_t)127));
+        };
+        const size_t tiles_off = ((reinterpret_cast<unsigned char*>(patch_rows() + 2 * D) - smem_raw) + 127) & ~(size_t)127;
+        const bool early = appender && tiles_off + 2 * (size_t)(r1 - r0) * D * sizeof(T) <= (size_t)a.region0;
+        if (early) {
+            Kt = reinterpret_cast<T*>(smem_raw + tiles_off);
+            Vt = Kt + (size_t)(r1 - r0) * D;
+        }
+        if (tid == 0 && (!appender || early)) {
             issue(0, j, r0, r1);
             issue(1, j, r0, r1);
+        }
+        int patch_row = -1;  // row of this CTA's first tiles to overwrite
+        if (appender) {
+            const int jf = j;
+            const T* kn = reinterpret_cast<const T*>(a.k_new) + u * D;
+            const T* vn = reinterpret_cast<const T*>(a.v_new) + u * D;
+            const bool ok = append_token<T, D>(
+                p, u, Lraw, kn, vn, reinterpret_cast<const T*>(smem_raw),
+                reinterpret_cast<float*>(smem_raw + D * D * sizeof(T)),
+                [&]() {
+                    const int timed_out = !mbar_wait(&sm->bar[2], 0);
+                    if (__syncthreads_or(timed_out)) {
+                        if (tid == 0) flag_error(p.err, ERR_TIMEOUT);
+                        return false;
+                    }
+                    return true;
+                },
+                [&](int jj, T ky, T vy) {
+                    if (jj == jf) {
+                        patch_rows()[tid] = ky;
+                        patch_rows()[D + tid] = vy;
+                    }
+                });
+            if (jf == 0 && tid < D) {  // the first scored level is the tokens: the new one
+                patch_rows()[tid] = kn[tid];
+                patch_rows()[D + tid] = vn[tid];
+            }
+            appended = ok;
+            if (!ok) bad = true;
+            fence_proxy_async_global();  // this CTA's writes, before its own bulk reads
+            __syncthreads();             // pooler, scratch and patch rows in place
+            if (early)
+                patch_row = ncand - 1 - r0;
+            else if (tid == 0) {
+                issue(0, j, r0, r1);
+                issue(1, j, r0, r1);
+            }
         }
         for (;;) {
             const int nmy = r1 - r0;
             const int P = ncand > 0 ? ncand - 1 : 0;  // query position at this level
             wait_tile(0);
+            if (patch_row >= 0) {
+                if (tid < D) Kt[(size_t)patch_row * D + tid] = patch_rows()[tid];
+                __syncthreads();
+            }
             krows += ncand;
-            // Scoring. A group of LPC lanes takes one candidate, PL rotation
-            // pairs per lane. Index r*b + o: the key is rotated by o, the query
-            // by P - r*b (angle difference), so the key needs one small table
-            // row and the query is re-rotated only when the block r changes.
-            {
-                const int grp = lane / LPC, gl = lane % LPC;
-                const int chunk = (nmy + W - 1) / W;
-                const int w_lo = warp * chunk, w_hi = min(nmy, w_lo + chunk);
-                constexpr int P2 = PL / 2;
-                float2 qa2[G][P2], qb2[G][P2];
-                int rcur = -1;
-                for (int base = w_lo; base < w_hi; base += CPW) {
-                    const int i = base + grp;
-                    float v[G];
-#pragma unroll
-                    for (int g = 0; g < G; g++) v[g] = 0.f;
-                    if (i < w_hi) {
-                        const int rnk = r0 + i, r = rnk / b, o = rnk - r * b;
-                        if (r != rcur) {  // query rotated by P - r*b
-                            const float* row = p.rope + (size_t)(P - r * b) * 3 * HD + gl * PL;
-                            float2 c2[P2], s2[P2], n2[P2];
-                            load_tab2<PL>(row, c2);
-                            load_tab2<PL>(row + HD, s2);
-                            load_tab2<PL>(row + 2 * HD, n2);
-#pragma unroll
-                            for (int g = 0; g < G; g++)
-#pragma unroll
-                                for (int x = 0; x < P2; x++) {
-                                    const float2 xa = make_float2(qf[g * D + gl * PL + 2 * x], qf[g * D + gl * PL + 2 * x + 1]);
-                                    const float2 xb = make_float2(qf[g * D + HD + gl * PL + 2 * x],
-                                                                  qf[g * D + HD + gl * PL + 2 * x + 1]);
-                                    qa2[g][x] = ffma2(xa, c2[x], fmul2(xb, n2[x]));
-                                    qb2[g][x] = ffma2(xb, c2[x], fmul2(xa, s2[x]));
-                                }
-                            rcur = r;
-                        }
-                        // key rotated by o
-                        const float* row = p.rope + (size_t)o * 3 * HD + gl * PL;
-                        float2 c2[P2], s2[P2], n2[P2], ka[P2], kb[P2];
-                        load_tab2<PL>(row, c2);
-                        load_tab2<PL>(row + HD, s2);
-                        load_tab2<PL>(row + 2 * HD, n2);
-                        load_row2<T, PL>(Kt + (size_t)i * D + gl * PL, ka);
-                        load_row2<T, PL>(Kt + (size_t)i * D + HD + gl * PL, kb);
-                        float2 v2[G];
-#pragma unroll
-                        for (int g = 0; g < G; g++) v2[g] = make_float2(0.f, 0.f);
-#pragma unroll
-                        for (int x = 0; x < P2; x++) {
-                            const float2 ra = ffma2(ka[x], c2[x], fmul2(kb[x], n2[x]));
-                            const float2 rb = ffma2(kb[x], c2[x], fmul2(ka[x], s2[x]));
-#pragma unroll
-                            for (int g = 0; g < G; g++) v2[g] = ffma2(qa2[g][x], ra, ffma2(qb2[g][x], rb, v2[g]));
-                        }
-#pragma unroll
-                        for (int g = 0; g < G; g++) v[g] = v2[g].x + v2[g].y;
+            // logits of this CTA's rows, each warp's largest logit per head,
+            // selection keys (score, node id)
+            score_rows<T, D, G, W>(p.rope, p.scale, b, Kt, qf, r0, nmy, P, warp, lane, sm->red[warp],
+                                   [&](int i, int h, float logit, float S, int r, int o) {
+                                       lg[i * G + h] = logit;
+                                       if (h == 0 && j > 0) key[i] = sel_key(S, sm->par[r] * b + o);
+                                   });
+            const int kk = max(1, min(p.k, ncand));
+            const int chunk = (nmy + W - 1) / W;  // rows per warp, as in the scoring
+            if (j > 0) {  // each warp's top keys, sorted (its own rows: a warp barrier suffices)
+                __syncwarp();
+                const int w_lo = warp * chunk, nw = max(0, min(nmy, w_lo + chunk) - w_lo);
+                unsigned long long* wl = sm->wl[warp];
+                if (chunk <= 32) {
+                    unsigned long long x = lane < nw ? key[w_lo + lane] : 0ull;
+                    x = warp_sort_desc(x, lane);
+                    if (lane < kk) wl[lane] = x;
+                    for (int y = 32 + lane; y < kk; y += 32) wl[y] = 0ull;
+                } else {
+                    for (int e = lane; e < nw; e += 32) {
+                        const unsigned long long kt = key[w_lo + e];
+                        const int c = rank_among(key + w_lo, nw, kt);
+                        if (c < kk) wl[c] = kt;
                     }
-                    // reduce over the group's lanes; transposing while G > 1 value
-                    int cnt = G, h = 0, tbits = 0;
-#pragma unroll
-                    for (int sft = LPC / 2; sft >= 1; sft >>= 1) {
-                        if (cnt > 1) {
-                            const int half = cnt / 2;
-                            const bool hi = (gl & sft) != 0;
-#pragma unroll
-                            for (int x = 0; x < G / 2; x++) {
-                                if (x < half) {
-                                    const float send = hi ? v[x] : v[x + half];
-                                    const float keep = hi ? v[x + half] : v[x];
-                                    v[x] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
-                                }
-                            }
-                            h += hi ? half : 0;
-                            tbits |= sft;
-                            cnt = half;
-                        } else {
-                            v[0] += __shfl_xor_sync(0xffffffffu, v[0], sft);
-                        }
-                    }
-                    const float logit = v[0] * p.scale;
-                    float S = logit;
-#pragma unroll
-                    for (int sft = LPC / 2; sft >= 1; sft >>= 1)
-                        if (tbits & sft) S += __shfl_xor_sync(0xffffffffu, S, sft);
-                    if (i < w_hi && (gl & ~tbits) == 0) {
-                        lg[h * MY + i] = logit;
-                        if (h == 0 && j > 0) {
-                            const int rnk = r0 + i, q = rnk / b;
-                            key[i] = sel_key(S, sm->par[q] * b + (rnk - q * b));
-                        }
-                    }
+                    for (int x = nw + lane; x < kk; x += 32) wl[x] = 0ull;
                 }
             }
-            __syncthreads();  // logits and keys of every warp in place; key tile free
+            __syncthreads();  // logits, keys and warp lists in place; key tile free
 
             if (j == 0) {
                 wait_tile(1);
+                if (patch_row >= 0) {
+                    if (tid < D) Vt[(size_t)patch_row * D + tid] = patch_rows()[D + tid];
+                    __syncthreads();
+                }
                 accumulate(nmy, true);
                 vrows += ncand;
                 break;
             }
-            const int kk = max(1, min(p.k, ncand));
-            unsigned long long* mybuf = sm->topbuf[j & 1];
-            // local top-kk: each key's rank among this CTA's keys (two threads per key)
-            for (int base2 = warp * 32; base2 < 2 * nmy; base2 += DEC_THREADS) {
-                const int x = base2 + lane, e = x >> 1, half = x & 1;
-                const bool act = x < 2 * nmy;
-                const unsigned long long kt = act ? key[e] : 0ull;
-                const int lo = half ? nmy / 2 : 0, hi = half ? nmy : nmy / 2;
-                int c = act ? rank_among(key + lo, hi - lo, kt) : 0;
-                c += __shfl_xor_sync(0xffffffffu, c, 1);
-                if (act && half == 0 && c < kk) mybuf[c] = kt;
+            // this CTA's top keys, written to slot `rank` of every CTA's list
+            // area for this level
+            unsigned long long* gk = gkeys + (j & 1) * (DEC_CLUSTER * KMAX);
+            for (int t = tid; t < W * kk; t += DEC_THREADS) {
+                const unsigned long long x = sm->wl[t / kk][t % kk];
+                if (x == 0ull) continue;
+                const int c = rank_in_lists<W>(&sm->wl[0][0], KMAX, kk, x);
+                if (c < kk)
+                    for (int r = 0; r < CS; r++) cluster.map_shared_rank(gk, r)[rank * KMAX + c] = x;
             }
-            if (tid >= nmy && tid < kk) mybuf[tid] = 0ull;
+            for (int t = nmy + tid; t < kk; t += DEC_THREADS)  // fewer rows than kk
+                for (int r = 0; r < CS; r++) cluster.map_shared_rank(gk, r)[rank * KMAX + t] = 0ull;
             cluster.sync();
-            // global top-kk: merge the CTAs' sorted lists (same result in every CTA)
-            const int total = CS * kk;
-            for (int t = tid; t < total; t += DEC_THREADS)
-                gkeys[t] = cluster.map_shared_rank(mybuf, t / kk)[t % kk];
-            __syncthreads();
-            for (int base2 = warp * 32; base2 < 2 * total; base2 += DEC_THREADS) {
-                const int x = base2 + lane, t = x >> 1, half = x & 1;
-                const bool act = x < 2 * total;
-                const unsigned long long kt = act ? gkeys[t] : 0ull;
-                const int lo = half ? total / 2 : 0, hi = half ? total : total / 2;
-                int c = (act && kt != 0ull) ? rank_among(gkeys + lo, hi - lo, kt) : 0;
-                c += __shfl_xor_sync(0xffffffffu, c, 1);
-                if (act && half == 0 && kt != 0ull && c < kk) sm->picked[c] = kt;
+            // global top-kk (the same in every CTA) and the kept ids in
+            // ascending order (ids are distinct)
+            for (int t = tid; t < CS * kk; t += DEC_THREADS) {
+                const unsigned long long x = gk[(t / kk) * KMAX + t % kk];
+                if (x == 0ull) continue;
+                const int c = rank_in_lists<DEC_CLUSTER>(gk, KMAX, kk, x);
+                if (c < kk) sm->picked[c] = x;
             }
             __syncthreads();
-            if (tid < kk) {  // kept ids in ascending order (ids are distinct)
+            if (tid < kk) {
                 const int id = (int)key_id(sm->picked[tid]);
                 int pos = 0;
                 for (int r = 0; r < kk; r++) pos += (int)key_id(sm->picked[r]) < id;
@@ -452,8 +504,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
             }
             if (tid == 0) sm->thresh = sm->picked[kk - 1];
             __syncthreads();
-            if (rank == 0 && a.sel_out)
-                for (int x = tid; x < p.k; x += DEC_THREADS)
+            if (rank == 0 && a.sel_out)  // not thread 0: it issues the copies
+                for (int x = tid - 32; x >= 0 && x < p.k; x += DEC_THREADS - 32)
                     a.sel_out[(u * p.J_cap + (j - 1)) * p.k + x] = x < kk ? sm->chosen[x] : -1;
             if (tid < kk) sm->par[tid] = sm->chosen[tid];
             __syncthreads();
@@ -464,12 +516,19 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
                 if (tid == 0) flag_error(p.err, ERR_SHAPE);
             }
             const int per_n = (nc_next + CS - 1) / CS;
-            const int r0n = min(nc_next, rank * per_n), r1n = min(nc_next, r0n + per_n);
+            const int r0n = max(0, nc_next - (CS - rank) * per_n), r1n = max(0, nc_next - (CS - 1 - rank) * per_n);
+            Kt = reinterpret_cast<T*>(smem_raw);
             if (tid == 0) issue(0, j - 1, r0n, r1n);  // key tile is free since the barriers above
             wait_tile(1);
+            if (patch_row >= 0) {
+                if (tid < D) Vt[(size_t)patch_row * D + tid] = patch_rows()[D + tid];
+                __syncthreads();
+                patch_row = -1;
+            }
             accumulate(nmy, false);  // summaries of the candidates not kept
             vrows += ncand - kk;
             __syncthreads();         // value tile and weights consumed
+            Vt = reinterpret_cast<T*>(smem_raw) + (size_t)MY * D;
             if (tid == 0) issue(1, j - 1, r0n, r1n);
             npar = kk;
             j--;
@@ -514,6 +573,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
         for (int idx = tid; idx < G * D + 2 * G; idx += DEC_THREADS) dst[idx] = idx < G * D ? cacc[idx] : cml[idx - G * D];
     }
     cluster.sync();  // the gather area of rank 0 is complete
+    if (appended && tid == 0) p.len[u] = Lraw + 1;  // every CTA has read the old length
     if (rank == 0) {
         T* outp = reinterpret_cast<T*>(a.out) + (u * G) * D;
         const int stride = G * D + 2 * G;
@@ -546,13 +606,16 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
     }
 }
 
+// k_new, v_new: null for a decode alone; else the fused step (append the
+// token of every unit, then decode against the grown tree).
 template <typename T, int D, int G>
-cudaError_t launch_decode(const TreeParams& p, const void* q, void* out, int* sel_out, long long* rows_out,
-                          cudaStream_t s) {
+cudaError_t launch_decode(const TreeParams& p, const void* k_new, const void* v_new, const void* q, void* out,
+                          int* sel_out, long long* rows_out, cudaStream_t s) {
     const int CS = DEC_CLUSTER;
     const long long maxc = (long long)p.k * p.b > p.b ? (long long)p.k * p.b : p.b;
-    DecodeArgs a{q, out, sel_out, rows_out, (int)((maxc + CS - 1) / CS), 0};
-    a.region0 = (int)decode_region0(D, G, a.my_max, (int)sizeof(T));
+    const bool fused = k_new != nullptr;
+    DecodeArgs a{k_new, v_new, q, out, sel_out, rows_out, (int)((maxc + CS - 1) / CS), 0};
+    a.region0 = (int)decode_region0(D, G, a.my_max, (int)sizeof(T), p.J_cap, fused);
     const size_t smem = a.region0 + decode_smem_tail(D, G, a.my_max);
     auto kern = decode_kernel<T, D, G>;
     static bool attr_set = false;  // per instantiation
@@ -572,8 +635,8 @@ cudaError_t launch_decode(const TreeParams& p, const void* q, void* out, int* se
     attr[0].val.clusterDim.x = CS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    // may start while the previous kernel on the stream (the append) finishes;
-    // the kernel waits for it before reading the tree
+    // may start while the previous kernel on the stream finishes; the kernel
+    // waits for it before reading the tree
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
@@ -582,7 +645,8 @@ cudaError_t launch_decode(const TreeParams& p, const void* q, void* out, int* se
 }
 
 #define RECSA_INST_DEC(T, D, G) \
-    template cudaError_t launch_decode<T, D, G>(const TreeParams&, const void*, void*, int*, long long*, cudaStream_t);
+    template cudaError_t launch_decode<T, D, G>(const TreeParams&, const void*, const void*, const void*, void*, \
+                                                int*, long long*, cudaStream_t);
 #define RECSA_INST_DEC_G(T, D) RECSA_INST_DEC(T, D, 1) RECSA_INST_DEC(T, D, 2) RECSA_INST_DEC(T, D, 4) RECSA_INST_DEC(T, D, 8)
 RECSA_INST_DEC_G(float, 64)
 RECSA_INST_DEC_G(float, 128)

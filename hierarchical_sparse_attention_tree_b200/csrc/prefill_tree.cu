@@ -17,6 +17,7 @@
 // keys; the value rows of the candidates not kept are then streamed for the
 // softmax. Level-0 candidates are scored and accumulated tile by tile.
 #include "common.cuh"
+#include "score.cuh"
 
 namespace recsa {
 
@@ -64,12 +65,6 @@ __host__ __device__ inline size_t prefill_tree_tiles(int D, int G, int elem) {
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams p, PrefillTreeArgs a) {
-    constexpr int HD = D / 2;
-    constexpr int PL = 4;
-    constexpr int P2 = PL / 2;
-    constexpr int LPC = HD / PL;
-    constexpr int CPW = 32 / LPC;
-    static_assert(G <= LPC && 32 % LPC == 0 && G <= 8, "scoring layout");
     constexpr int NCC = D / PT_CPT, NEG = PT_THREADS / NCC;
     constexpr int W = PT_WARPS;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -169,92 +164,13 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
     };
 
     // Scores of tile rows [0, nmy) = candidate ranks [r0, r0 + nmy) with the
-    // query at index P: key rotated by (rank mod b), query by P - b*(rank / b).
+    // query at index P (logits, and the selection keys when want_keys).
     auto score_tile = [&](int r0, int nmy, int P, bool want_keys) {
-        const int grp = lane / LPC, gl = lane % LPC;
-        const int chunk = (nmy + W - 1) / W;
-        const int w_lo = warp * chunk, w_hi = min(nmy, w_lo + chunk);
-        float2 qa2[G][P2], qb2[G][P2];
-        int rcur = -1;
-        for (int base = w_lo; base < w_hi; base += CPW) {
-            const int i = base + grp;
-            float v[G];
-#pragma unroll
-            for (int g = 0; g < G; g++) v[g] = 0.f;
-            if (i < w_hi) {
-                const int rnk = r0 + i, r = rnk / b, o = rnk - r * b;
-                if (r != rcur) {
-                    const float* row = p.rope + (size_t)(P - r * b) * 3 * HD + gl * PL;
-                    float2 c2[P2], s2[P2], n2[P2];
-                    load_tab2<PL>(row, c2);
-                    load_tab2<PL>(row + HD, s2);
-                    load_tab2<PL>(row + 2 * HD, n2);
-#pragma unroll
-                    for (int g = 0; g < G; g++)
-#pragma unroll
-                        for (int x = 0; x < P2; x++) {
-                            const float2 xa = make_float2(qf[g * D + gl * PL + 2 * x], qf[g * D + gl * PL + 2 * x + 1]);
-                            const float2 xb = make_float2(qf[g * D + HD + gl * PL + 2 * x],
-                                                          qf[g * D + HD + gl * PL + 2 * x + 1]);
-                            qa2[g][x] = ffma2(xa, c2[x], fmul2(xb, n2[x]));
-                            qb2[g][x] = ffma2(xb, c2[x], fmul2(xa, s2[x]));
-                        }
-                    rcur = r;
-                }
-                const float* row = p.rope + (size_t)o * 3 * HD + gl * PL;
-                float2 c2[P2], s2[P2], n2[P2], ka[P2], kb[P2];
-                load_tab2<PL>(row, c2);
-                load_tab2<PL>(row + HD, s2);
-                load_tab2<PL>(row + 2 * HD, n2);
-                load_row2<T, PL>(Kt + (size_t)i * D + gl * PL, ka);
-                load_row2<T, PL>(Kt + (size_t)i * D + HD + gl * PL, kb);
-                float2 v2[G];
-#pragma unroll
-                for (int g = 0; g < G; g++) v2[g] = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int x = 0; x < P2; x++) {
-                    const float2 ra = ffma2(ka[x], c2[x], fmul2(kb[x], n2[x]));
-                    const float2 rb = ffma2(kb[x], c2[x], fmul2(ka[x], s2[x]));
-#pragma unroll
-                    for (int g = 0; g < G; g++) v2[g] = ffma2(qa2[g][x], ra, ffma2(qb2[g][x], rb, v2[g]));
-                }
-#pragma unroll
-                for (int g = 0; g < G; g++) v[g] = v2[g].x + v2[g].y;
-            }
-            int cnt = G, hh = 0, tbits = 0;
-#pragma unroll
-            for (int sft = LPC / 2; sft >= 1; sft >>= 1) {
-                if (cnt > 1) {
-                    const int half = cnt / 2;
-                    const bool hi = (gl & sft) != 0;
-#pragma unroll
-                    for (int x = 0; x < G / 2; x++) {
-                        if (x < half) {
-                            const float send = hi ? v[x] : v[x + half];
-                            const float keep = hi ? v[x + half] : v[x];
-                            v[x] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
-                        }
-                    }
-                    hh += hi ? half : 0;
-                    tbits |= sft;
-                    cnt = half;
-                } else {
-                    v[0] += __shfl_xor_sync(0xffffffffu, v[0], sft);
-                }
-            }
-            const float logit = v[0] * p.scale;
-            float Ssum = logit;
-#pragma unroll
-            for (int sft = LPC / 2; sft >= 1; sft >>= 1)
-                if (tbits & sft) Ssum += __shfl_xor_sync(0xffffffffu, Ssum, sft);
-            if (i < w_hi && (gl & ~tbits) == 0) {
-                lg[hh * MC + r0 + i] = logit;
-                if (hh == 0 && want_keys) {
-                    const int rnk = r0 + i, q = rnk / b;
-                    key[r0 + i] = sel_key(Ssum, sm->par[q] * b + (rnk - q * b));
-                }
-            }
-        }
+        score_rows<T, D, G, W>(p.rope, p.scale, b, Kt, qf, r0, nmy, P, warp, lane, nullptr,
+                               [&](int i, int hh, float logit, float Ssum, int r, int o) {
+                                   lg[hh * MC + r0 + i] = logit;
+                                   if (hh == 0 && want_keys) key[r0 + i] = sel_key(Ssum, sm->par[r] * b + o);
+                               });
     };
 
     // Entries of tile rows [0, nmy) (ranks r0..) join the CTA's softmax:

@@ -17,6 +17,7 @@
 //              last node but its last child, so an append only adds the
 //              completed child and the new last child.
 #include "common.cuh"
+#include "append.cuh"
 
 namespace recsa {
 
@@ -143,17 +144,28 @@ __global__ void __launch_bounds__(256) build_level_kernel(TreeParams p, int j, l
 #pragma unroll
     for (int e = 0; e < DPL; e++) kmw[lane * DPL + e] = __fdiv_rn(ks[e], fnc);
     __syncwarp();
+    // the pooler product as the append computes it: one fmaf chain per
+    // quarter of the input coordinate, then (y0 + y1) + (y2 + y3)
+    constexpr int Q = D / 4;
+    float y4[4][DPL];
+#pragma unroll
+    for (int q = 0; q < 4; q++)
+#pragma unroll
+        for (int e = 0; e < DPL; e++) y4[q][e] = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < Q; c++) {
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            const float x = kmw[q * Q + c];
+            float w[DPL];
+            load_vec<T, DPL>(Wt + (q * Q + c) * D + lane * DPL, w);
+#pragma unroll
+            for (int e = 0; e < DPL; e++) y4[q][e] = fmaf(w[e], x, y4[q][e]);
+        }
+    }
     float y[DPL];
 #pragma unroll
-    for (int e = 0; e < DPL; e++) y[e] = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < D; c++) {
-        const float x = kmw[c];
-        float w[DPL];
-        load_vec<T, DPL>(Wt + c * D + lane * DPL, w);
-#pragma unroll
-        for (int e = 0; e < DPL; e++) y[e] = fmaf(w[e], x, y[e]);
-    }
+    for (int e = 0; e < DPL; e++) y[e] = (y4[0][e] + y4[1][e]) + (y4[2][e] + y4[3][e]);
     T* k_out = reinterpret_cast<T*>(p.K[j]) + (u * p.rows[j] + m) * D + lane * DPL;
     store_vec<T, DPL>(k_out, y);
 }
@@ -161,118 +173,41 @@ __global__ void __launch_bounds__(256) build_level_kernel(TreeParams p, int j, l
 // ----------------------------------------------------------- append one
 
 // Appends one token per unit and refreshes the right edge of every level.
-// One CTA of D threads per unit; thread t owns coordinate t. Every global
-// load that does not depend on this call's results (the pooler, the prefix
-// sums, the child that completed at this token) is issued before the level
-// chain starts, so the chain itself touches only shared memory and registers.
+// One CTA of D threads per unit; the pooler comes into shared memory by one
+// bulk async copy while the per-level loads are in flight.
 template <typename T, int D>
 __global__ void __launch_bounds__(D) append_one_kernel(TreeParams p, const T* __restrict__ k_new,
                                                        const T* __restrict__ v_new) {
     extern __shared__ __align__(128) unsigned char smem_a[];
-    T* Wt = reinterpret_cast<T*>(smem_a);                                  // [D][D]
-    float* km = reinterpret_cast<float*>(smem_a + D * D * sizeof(T));     // [D]
-    float* pre = km + D;                                                   // [J_cap][4][D]: pk, pv, kold, vold
+    T* Wt = reinterpret_cast<T*>(smem_a);                                   // [D][D]
+    float* scratch = reinterpret_cast<float*>(smem_a + D * D * sizeof(T));  // append_scratch_floats
     __shared__ uint64_t wbar;
-    const int t = threadIdx.x;
     const long long u = blockIdx.x;
-    const int bseq = (int)(u / p.H), h = (int)(u % p.H);
     // the next kernel on the stream (a decode) may start its own set-up now
     asm volatile("griddepcontrol.launch_dependents;");
     const long long P = p.len[u];  // position of the new token
     if (P >= p.cap) {
-        if (t == 0) flag_error(p.err, ERR_LENGTH);
+        if (threadIdx.x == 0) flag_error(p.err, ERR_LENGTH);
         return;
     }
-    // pooler -> shared memory: one bulk async copy
-    if (t == 0) {
+    if (threadIdx.x == 0) {
         mbar_init(&wbar, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(&wbar, (uint32_t)(D * D * sizeof(T)));
         bulk_g2s(Wt, p.Wt, (uint32_t)(D * D * sizeof(T)), &wbar);
     }
-    const long long src = ((long long)bseq * p.H + h) * D + t;  // [B][1][H][D]
-    const T kn = k_new[src], vn = v_new[src];
-    T* Kt = reinterpret_cast<T*>(p.K[0]) + u * p.cap * D;
-    T* Vt = reinterpret_cast<T*>(p.V[0]) + u * p.cap * D;
-    // per level j: prefix sums of the right edge and, if a child of level j-1
-    // completed at this token, that child's stored key and value sum
-    auto load_level = [&](int j, float& pk, float& pv, float& ko, float& vo) {
-        pk = pv = ko = vo = 0.f;
-        if (j > p.J_cap) return;
-        const long long sj = p.span[j], sjm = p.span[j - 1];
-        if ((P % sj) == 0) return;  // a new node starts at this token
-        pk = p.PK[j][u * D + t];
-        pv = p.PV[j][u * D + t];
-        if ((P % sjm) == 0) {
-            const long long c = P / sjm - 1;  // completed child of level j-1
-            if (j == 1) {
-                ko = to_f(Kt[c * D + t]);
-                vo = to_f(Vt[c * D + t]);
-            } else {
-                const long long row = u * p.rows[j - 1] + c;
-                ko = to_f(reinterpret_cast<const T*>(p.K[j - 1])[row * D + t]);
-                vo = p.VS[j - 1][row * D + t];
+    const bool ok = append_token<T, D>(
+        p, u, P, k_new + u * D, v_new + u * D, Wt, scratch,
+        [&]() {
+            const int timed_out = !mbar_wait(&wbar, 0);
+            if (__syncthreads_or(timed_out)) {  // same decision in every thread
+                if (threadIdx.x == 0) flag_error(p.err, ERR_TIMEOUT);
+                return false;
             }
-        }
-    };
-    constexpr int JU = 6;  // levels whose loads are all issued together
-    {
-        float r[JU][4];
-#pragma unroll
-        for (int jj = 0; jj < JU; jj++) load_level(jj + 1, r[jj][0], r[jj][1], r[jj][2], r[jj][3]);
-#pragma unroll
-        for (int jj = 0; jj < JU; jj++)
-            if (jj + 1 <= p.J_cap)
-#pragma unroll
-                for (int x = 0; x < 4; x++) pre[((size_t)jj * 4 + x) * D + t] = r[jj][x];
-    }
-    for (int j = JU + 1; j <= p.J_cap; j++) {
-        float r4[4];
-        load_level(j, r4[0], r4[1], r4[2], r4[3]);
-        for (int x = 0; x < 4; x++) pre[((size_t)(j - 1) * 4 + x) * D + t] = r4[x];
-    }
-    Kt[P * D + t] = kn;
-    Vt[P * D + t] = vn;
-    const int timed_out = !mbar_wait(&wbar, 0);
-    if (__syncthreads_or(timed_out)) {  // same decision in every thread
-        if (t == 0) flag_error(p.err, ERR_TIMEOUT);
-        return;  // no node has been written yet; the length stays
-    }
-
-    float kcur = to_f(kn), vcur = to_f(vn);  // new last child of level j-1
-    for (int j = 1; j <= p.J_cap; j++) {
-        const long long sj = p.span[j], sjm = p.span[j - 1];
-        const long long m = P / sj;
-        const bool new_node = (P % sj) == 0;
-        const bool child_done = (P % sjm) == 0;
-        const float* q4 = pre + (size_t)(j - 1) * 4 * D;
-        float pk = q4[t], pv = q4[D + t];
-        if (!new_node && child_done) {
-            pk = pk + q4[2 * D + t];
-            pv = pv + q4[3 * D + t];
-        }
-        if (new_node || child_done) {
-            p.PK[j][u * D + t] = pk;
-            p.PV[j][u * D + t] = pv;
-        }
-        const float ks = pk + kcur, vsum = pv + vcur;
-        const long long cnt = P + 1 - m * sj;
-        const long long nc = P / sjm - m * p.b + 1;
-        const long long row = u * p.rows[j] + m;
-        p.VS[j][row * D + t] = vsum;
-        reinterpret_cast<T*>(p.V[j])[row * D + t] = from_f<T>(__fdiv_rn(vsum, (float)cnt));
-        km[t] = __fdiv_rn(ks, (float)nc);
-        __syncthreads();
-        float y = 0.f;
-#pragma unroll 16
-        for (int c = 0; c < D; c++) y = fmaf(to_f(Wt[c * D + t]), km[c], y);
-        const T ky = from_f<T>(y);
-        reinterpret_cast<T*>(p.K[j])[row * D + t] = ky;
-        kcur = to_f(ky);
-        vcur = vsum;
-        __syncthreads();
-    }
-    if (t == 0) p.len[u] = P + 1;
+            return true;
+        },
+        [](int, T, T) {});
+    if (ok && threadIdx.x == 0) p.len[u] = P + 1;
 }
 
 // --------------------------------------------------------------- launch
@@ -294,7 +229,7 @@ cudaError_t launch_build_level(const TreeParams& p, int j, long long add, int fr
 
 template <typename T, int D>
 cudaError_t launch_append_one(const TreeParams& p, const void* k_new, const void* v_new, cudaStream_t s) {
-    size_t smem = (size_t)D * D * sizeof(T) + (size_t)(D + 4 * p.J_cap * D) * sizeof(float);
+    size_t smem = (size_t)D * D * sizeof(T) + append_scratch_floats(D, p.J_cap) * sizeof(float);
     auto kern = append_one_kernel<T, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -43,6 +43,14 @@ class RecsaLayer:
         self.ctx.decode(q, out, sel_out, rows_out, stream)
         return out
 
+    def append_decode(self, k_new, v_new, q, out=None, sel_out=None, rows_out=None, stream=None):
+        """One decode step in one launch: append k_new, v_new [B][1][H_kv][d],
+        then attend q [B][H_q][d] over the grown tree."""
+        if out is None:
+            out = torch.empty_like(q)
+        self.ctx.append_decode(k_new, v_new, q, out, sel_out, rows_out, stream)
+        return out
+
     def prefill(self, q, k, v, out=None, sel_out=None, stream=None):
         if out is None:
             out = torch.empty_like(q)

@@ -19,7 +19,7 @@ F32, BF16 = 0, 1
 _TORCH_DTYPE = {F32: torch.float32, BF16: torch.bfloat16}
 
 EXPORTS = [
-    "recsa_workspace_bytes", "recsa_init", "recsa_build_tree", "recsa_append", "recsa_decode",
+    "recsa_workspace_bytes", "recsa_init", "recsa_build_tree", "recsa_append", "recsa_decode", "recsa_append_decode",
     "recsa_prefill_scratch_bytes", "recsa_prefill", "recsa_get_lengths", "recsa_tree_shape", "recsa_level_arrays",
     "recsa_check_device", "recsa_last_error", "recsa_destroy", "recsa_dense_decode_scratch_bytes",
     "recsa_dense_decode", "recsa_dense_decode_static",
@@ -57,6 +57,7 @@ def lib():
             "recsa_build_tree": (i32, [vp, P(i64), vp]),
             "recsa_append": (i32, [vp, vp, vp, i32, vp]),
             "recsa_decode": (i32, [vp, vp, vp, vp, vp, vp]),
+            "recsa_append_decode": (i32, [vp, vp, vp, vp, vp, vp, vp, vp]),
             "recsa_prefill_scratch_bytes": (sz, [P(Config), i32]),
             "recsa_prefill": (i32, [vp, vp, vp, vp, i32, vp, vp, vp, sz, vp]),
             "recsa_get_lengths": (i32, [vp, P(i64)]),
@@ -162,6 +163,10 @@ class Context:
 
     def decode(self, q, out, sel_out=None, rows_out=None, stream=None):
         _check(lib().recsa_decode(self.handle, _ptr(q), _ptr(out), _ptr(sel_out), _ptr(rows_out), _stream(stream)))
+
+    def append_decode(self, k_new, v_new, q, out, sel_out=None, rows_out=None, stream=None):
+        _check(lib().recsa_append_decode(self.handle, _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(out), _ptr(sel_out),
+                                         _ptr(rows_out), _stream(stream)))
 
     def prefill(self, q, k, v, out, sel_out=None, scratch=None, stream=None):
         C = q.shape[1]

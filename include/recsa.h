@@ -116,6 +116,15 @@ recsa_status recsa_append(recsa_ctx* ctx, const void* k_new, const void* v_new, 
 recsa_status recsa_decode(recsa_ctx* ctx, const void* q, void* out, int* sel_out, long long* rows_out,
                           recsa_stream_t stream);
 
+/* One decode step in a single launch: appends one token per sequence (as
+ * recsa_append with n = 1, same node arithmetic) and decodes q against the
+ * grown tree (as recsa_decode). k_new, v_new [B][1][H_kv][d], q, out
+ * [B][H_q][d] (device, 16-byte aligned); sel_out and rows_out as in
+ * recsa_decode. RECSA_ERR_CAPACITY (nothing launched) if a sequence is full.
+ * The appended token is the one q belongs to: the query attends it. */
+recsa_status recsa_append_decode(recsa_ctx* ctx, const void* k_new, const void* v_new, const void* q, void* out,
+                                 int* sel_out, long long* rows_out, recsa_stream_t stream);
+
 /* Chunked causal prefill of C tokens per sequence (1 <= C <= max_chunk):
  * token t of the chunk attends the tree over the sequence's cached tokens
  * [0, s) plus the chunk's own tokens s..t exactly; those follow the level-0

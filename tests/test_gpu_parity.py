@@ -145,7 +145,7 @@ def test_tiny_f32_build_and_decode():
 # -------------------------------------------------- bf16, several units
 
 
-@pytest.mark.parametrize("D,G", [(128, 4), (64, 2), (128, 1), (64, 8)])
+@pytest.mark.parametrize("D,G", [(128, 4), (64, 2), (128, 1), (64, 8), (128, 8)])
 def test_bf16_ragged_batch(D, G):
     w = small(batch=3, n_kv_heads=2, group=G, head_dim=D, branching=8, k=3)
     lengths = [1, 517, 3001]
@@ -157,6 +157,21 @@ def test_bf16_ragged_batch(D, G):
         q = per_seq_queries(w, runs, s, lengths)
         gout, gsel, grows = run_decode(layer, w, q)
         check_units(layer, w, K, V, Wp, lengths, q, gout, gsel, grows)
+
+
+@pytest.mark.parametrize("k,L", [(24, 20000), (40, 200000)])
+def test_large_k_selection(k, L):
+    """k > 16: the CTA and cluster top-k are merged by rank search; at
+    L = 200000 (b = 64, k = 40) a CTA holds 320 level-1 rows, more than 32 per
+    warp, so each warp ranks its rows instead of sorting them in registers."""
+    w = small(batch=1, n_kv_heads=2, group=4, head_dim=128, branching=64, k=k)
+    K, V, runs = synth.cache_arrays(w, L)
+    layer, Wp = make_layer(w, L)
+    layer.load(parity.to_dev(K, True), parity.to_dev(V, True), [L])
+    for s in range(2):
+        q = per_seq_queries(w, runs, s, [L])
+        gout, gsel, grows = run_decode(layer, w, q)
+        check_units(layer, w, K, V, Wp, [L], q, gout, gsel, grows, free=False)
 
 
 def test_f32_d128_matches_free_oracle():
@@ -245,6 +260,66 @@ def test_append_matches_rebuild_bitwise(bf16):
     q = per_seq_queries(w, runs, 0, pos)
     gout, gsel, grows = run_decode(inc, w, q)
     check_units(inc, w, K, V, Wp, pos, q, gout, gsel, grows, free_exact=not bf16)
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_fused_append_decode(bf16):
+    """recsa_append_decode (one launch per step) leaves the node arrays and
+    returns the selections and row counts of recsa_append then recsa_decode,
+    bit for bit, across node and level boundaries (sequence 1 grows from 61
+    past 64 = b^3 tokens). The outputs agree to rounding: the fused launch
+    splits the first level's rows differently over the cluster, so the
+    per-CTA softmax sums are added in another order. The last step also
+    matches the oracle."""
+    w = small(batch=2, n_kv_heads=2, group=4, head_dim=128, branching=4, k=2, bf16=bf16)
+    start = [30, 61]
+    steps = 40
+    cap = max(start) + steps
+    K, V, runs = synth.cache_arrays(w, cap)
+    Kd, Vd = parity.to_dev(K, bf16), parity.to_dev(V, bf16)
+    fused, Wp = make_layer(w, cap)
+    split, _ = make_layer(w, cap)
+    K0, V0 = Kd.clone(), Vd.clone()
+    for b in range(w.batch):
+        K0[b, :, start[b]:] = 0
+        V0[b, :, start[b]:] = 0
+    fused.load(K0.clone(), V0.clone(), start)
+    split.load(K0.clone(), V0.clone(), start)
+    J_cap, _ = fused.tree_shape()
+    pos = list(start)
+    for s in range(steps):
+        kn = torch.stack([Kd[b, :, pos[b]:pos[b] + 1] for b in range(w.batch)]).permute(0, 2, 1, 3).contiguous()
+        vn = torch.stack([Vd[b, :, pos[b]:pos[b] + 1] for b in range(w.batch)]).permute(0, 2, 1, 3).contiguous()
+        pos = [p + 1 for p in pos]
+        q_np = per_seq_queries(w, runs, s, pos)
+        q = parity.to_dev(q_np, bf16)
+        outs = []
+        for layer in (fused, split):
+            sel = torch.full((w.batch, w.n_kv_heads, J_cap, w.k), -7, dtype=torch.int32, device="cuda")
+            rows = torch.zeros((w.batch, w.n_kv_heads, 2), dtype=torch.int64, device="cuda")
+            if layer is fused:
+                out = layer.append_decode(kn, vn, q, sel_out=sel, rows_out=rows)
+            else:
+                layer.append(kn, vn)
+                out = layer.decode(q, sel_out=sel, rows_out=rows)
+            outs.append((out, sel, rows))
+        torch.cuda.synchronize()
+        assert torch.equal(outs[0][1], outs[1][1]) and torch.equal(outs[0][2], outs[1][2]), s
+        diff = (outs[0][0].float() - outs[1][0].float()).abs().max().item()
+        assert diff <= (1e-2 if bf16 else 1e-5), (s, diff)
+    fused.check()
+    split.check()
+    assert fused.lengths() == pos == split.lengths()
+    for j in range(1, J_cap + 1):
+        for x, y in zip(fused.level(j), split.level(j)):
+            for b in range(w.batch):
+                n_j = -(-pos[b] // w.branching ** j)
+                assert torch.equal(x[b, :, :n_j], y[b, :, :n_j]), (j, b)
+    for b in range(w.batch):
+        assert torch.equal(fused.k_cache[b, :, :pos[b]], Kd[b, :, :pos[b]])
+        assert torch.equal(fused.v_cache[b, :, :pos[b]], Vd[b, :, :pos[b]])
+    gout, gsel, grows = parity.to_f64(outs[0][0]), outs[0][1].cpu().numpy(), outs[0][2].cpu().numpy()
+    check_units(fused, w, K, V, Wp, pos, q_np, gout, gsel, grows, free_exact=not bf16)
 
 
 def test_capacity_and_argument_errors():

@@ -84,7 +84,7 @@ def test_prefill_small_multichunk():
     assert rep["checked"] > 300, rep
 
 
-@pytest.mark.parametrize("D,G", [(64, 2), (128, 1), (64, 8)])
+@pytest.mark.parametrize("D,G", [(64, 2), (128, 1), (64, 8), (128, 8)])
 def test_prefill_shapes(D, G):
     w = small(batch=1, n_kv_heads=2, group=G, head_dim=D, branching=4, k=2)
     _, _, _, _, _, rep = run_prefill(w, 300, 64, lambda ci, C: list(range(0, C, 5)) + [C - 1])
