@@ -60,11 +60,13 @@ __host__ __device__ inline size_t append_scratch_floats(int D, int J_cap) { retu
 // and must return the same answer in all of them). scratch: shared memory of
 // append_scratch_floats(D, J_cap) floats. on_node(j, key, value) runs in
 // thread t < D with coordinate t of the refreshed right-edge node of level j.
-// Returns false (nothing of the tree written) if the pooler did not arrive.
+// lv: the levels' addresses (load_levels), in shared memory. Returns false
+// (nothing of the tree written) if the pooler did not arrive.
 // With at least 2D threads the pooler product is split over two threads per
 // output coordinate (same arithmetic).
 template <typename T, int D, typename WaitW, typename OnNode>
-__device__ __forceinline__ bool append_token(const TreeParams& p, long long u, long long P, const T* k_row,
+__device__ __forceinline__ bool append_token(const TreeParams& p, const LevelRef* lv, long long u, long long P,
+                                             const T* k_row,
                                              const T* v_row, const T* Wsm, float* scratch, WaitW wait_w,
                                              OnNode on_node) {
     const int t = threadIdx.x;
@@ -74,28 +76,28 @@ __device__ __forceinline__ bool append_token(const TreeParams& p, long long u, l
     float* part = scratch + D;
     float* pre = scratch + 3 * D;
     T kn = from_f<T>(0.f), vn = from_f<T>(0.f);
-    T* K0 = reinterpret_cast<T*>(p.K[0]) + u * p.cap * D;
-    T* V0 = reinterpret_cast<T*>(p.V[0]) + u * p.cap * D;
+    T* K0 = reinterpret_cast<T*>(lv[0].K) + u * p.cap * D;
+    T* V0 = reinterpret_cast<T*>(lv[0].V) + u * p.cap * D;
     // per level j: prefix sums of the right edge and, if a child of level
     // j-1 completed at this token, that child's stored key and value sum
     auto load_level = [&](int j, float& pk, float& pv, float& ko, float& vo) {
         pk = pv = ko = vo = 0.f;
         if (j > p.J_cap) return;
         long long qj, rj, qm, rm;
-        divmod_pos(P, p.span[j], qj, rj);
-        divmod_pos(P, p.span[j - 1], qm, rm);
+        divmod_pos(P, lv[j].span, qj, rj);
+        divmod_pos(P, lv[j - 1].span, qm, rm);
         if (rj == 0) return;  // a new node starts at this token
-        pk = p.PK[j][u * D + t];
-        pv = p.PV[j][u * D + t];
+        pk = lv[j].PK[u * D + t];
+        pv = lv[j].PV[u * D + t];
         if (rm == 0) {
             const long long c = qm - 1;  // completed child of level j-1
             if (j == 1) {
                 ko = to_f(K0[c * D + t]);
                 vo = to_f(V0[c * D + t]);
             } else {
-                const long long row = u * p.rows[j - 1] + c;
-                ko = to_f(reinterpret_cast<const T*>(p.K[j - 1])[row * D + t]);
-                vo = p.VS[j - 1][row * D + t];
+                const long long row = u * lv[j - 1].rows + c;
+                ko = to_f(reinterpret_cast<const T*>(lv[j - 1].K)[row * D + t]);
+                vo = lv[j - 1].VS[row * D + t];
             }
         }
     };
@@ -125,13 +127,13 @@ __device__ __forceinline__ bool append_token(const TreeParams& p, long long u, l
 
     float kcur = to_f(kn), vcur = to_f(vn);  // new last child of level j-1
     for (int j = 1; j <= p.J_cap; j++) {
-        const long long sj = p.span[j];
+        const long long sj = lv[j].span;
         long long m, rj, qm, rm;
         divmod_pos(P, sj, m, rj);
-        divmod_pos(P, p.span[j - 1], qm, rm);
+        divmod_pos(P, lv[j - 1].span, qm, rm);
         const bool new_node = rj == 0;
         const bool child_done = rm == 0;
-        const long long row = u * p.rows[j] + m;
+        const long long row = u * lv[j].rows + m;
         T vy = from_f<T>(0.f);
         if (own) {
             const float* q4 = pre + (size_t)(j - 1) * 4 * D;
@@ -141,15 +143,15 @@ __device__ __forceinline__ bool append_token(const TreeParams& p, long long u, l
                 pv = pv + q4[3 * D + t];
             }
             if (new_node || child_done) {
-                p.PK[j][u * D + t] = pk;
-                p.PV[j][u * D + t] = pv;
+                lv[j].PK[u * D + t] = pk;
+                lv[j].PV[u * D + t] = pv;
             }
             const float ks = pk + kcur, vsum = pv + vcur;
             const long long cnt = rj + 1;
             const long long nc = qm - m * p.b + 1;
-            p.VS[j][row * D + t] = vsum;
+            lv[j].VS[row * D + t] = vsum;
             vy = from_f<T>(__fdiv_rn(vsum, (float)cnt));
-            reinterpret_cast<T*>(p.V[j])[row * D + t] = vy;
+            reinterpret_cast<T*>(lv[j].V)[row * D + t] = vy;
             km[t] = __fdiv_rn(ks, (float)nc);
             vcur = vsum;
         }
@@ -164,7 +166,7 @@ __device__ __forceinline__ bool append_token(const TreeParams& p, long long u, l
         }
         if (own) {
             const T ky = from_f<T>(y);
-            reinterpret_cast<T*>(p.K[j])[row * D + t] = ky;
+            reinterpret_cast<T*>(lv[j].K)[row * D + t] = ky;
             kcur = to_f(ky);
             on_node(j, ky, vy);
         }

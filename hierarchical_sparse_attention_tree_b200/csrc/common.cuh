@@ -36,6 +36,35 @@ struct TreeParams {
     float scale;               // 1 / sqrt(D)
 };
 
+// One level's addresses and sizes together. Kernels that index the levels
+// with a runtime j copy these into shared memory once: kernel parameters
+// indexed at run time are constant-cache reads, one line per array, each a
+// miss the first time it is touched.
+struct LevelRef {
+    void* K;
+    void* V;
+    float* VS;
+    float* PK;
+    float* PV;
+    long long rows;
+    long long span;
+};
+
+// Threads 0..J_cap each copy one level.
+__device__ __forceinline__ void load_levels(const TreeParams& p, LevelRef* lv, int tid) {
+    if (tid <= p.J_cap) {
+        LevelRef r;
+        r.K = p.K[tid];
+        r.V = p.V[tid];
+        r.VS = p.VS[tid];
+        r.PK = p.PK[tid];
+        r.PV = p.PV[tid];
+        r.rows = p.rows[tid];
+        r.span = p.span[tid];
+        lv[tid] = r;
+    }
+}
+
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 

@@ -59,6 +59,7 @@ struct DecSmem {
     int par[KMAX];                       // kept parents of the current level, ascending
     int chosen[KMAX];                    // kept nodes of the current level, ascending
     int nlev[MAXJ + 1];                  // nodes per level over L tokens
+    LevelRef lv[MAXJ + 1];               // the levels' addresses
     float red[DEC_WARPS][8];             // per-warp partial maxima / sums (G <= 8)
     float M[8];                          // running softmax maximum per head (this CTA)
 };
@@ -109,9 +110,9 @@ __device__ __forceinline__ int rank_among(const unsigned long long* key, int n, 
 
 // Sorts one key per lane in descending order across the warp (bitonic network).
 __device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
-#pragma unroll
+#pragma unroll 1
     for (int k2 = 2; k2 <= 32; k2 <<= 1)
-#pragma unroll
+#pragma unroll 1
         for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
             const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j2);
             const bool desc = (lane & k2) == 0, lower = (lane & j2) == 0;
@@ -129,7 +130,7 @@ __device__ __forceinline__ int rank_in_lists(const unsigned long long* lists, in
     int cnt[NL];
 #pragma unroll
     for (int l = 0; l < NL; l++) cnt[l] = 0;
-#pragma unroll
+#pragma unroll 1
     for (int st = KMAX; st >= 1; st >>= 1) {
         if (st > n) continue;  // uniform: n is the same in every thread
         // every probe is a load at a valid index (clamped), so the NL loads of
@@ -145,6 +146,36 @@ __device__ __forceinline__ int rank_in_lists(const unsigned long long* lists, in
 #pragma unroll
     for (int l = 0; l < NL; l++) r += cnt[l];
     return r;
+}
+
+// Thread 0: request rows [r0, r1) of a level's candidate list (the children
+// of the kept parents par[], b per parent, n_j nodes in the level) from the
+// node rows at `base` into dst, one 1D bulk copy per contiguous piece, all
+// counted on one mbarrier. Out-of-range pieces are flagged, not copied. Kept
+// out of line: it runs a few times per launch, on one thread.
+template <typename T, int D>
+__device__ __noinline__ void issue_rows(T* dst, const T* base, const int* par, int n_j, int b, int r0, int r1,
+                                        uint64_t* bar, int* err) {
+    const int pr = r0 / b, o0 = r0 - pr * b;
+    uint32_t total = 0;
+    for (int r = r0, q = pr, o = o0; r < r1; q++, o = 0) {
+        const int n = min(b - o, r1 - r);
+        const int id0 = par[q] * b + o;
+        if (id0 >= 0 && id0 + n <= n_j) total += (uint32_t)(n * D * sizeof(T));
+        r += n;
+    }
+    fence_proxy_async_shared();
+    fence_proxy_async_global();  // global writes of a fused append seen by the bulk reads
+    mbar_arrive_expect_tx(bar, total);
+    for (int r = r0, q = pr, o = o0; r < r1; q++, o = 0) {
+        const int n = min(b - o, r1 - r);
+        const int id0 = par[q] * b + o;
+        if (id0 >= 0 && id0 + n <= n_j)
+            bulk_g2s(dst + (size_t)(r - r0) * D, base + (size_t)id0 * D, (uint32_t)(n * D * sizeof(T)), bar);
+        else
+            flag_error(err, ERR_SHAPE);
+        r += n;
+    }
 }
 
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -192,6 +223,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
         }
     }
     asm volatile("griddepcontrol.launch_dependents;");
+    load_levels(p, sm->lv, tid);  // visible after the set-up barrier below
     if (tid < 8) sm->M[tid] = -INFINITY;
     grid_dependency_wait();  // from here on, every earlier kernel's writes are visible
     const long long Lraw = p.len[u];  // both loads in flight together
@@ -235,30 +267,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
     // Thread 0: request rows [r0, r1) of level j's candidate list (children of
     // sm->par) into the key (which = 0) or value (which = 1) tile.
     auto issue = [&](int which, int j, int r0, int r1) {
-        T* dst = which == 0 ? Kt : Vt;
-        const T* base = reinterpret_cast<const T*>(which == 0 ? p.K[j] : p.V[j]) + (u * p.rows[j]) * D;
-        const int n_j = sm->nlev[j];
-        const int pr = r0 / b, o0 = r0 - pr * b;
-        uint32_t total = 0;
-        for (int r = r0, q = pr, o = o0; r < r1; q++, o = 0) {
-            const int n = min(b - o, r1 - r);
-            const int id0 = sm->par[q] * b + o;
-            if (id0 >= 0 && id0 + n <= n_j) total += (uint32_t)(n * D * sizeof(T));
-            r += n;
-        }
-        fence_proxy_async_shared();
-        fence_proxy_async_global();  // global writes of a fused append seen by the bulk reads
-        mbar_arrive_expect_tx(&sm->bar[which], total);
-        for (int r = r0, q = pr, o = o0; r < r1; q++, o = 0) {
-            const int n = min(b - o, r1 - r);
-            const int id0 = sm->par[q] * b + o;
-            if (id0 >= 0 && id0 + n <= n_j)
-                bulk_g2s(dst + (size_t)(r - r0) * D, base + (size_t)id0 * D, (uint32_t)(n * D * sizeof(T)),
-                         &sm->bar[which]);
-            else
-                flag_error(p.err, ERR_SHAPE);
-            r += n;
-        }
+        issue_rows<T, D>(which == 0 ? Kt : Vt,
+                         reinterpret_cast<const T*>(which == 0 ? sm->lv[j].K : sm->lv[j].V) + (u * sm->lv[j].rows) * D,
+                         sm->par,
+                         sm->nlev[j], b, r0, r1, &sm->bar[which], p.err);
     };
     auto wait_tile = [&](int which) {
         if (!mbar_wait(&sm->bar[which], phase[which])) {
@@ -395,7 +407,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
             const T* kn = reinterpret_cast<const T*>(a.k_new) + u * D;
             const T* vn = reinterpret_cast<const T*>(a.v_new) + u * D;
             const bool ok = append_token<T, D>(
-                p, u, Lraw, kn, vn, reinterpret_cast<const T*>(smem_raw),
+                p, sm->lv, u, Lraw, kn, vn, reinterpret_cast<const T*>(smem_raw),
                 reinterpret_cast<float*>(smem_raw + D * D * sizeof(T)),
                 [&]() {
                     const int timed_out = !mbar_wait(&sm->bar[2], 0);
@@ -464,70 +476,66 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
             }
             __syncthreads();  // logits, keys and warp lists in place; key tile free
 
-            if (j == 0) {
-                wait_tile(1);
-                if (patch_row >= 0) {
-                    if (tid < D) Vt[(size_t)patch_row * D + tid] = patch_rows()[D + tid];
-                    __syncthreads();
+            int nc_next = 0, per_n = 0, r0n = 0, r1n = 0;
+            if (j > 0) {
+                // this CTA's top keys, written to slot `rank` of every CTA's
+                // list area for this level
+                unsigned long long* gk = gkeys + (j & 1) * (DEC_CLUSTER * KMAX);
+                for (int t = tid; t < W * kk; t += DEC_THREADS) {
+                    const unsigned long long x = sm->wl[t / kk][t % kk];
+                    if (x == 0ull) continue;
+                    const int c = rank_in_lists<W>(&sm->wl[0][0], KMAX, kk, x);
+                    if (c < kk)
+                        for (int r = 0; r < CS; r++) cluster.map_shared_rank(gk, r)[rank * KMAX + c] = x;
                 }
-                accumulate(nmy, true);
-                vrows += ncand;
-                break;
+                for (int t = nmy + tid; t < kk; t += DEC_THREADS)  // fewer rows than kk
+                    for (int r = 0; r < CS; r++) cluster.map_shared_rank(gk, r)[rank * KMAX + t] = 0ull;
+                cluster.sync();
+                // global top-kk (the same in every CTA) and the kept ids in
+                // ascending order (ids are distinct)
+                for (int t = tid; t < CS * kk; t += DEC_THREADS) {
+                    const unsigned long long x = gk[(t / kk) * KMAX + t % kk];
+                    if (x == 0ull) continue;
+                    const int c = rank_in_lists<DEC_CLUSTER>(gk, KMAX, kk, x);
+                    if (c < kk) sm->picked[c] = x;
+                }
+                __syncthreads();
+                if (tid < kk) {
+                    const int id = (int)key_id(sm->picked[tid]);
+                    int pos = 0;
+                    for (int r = 0; r < kk; r++) pos += (int)key_id(sm->picked[r]) < id;
+                    sm->chosen[pos] = id;
+                }
+                if (tid == 0) sm->thresh = sm->picked[kk - 1];
+                __syncthreads();
+                if (rank == 0 && a.sel_out)  // not thread 0: it issues the copies
+                    for (int x = tid - 32; x >= 0 && x < p.k; x += DEC_THREADS - 32)
+                        a.sel_out[(u * p.J_cap + (j - 1)) * p.k + x] = x < kk ? sm->chosen[x] : -1;
+                if (tid < kk) sm->par[tid] = sm->chosen[tid];
+                __syncthreads();
+                // the next level's candidates are the children of the kept nodes
+                nc_next = ncand_of(j - 1, kk);
+                if (nc_next < 1) {
+                    bad = true;
+                    if (tid == 0) flag_error(p.err, ERR_SHAPE);
+                }
+                per_n = (nc_next + CS - 1) / CS;
+                r0n = max(0, nc_next - (CS - rank) * per_n);
+                r1n = max(0, nc_next - (CS - 1 - rank) * per_n);
+                Kt = reinterpret_cast<T*>(smem_raw);
+                if (tid == 0) issue(0, j - 1, r0n, r1n);  // key tile is free since the barriers above
             }
-            // this CTA's top keys, written to slot `rank` of every CTA's list
-            // area for this level
-            unsigned long long* gk = gkeys + (j & 1) * (DEC_CLUSTER * KMAX);
-            for (int t = tid; t < W * kk; t += DEC_THREADS) {
-                const unsigned long long x = sm->wl[t / kk][t % kk];
-                if (x == 0ull) continue;
-                const int c = rank_in_lists<W>(&sm->wl[0][0], KMAX, kk, x);
-                if (c < kk)
-                    for (int r = 0; r < CS; r++) cluster.map_shared_rank(gk, r)[rank * KMAX + c] = x;
-            }
-            for (int t = nmy + tid; t < kk; t += DEC_THREADS)  // fewer rows than kk
-                for (int r = 0; r < CS; r++) cluster.map_shared_rank(gk, r)[rank * KMAX + t] = 0ull;
-            cluster.sync();
-            // global top-kk (the same in every CTA) and the kept ids in
-            // ascending order (ids are distinct)
-            for (int t = tid; t < CS * kk; t += DEC_THREADS) {
-                const unsigned long long x = gk[(t / kk) * KMAX + t % kk];
-                if (x == 0ull) continue;
-                const int c = rank_in_lists<DEC_CLUSTER>(gk, KMAX, kk, x);
-                if (c < kk) sm->picked[c] = x;
-            }
-            __syncthreads();
-            if (tid < kk) {
-                const int id = (int)key_id(sm->picked[tid]);
-                int pos = 0;
-                for (int r = 0; r < kk; r++) pos += (int)key_id(sm->picked[r]) < id;
-                sm->chosen[pos] = id;
-            }
-            if (tid == 0) sm->thresh = sm->picked[kk - 1];
-            __syncthreads();
-            if (rank == 0 && a.sel_out)  // not thread 0: it issues the copies
-                for (int x = tid - 32; x >= 0 && x < p.k; x += DEC_THREADS - 32)
-                    a.sel_out[(u * p.J_cap + (j - 1)) * p.k + x] = x < kk ? sm->chosen[x] : -1;
-            if (tid < kk) sm->par[tid] = sm->chosen[tid];
-            __syncthreads();
-            // the next level's candidates are the children of the kept nodes
-            const int nc_next = ncand_of(j - 1, kk);
-            if (nc_next < 1) {
-                bad = true;
-                if (tid == 0) flag_error(p.err, ERR_SHAPE);
-            }
-            const int per_n = (nc_next + CS - 1) / CS;
-            const int r0n = max(0, nc_next - (CS - rank) * per_n), r1n = max(0, nc_next - (CS - 1 - rank) * per_n);
-            Kt = reinterpret_cast<T*>(smem_raw);
-            if (tid == 0) issue(0, j - 1, r0n, r1n);  // key tile is free since the barriers above
             wait_tile(1);
             if (patch_row >= 0) {
                 if (tid < D) Vt[(size_t)patch_row * D + tid] = patch_rows()[D + tid];
                 __syncthreads();
                 patch_row = -1;
             }
-            accumulate(nmy, false);  // summaries of the candidates not kept
-            vrows += ncand - kk;
-            __syncthreads();         // value tile and weights consumed
+            // level 0: every token; above: the summaries of the candidates not kept
+            accumulate(nmy, j == 0);
+            vrows += j == 0 ? ncand : ncand - kk;
+            if (j == 0) break;
+            __syncthreads();  // value tile and weights consumed
             Vt = reinterpret_cast<T*>(smem_raw) + (size_t)MY * D;
             if (tid == 0) issue(1, j - 1, r0n, r1n);
             npar = kk;

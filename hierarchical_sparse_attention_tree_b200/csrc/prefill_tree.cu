@@ -42,6 +42,7 @@ struct PtSmem {
     unsigned long long thresh;
     int par[PT_KMAX], chosen[PT_KMAX];
     int nlev[MAXJ + 1];
+    LevelRef lv[MAXJ + 1];  // the levels' addresses
     float red[PT_WARPS][8];
     float M[8];
 };
@@ -93,6 +94,7 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
         fence_mbar_init();
     }
     if (tid < 8) sm->M[tid] = -INFINITY;
+    load_levels(p, sm->lv, tid);  // visible after the set-up barrier below
     {
         const T* qg = reinterpret_cast<const T*>(a.q) + (((size_t)bseq * a.C + t) * a.Hq + h * G) * D;
         for (int i = tid; i < G * D; i += PT_THREADS) qf[i] = to_f(qg[i]);
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
     // thread 0: rows [r0, r1) of level j's candidate list (children of sm->par)
     auto issue = [&](int which, int j, int r0, int r1) {
         T* dst = which == 0 ? Kt : Vt;
-        const T* base = reinterpret_cast<const T*>(which == 0 ? p.K[j] : p.V[j]) + (u * p.rows[j]) * D;
+        const T* base = reinterpret_cast<const T*>(which == 0 ? sm->lv[j].K : sm->lv[j].V) + (u * sm->lv[j].rows) * D;
         const int n_j = sm->nlev[j];
         const int pr = r0 / b, o0 = r0 - pr * b;
         uint32_t total = 0;

@@ -182,6 +182,7 @@ __global__ void __launch_bounds__(D) append_one_kernel(TreeParams p, const T* __
     T* Wt = reinterpret_cast<T*>(smem_a);                                   // [D][D]
     float* scratch = reinterpret_cast<float*>(smem_a + D * D * sizeof(T));  // append_scratch_floats
     __shared__ uint64_t wbar;
+    __shared__ LevelRef lv[MAXJ + 1];
     const long long u = blockIdx.x;
     // the next kernel on the stream (a decode) may start its own set-up now
     asm volatile("griddepcontrol.launch_dependents;");
@@ -196,8 +197,10 @@ __global__ void __launch_bounds__(D) append_one_kernel(TreeParams p, const T* __
         mbar_arrive_expect_tx(&wbar, (uint32_t)(D * D * sizeof(T)));
         bulk_g2s(Wt, p.Wt, (uint32_t)(D * D * sizeof(T)), &wbar);
     }
+    load_levels(p, lv, threadIdx.x);
+    __syncthreads();
     const bool ok = append_token<T, D>(
-        p, u, P, k_new + u * D, v_new + u * D, Wt, scratch,
+        p, lv, u, P, k_new + u * D, v_new + u * D, Wt, scratch,
         [&]() {
             const int timed_out = !mbar_wait(&wbar, 0);
             if (__syncthreads_or(timed_out)) {  // same decision in every thread
