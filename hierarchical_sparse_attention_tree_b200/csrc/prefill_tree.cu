@@ -76,8 +76,6 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
 
     extern __shared__ __align__(128) unsigned char smem_pt[];
     const size_t tiles_bytes = prefill_tree_tiles(D, G, (int)sizeof(T));
-    T* Kt = reinterpret_cast<T*>(smem_pt);
-    T* Vt = Kt + (size_t)PT_TILE * D;
     float* egacc = reinterpret_cast<float*>(smem_pt);
     PtSmem* sm = reinterpret_cast<PtSmem*>(smem_pt + tiles_bytes);
     unsigned long long* key = reinterpret_cast<unsigned long long*>(sm + 1);
@@ -125,10 +123,15 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
     }
     uint32_t phase[2] = {0u, 0u};
 
-    // thread 0: rows [r0, r1) of level j's candidate list (children of sm->par)
-    auto issue = [&](int which, int j, int r0, int r1) {
-        T* dst = which == 0 ? Kt : Vt;
-        const T* base = reinterpret_cast<const T*>(which == 0 ? sm->lv[j].K : sm->lv[j].V) + (u * sm->lv[j].rows) * D;
+    // Thread 0: rows [r0, r1) of level j's candidate list (children of
+    // sm->par) into tile buffer buf (two buffers of PT_TILE rows, one
+    // mbarrier each): what = 0 keys, 1 values, 2 both (keys in the first half
+    // of the buffer, values in the second; at most PT_TILE / 2 rows).
+    auto issue = [&](int buf, int what, int j, int r0, int r1) {
+        T* dst = reinterpret_cast<T*>(smem_pt) + (size_t)buf * PT_TILE * D;
+        T* dstv = what == 2 ? dst + (size_t)(PT_TILE / 2) * D : dst;
+        const T* kb = reinterpret_cast<const T*>(sm->lv[j].K) + (u * sm->lv[j].rows) * D;
+        const T* vb = reinterpret_cast<const T*>(sm->lv[j].V) + (u * sm->lv[j].rows) * D;
         const int n_j = sm->nlev[j];
         const int pr = r0 / b, o0 = r0 - pr * b;
         uint32_t total = 0;
@@ -139,18 +142,21 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
             r += n;
         }
         fence_proxy_async_shared();
-        mbar_arrive_expect_tx(&sm->bar[which], total);
+        mbar_arrive_expect_tx(&sm->bar[buf], what == 2 ? 2 * total : total);
         for (int r = r0, q = pr, o = o0; r < r1; q++, o = 0) {
             const int n = min(b - o, r1 - r);
             const int id0 = sm->par[q] * b + o;
-            if (id0 >= 0 && id0 + n <= n_j)
-                bulk_g2s(dst + (size_t)(r - r0) * D, base + (size_t)id0 * D, (uint32_t)(n * D * sizeof(T)),
-                         &sm->bar[which]);
-            else
+            const uint32_t bytes = (uint32_t)(n * D * sizeof(T));
+            if (id0 >= 0 && id0 + n <= n_j) {
+                if (what != 1) bulk_g2s(dst + (size_t)(r - r0) * D, kb + (size_t)id0 * D, bytes, &sm->bar[buf]);
+                if (what != 0) bulk_g2s(dstv + (size_t)(r - r0) * D, vb + (size_t)id0 * D, bytes, &sm->bar[buf]);
+            } else {
                 flag_error(p.err, ERR_SHAPE);
+            }
             r += n;
         }
     };
+    auto tile = [&](int buf) { return reinterpret_cast<T*>(smem_pt) + (size_t)buf * PT_TILE * D; };
     auto wait_tile = [&](int which) {
         if (!mbar_wait(&sm->bar[which], phase[which])) {
             if (lane == 0) flag_error(p.err, ERR_TIMEOUT);
@@ -167,7 +173,7 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
 
     // Scores of tile rows [0, nmy) = candidate ranks [r0, r0 + nmy) with the
     // query at index P (logits, and the selection keys when want_keys).
-    auto score_tile = [&](int r0, int nmy, int P, bool want_keys) {
+    auto score_tile = [&](const T* Kt, int r0, int nmy, int P, bool want_keys) {
         score_rows<T, D, G, W>(p.rope, p.scale, b, Kt, qf, r0, nmy, P, warp, lane, nullptr,
                                [&](int i, int hh, float logit, float Ssum, int r, int o) {
                                    lg[hh * MC + r0 + i] = logit;
@@ -177,7 +183,7 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
 
     // Entries of tile rows [0, nmy) (ranks r0..) join the CTA's softmax:
     // all of them (tokens) or the candidates not kept (key < threshold).
-    auto accumulate = [&](int r0, int nmy, bool tokens) {
+    auto accumulate = [&](const T* Vt, int r0, int nmy, bool tokens) {
         float mx[G];
 #pragma unroll
         for (int g = 0; g < G; g++) mx[g] = -INFINITY;
@@ -250,20 +256,27 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
             }
             const int kk = min(p.k, ncand);
             if (ncand > p.k) {
-                // score every candidate, tile by tile
-                for (int r0 = 0; r0 < ncand; r0 += PT_TILE) {
-                    const int nmy = min(PT_TILE, ncand - r0);
-                    if (tid == 0) issue(0, j, r0, r0 + nmy);
-                    wait_tile(0);
-                    score_tile(r0, nmy, ncand - 1, true);
+                // score every candidate, tile by tile; the next tile is in
+                // flight while one is scored
+                const int nt = (ncand + PT_TILE - 1) / PT_TILE;
+                if (tid == 0) issue(0, 0, j, 0, min(PT_TILE, ncand));
+                for (int ti = 0; ti < nt; ti++) {
+                    const int bi = ti & 1, r0 = ti * PT_TILE, nmy = min(PT_TILE, ncand - r0);
+                    if (tid == 0 && ti + 1 < nt) issue(bi ^ 1, 0, j, r0 + PT_TILE, min(r0 + 2 * PT_TILE, ncand));
+                    wait_tile(bi);
+                    score_tile(tile(bi), r0, nmy, ncand - 1, true);
                     __syncthreads();
                 }
+                // the values of the first tile are requested before the sort
+                if (tid == 0) issue(0, 1, j, 0, min(PT_TILE, ncand));
                 // top kk by a descending bitonic sort of the packed keys
-                for (int i = tid; i < a.sortn; i += PT_THREADS) skey[i] = i < ncand ? key[i] : 0ull;
+                int sn = 2;
+                while (sn < ncand) sn <<= 1;
+                for (int i = tid; i < sn; i += PT_THREADS) skey[i] = i < ncand ? key[i] : 0ull;
                 __syncthreads();
-                for (int k2 = 2; k2 <= a.sortn; k2 <<= 1)
+                for (int k2 = 2; k2 <= sn; k2 <<= 1)
                     for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
-                        for (int i = tid; i < a.sortn; i += PT_THREADS) {
+                        for (int i = tid; i < sn; i += PT_THREADS) {
                             const int ixj = i ^ j2;
                             if (ixj > i) {
                                 const unsigned long long x = skey[i], y = skey[ixj];
@@ -284,12 +297,12 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
                 }
                 if (tid == 0) sm->thresh = skey[kk - 1];
                 __syncthreads();
-                // summaries of the candidates not kept
-                for (int r0 = 0; r0 < ncand; r0 += PT_TILE) {
-                    const int nmy = min(PT_TILE, ncand - r0);
-                    if (tid == 0) issue(1, j, r0, r0 + nmy);
-                    wait_tile(1);
-                    accumulate(r0, nmy, false);
+                // summaries of the candidates not kept, tile by tile
+                for (int ti = 0; ti < nt; ti++) {
+                    const int bi = ti & 1, r0 = ti * PT_TILE, nmy = min(PT_TILE, ncand - r0);
+                    if (tid == 0 && ti + 1 < nt) issue(bi ^ 1, 1, j, r0 + PT_TILE, min(r0 + 2 * PT_TILE, ncand));
+                    wait_tile(bi);
+                    accumulate(tile(bi), r0, nmy, false);
                     __syncthreads();
                 }
             } else {  // keeps every candidate: nothing to read or score
@@ -306,17 +319,17 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
         // order) the chunk's own tokens, already in the local state
         const int n0 = bad ? 0 : ncand_of(0, npar);
         const int P0 = n0 + t;
-        for (int r0 = 0; r0 < n0; r0 += PT_TILE) {
-            const int nmy = min(PT_TILE, n0 - r0);
-            if (tid == 0) {
-                issue(0, 0, r0, r0 + nmy);
-                issue(1, 0, r0, r0 + nmy);
-            }
-            wait_tile(0);
-            score_tile(r0, nmy, P0, false);
+        // keys and values of half-size tiles together, the next tile in flight
+        constexpr int T0 = PT_TILE / 2;
+        const int nt0 = (n0 + T0 - 1) / T0;
+        if (tid == 0 && nt0 > 0) issue(0, 2, 0, 0, min(T0, n0));
+        for (int ti = 0; ti < nt0; ti++) {
+            const int bi = ti & 1, r0 = ti * T0, nmy = min(T0, n0 - r0);
+            if (tid == 0 && ti + 1 < nt0) issue(bi ^ 1, 2, 0, r0 + T0, min(r0 + 2 * T0, n0));
+            wait_tile(bi);
+            score_tile(tile(bi), r0, nmy, P0, false);
             __syncthreads();
-            wait_tile(1);
-            accumulate(r0, nmy, true);
+            accumulate(tile(bi) + (size_t)T0 * D, r0, nmy, true);
             __syncthreads();
         }
     }
