@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
     unsigned long long* key = reinterpret_cast<unsigned long long*>(sm + 1);
     unsigned long long* skey = key + MC;
     float* qf = reinterpret_cast<float*>(skey + a.sortn);
-    float* lg = qf + G * D;           // [G][MC]
+    float* lg = qf + G * D;           // [MC][G] logits of a level's candidates
     float* pbuf = lg + G * MC;        // [TILE][G]
     float* cacc = pbuf + PT_TILE * G;
     float* cl = cacc + G * D;
@@ -173,54 +173,53 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
 
     // Scores of tile rows [0, nmy) = candidate ranks [r0, r0 + nmy) with the
     // query at index P (logits, and the selection keys when want_keys).
+    // Each warp's largest logit per head is folded into sm->red[warp]
+    // (reset by reset_max).
     auto score_tile = [&](const T* Kt, int r0, int nmy, int P, bool want_keys) {
-        score_rows<T, D, G, W>(p.rope, p.scale, b, Kt, qf, r0, nmy, P, warp, lane, nullptr,
-                               [&](int i, int hh, float logit, float Ssum, int r, int o) {
-                                   lg[hh * MC + r0 + i] = logit;
-                                   if (hh == 0 && want_keys) key[r0 + i] = sel_key(Ssum, sm->par[r] * b + o);
-                               });
+        score_rows<T, D, G, W>(
+            p.rope, p.scale, b, Kt, qf, r0, nmy, P, warp, lane, sm->red[warp],
+            [&](int i, int hh, float logit, float Ssum, int r, int o) {
+                lg[(r0 + i) * G + hh] = logit;
+                if (hh == 0 && want_keys) key[r0 + i] = sel_key(Ssum, sm->par[r] * b + o);
+            },
+            true);
+    };
+    auto reset_max = [&]() {  // each warp its own slots
+        if (lane < G) sm->red[warp][lane] = -INFINITY;
+        __syncwarp();
     };
 
     // Entries of tile rows [0, nmy) (ranks r0..) join the CTA's softmax:
-    // all of them (tokens) or the candidates not kept (key < threshold).
+    // all of them (tokens) or the candidates not kept (key < threshold). The
+    // running maximum takes the scoring pass's per-warp maxima (over every
+    // scored row, kept ones included: a bound on the entries that join).
+    const int gt = tid % G;  // the head of this thread's weights (PT_THREADS % G == 0)
     auto accumulate = [&](const T* Vt, int r0, int nmy, bool tokens) {
-        float mx[G];
-#pragma unroll
-        for (int g = 0; g < G; g++) mx[g] = -INFINITY;
-        for (int e = tid; e < nmy; e += PT_THREADS) {
-            if (tokens || key[r0 + e] < sm->thresh)
-#pragma unroll
-                for (int g = 0; g < G; g++) mx[g] = fmaxf(mx[g], lg[g * MC + r0 + e]);
-        }
-#pragma unroll
-        for (int g = 0; g < G; g++) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], o));
-            if (lane == 0) sm->red[warp][g] = mx[g];
-        }
-        __syncthreads();
-        float Mn[G], alpha[G];
+        float Mt = 0.f, Mown = 0.f, alpha[G];
 #pragma unroll
         for (int g = 0; g < G; g++) {
             float m = sm->M[g];
             const float mold = m;
 #pragma unroll
             for (int w = 0; w < W; w++) m = fmaxf(m, sm->red[w][g]);
-            Mn[g] = m;
             alpha[g] = (m == -INFINITY) ? 1.f : (mold == -INFINITY ? 0.f : expf(mold - m));
             lpart[g] *= alpha[g];
+            if (g == gt) Mt = m;
+            if (g == tid) Mown = m;
         }
-        for (int e = tid; e < nmy; e += PT_THREADS) {
+        float lsum = 0.f;
+        for (int x = tid; x < nmy * G; x += PT_THREADS) {
+            const int e = x / G;
             const bool valid = tokens || key[r0 + e] < sm->thresh;
-#pragma unroll
-            for (int g = 0; g < G; g++) {
-                const float pe = valid ? expf(lg[g * MC + r0 + e] - Mn[g]) : 0.f;
-                pbuf[e * G + g] = pe;
-                lpart[g] += pe;
-            }
+            const float pe = valid ? expf(lg[r0 * G + x] - Mt) : 0.f;
+            pbuf[x] = pe;
+            lsum += pe;
         }
-        __syncthreads();
-        if (tid < G) sm->M[tid] = Mn[tid];
+#pragma unroll
+        for (int g = 0; g < G; g++)
+            if (g == gt) lpart[g] += lsum;
+        __syncthreads();  // weights in place; every thread has read sm->M
+        if (tid < G) sm->M[tid] = Mown;
 #pragma unroll
         for (int g = 0; g < G; g++)
 #pragma unroll
@@ -260,6 +259,7 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
                 // flight while one is scored
                 const int nt = (ncand + PT_TILE - 1) / PT_TILE;
                 if (tid == 0) issue(0, 0, j, 0, min(PT_TILE, ncand));
+                reset_max();
                 for (int ti = 0; ti < nt; ti++) {
                     const int bi = ti & 1, r0 = ti * PT_TILE, nmy = min(PT_TILE, ncand - r0);
                     if (tid == 0 && ti + 1 < nt) issue(bi ^ 1, 0, j, r0 + PT_TILE, min(r0 + 2 * PT_TILE, ncand));
@@ -327,6 +327,7 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
             const int bi = ti & 1, r0 = ti * T0, nmy = min(T0, n0 - r0);
             if (tid == 0 && ti + 1 < nt0) issue(bi ^ 1, 2, 0, r0 + T0, min(r0 + 2 * T0, n0));
             wait_tile(bi);
+            reset_max();
             score_tile(tile(bi), r0, nmy, P0, false);
             __syncthreads();
             accumulate(tile(bi) + (size_t)T0 * D, r0, nmy, true);

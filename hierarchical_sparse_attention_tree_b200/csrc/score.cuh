@@ -84,10 +84,12 @@ __device__ __forceinline__ void rotate_query(const float* rope, const float* qf,
 // of the W warps takes a contiguous slice of the rows. For every row and
 // head, emit(i, h, logit, S, r, o) runs on exactly one lane, where r*b + o is
 // the candidate index. If wmax is given, lane 0 stores there the warp's
-// largest logit per head (-inf for heads without rows).
+// largest logit per head (-inf for heads without rows), or, with
+// wmax_fold, the larger of that and the value already there.
 template <typename T, int D, int G, int W, typename Emit>
 __device__ __forceinline__ void score_rows(const float* rope, float scale, int b, const T* Kt, const float* qf,
-                                           int r0, int nmy, int P, int warp, int lane, float* wmax, Emit emit) {
+                                           int r0, int nmy, int P, int warp, int lane, float* wmax, Emit emit,
+                                           bool wmax_fold = false) {
     using SL = ScoreLayout<D, G>;
     constexpr int HD = SL::HD, PL = SL::PL, P2 = SL::P2, LPC = SL::LPC, CPW = SL::CPW, NC = SL::NC;
     constexpr int STEP = CPW * NC;
@@ -204,7 +206,7 @@ __device__ __forceinline__ void score_rows(const float* rope, float scale, int b
             float m = myh == g ? lmax : -INFINITY;
 #pragma unroll
             for (int sft = 16; sft > 0; sft >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, sft));
-            if (lane == 0) wmax[g] = m;
+            if (lane == 0) wmax[g] = wmax_fold ? fmaxf(wmax[g], m) : m;
         }
     }
 }
