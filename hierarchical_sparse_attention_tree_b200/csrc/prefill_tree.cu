@@ -41,6 +41,7 @@ struct PtSmem {
     uint64_t bar[2];
     unsigned long long thresh;
     int par[PT_KMAX], chosen[PT_KMAX];
+    unsigned long long picked[PT_KMAX];  // the level's top keys, best first
     int nlev[MAXJ + 1];
     LevelRef lv[MAXJ + 1];  // the levels' addresses
     float red[PT_WARPS][8];
@@ -62,6 +63,33 @@ __host__ __device__ inline size_t prefill_tree_tiles(int D, int G, int elem) {
     const size_t eg = (size_t)(PT_THREADS / (D / PT_CPT)) * G * D * 4;
     if (eg > tiles) tiles = eg;
     return (tiles + 127) & ~(size_t)127;
+}
+
+// Four independent runs of one key per lane, each sorted descending across
+// the warp (bitonic network; the four advance together).
+__device__ __forceinline__ void warp_sort4_desc32(unsigned long long (&x)[4], int lane) {
+#pragma unroll 1
+    for (int k2 = 2; k2 <= 32; k2 <<= 1)
+#pragma unroll 1
+        for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
+            const bool desc = (lane & k2) == 0, lower = (lane & j2) == 0;
+#pragma unroll
+            for (int r = 0; r < 4; r++) {
+                const unsigned long long y = __shfl_xor_sync(0xffffffffu, x[r], j2);
+                x[r] = (lower == desc) ? (x[r] > y ? x[r] : y) : (x[r] < y ? x[r] : y);
+            }
+        }
+}
+
+// The lanes hold a bitonic sequence (largest first run, then smallest);
+// returns it sorted descending.
+__device__ __forceinline__ unsigned long long warp_merge_desc32(unsigned long long x, int lane) {
+#pragma unroll
+    for (int j2 = 16; j2 > 0; j2 >>= 1) {
+        const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j2);
+        x = (lane & j2) == 0 ? (x > y ? x : y) : (x < y ? x : y);
+    }
+    return x;
 }
 
 template <typename T, int D, int G>
@@ -269,34 +297,87 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
                 }
                 // the values of the first tile are requested before the sort
                 if (tid == 0) issue(0, 1, j, 0, min(PT_TILE, ncand));
-                // top kk by a descending bitonic sort of the packed keys
-                int sn = 2;
-                while (sn < ncand) sn <<= 1;
-                for (int i = tid; i < sn; i += PT_THREADS) skey[i] = i < ncand ? key[i] : 0ull;
-                __syncthreads();
-                for (int k2 = 2; k2 <= sn; k2 <<= 1)
-                    for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
-                        for (int i = tid; i < sn; i += PT_THREADS) {
-                            const int ixj = i ^ j2;
-                            if (ixj > i) {
-                                const unsigned long long x = skey[i], y = skey[ixj];
-                                const bool desc = (i & k2) == 0;
-                                if (desc ? (x < y) : (x > y)) {
-                                    skey[i] = y;
-                                    skey[ixj] = x;
-                                }
+                if (kk <= 32 && ncand <= W * 128 && a.sortn >= W * 32) {
+                    // each warp: the top 32 of its 128 keys (four sorted runs
+                    // of 32, merged pairwise); then the CTA's top kk by rank
+                    // among the eight warp lists
+                    unsigned long long R[4];
+#pragma unroll
+                    for (int r = 0; r < 4; r++) {
+                        const int i = warp * 128 + r * 32 + lane;
+                        R[r] = i < ncand ? key[i] : 0ull;
+                    }
+                    warp_sort4_desc32(R, lane);
+#pragma unroll
+                    for (int m = 0; m < 2; m++) {
+                        const unsigned long long y = __shfl_sync(0xffffffffu, R[2 * m + 1], 31 - lane);
+                        R[m] = warp_merge_desc32(R[2 * m] > y ? R[2 * m] : y, lane);
+                    }
+                    const unsigned long long y = __shfl_sync(0xffffffffu, R[1], 31 - lane);
+                    skey[warp * 32 + lane] = warp_merge_desc32(R[0] > y ? R[0] : y, lane);
+                    __syncthreads();
+                    for (int x = tid; x < W * kk; x += PT_THREADS) {
+                        const unsigned long long kx = skey[(x / kk) * 32 + x % kk];
+                        if (kx == 0ull) continue;
+                        // keys of each list greater than kx (descending, distinct):
+                        // one binary search per list, the lists advancing together
+                        int lo[W];
+#pragma unroll
+                        for (int l = 0; l < W; l++) lo[l] = 0;
+#pragma unroll 1
+                        for (int st = 32; st >= 1; st >>= 1) {
+                            if (st > kk) continue;
+#pragma unroll
+                            for (int l = 0; l < W; l++) {
+                                const int pos = lo[l] + st;
+                                const unsigned long long yk = skey[l * 32 + min(pos, kk) - 1];
+                                lo[l] = (pos <= kk && yk > kx) ? pos : lo[l];
                             }
                         }
-                        __syncthreads();
+                        int c = 0;
+#pragma unroll
+                        for (int l = 0; l < W; l++) c += lo[l];
+                        if (c < kk) sm->picked[c] = kx;
                     }
-                if (tid < kk) {
-                    const int id = (int)key_id(skey[tid]);
-                    int pos = 0;
-                    for (int r = 0; r < kk; r++) pos += (int)key_id(skey[r]) < id;
-                    sm->chosen[pos] = id;
+                    __syncthreads();
+                    if (tid < kk) {
+                        const int id = (int)key_id(sm->picked[tid]);
+                        int pos = 0;
+                        for (int r = 0; r < kk; r++) pos += (int)key_id(sm->picked[r]) < id;
+                        sm->chosen[pos] = id;
+                    }
+                    if (tid == 0) sm->thresh = sm->picked[kk - 1];
+                    __syncthreads();
+                } else {
+                    // top kk by a descending bitonic sort of the packed keys
+                    int sn = 2;
+                    while (sn < ncand) sn <<= 1;
+                    for (int i = tid; i < sn; i += PT_THREADS) skey[i] = i < ncand ? key[i] : 0ull;
+                    __syncthreads();
+                    for (int k2 = 2; k2 <= sn; k2 <<= 1)
+                        for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
+                            for (int i = tid; i < sn; i += PT_THREADS) {
+                                const int ixj = i ^ j2;
+                                if (ixj > i) {
+                                    const unsigned long long x = skey[i], y = skey[ixj];
+                                    const bool desc = (i & k2) == 0;
+                                    if (desc ? (x < y) : (x > y)) {
+                                        skey[i] = y;
+                                        skey[ixj] = x;
+                                    }
+                                }
+                            }
+                            __syncthreads();
+                        }
+                    if (tid < kk) {
+                        const int id = (int)key_id(skey[tid]);
+                        int pos = 0;
+                        for (int r = 0; r < kk; r++) pos += (int)key_id(skey[r]) < id;
+                        sm->chosen[pos] = id;
+                    }
+                    if (tid == 0) sm->thresh = skey[kk - 1];
+                    __syncthreads();
                 }
-                if (tid == 0) sm->thresh = skey[kk - 1];
-                __syncthreads();
                 // summaries of the candidates not kept, tile by tile
                 for (int ti = 0; ti < nt; ti++) {
                     const int bi = ti & 1, r0 = ti * PT_TILE, nmy = min(PT_TILE, ncand - r0);
