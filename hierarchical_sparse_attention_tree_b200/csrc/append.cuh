@@ -50,6 +50,13 @@ __device__ __forceinline__ float pool_product_half(const T* Wt, const float* x, 
     return ya + yb;
 }
 
+// The tree sizes the append needs (a few scalars, so that the routine can be
+// called out of line without the whole parameter block).
+struct AppendDims {
+    long long cap;
+    int J_cap, b;
+};
+
 // Shared memory it needs besides the pooler: km [D], part [2][D] and pre
 // [J_cap][4][D] floats.
 __host__ __device__ inline size_t append_scratch_floats(int D, int J_cap) { return (size_t)3 * D + 4 * (size_t)J_cap * D; }
@@ -65,7 +72,7 @@ __host__ __device__ inline size_t append_scratch_floats(int D, int J_cap) { retu
 // With at least 2D threads the pooler product is split over two threads per
 // output coordinate (same arithmetic).
 template <typename T, int D, typename WaitW, typename OnNode>
-__device__ __forceinline__ bool append_token(const TreeParams& p, const LevelRef* lv, long long u, long long P,
+__device__ __forceinline__ bool append_token(const AppendDims& p, const LevelRef* lv, long long u, long long P,
                                              const T* k_row,
                                              const T* v_row, const T* Wsm, float* scratch, WaitW wait_w,
                                              OnNode on_node) {

@@ -83,7 +83,9 @@ __host__ __device__ inline size_t decode_smem_tail(int D, int G, int MY) {
 __host__ __device__ inline size_t decode_region0(int D, int G, int MY, int elem, int J_cap, bool fused) {
     // the appending CTA of a fused step first holds the pooler and the
     // append scratch here
-    const size_t app = fused ? (size_t)D * D * elem + append_scratch_floats(D, J_cap) * 4 : 0;
+    const size_t app = fused ? (((size_t)D * D * elem + append_scratch_floats(D, J_cap) * 4 + 127) & ~(size_t)127) +
+                                   128 + 4 * (size_t)D * elem + 128
+                             : 0;
     const size_t tiles0 = 2 * (size_t)MY * D * elem;
     const size_t tiles = tiles0 > app ? tiles0 : app;
     const size_t eg = (size_t)(DEC_THREADS / (D / CPT)) * G * D * 4;
@@ -176,6 +178,42 @@ __device__ __noinline__ void issue_rows(T* dst, const T* base, const int* par, i
             flag_error(err, ERR_SHAPE);
         r += n;
     }
+}
+
+// The fused step's append, out of line (one copy of its code): appends the
+// token of unit u at position P, leaves the refreshed node of level jf (the
+// first scored level; jf = 0: the token itself) in patch[0..D) (key) and
+// patch[D..2D) (value), and makes its global writes visible to later bulk
+// reads. Every thread of the block calls it. False if the pooler copy (on
+// wbar, into the start of smem) did not arrive.
+template <typename T, int D>
+__device__ __noinline__ bool fused_append(AppendDims dims, const LevelRef* lv, long long u, long long P, const T* kn,
+                                          const T* vn, unsigned char* smem, T* patch, int jf, uint64_t* wbar,
+                                          int* err) {
+    const int tid = threadIdx.x;
+    const bool ok = append_token<T, D>(
+        dims, lv, u, P, kn, vn, reinterpret_cast<const T*>(smem), reinterpret_cast<float*>(smem + D * D * sizeof(T)),
+        [&]() {
+            const int timed_out = !mbar_wait(wbar, 0);
+            if (__syncthreads_or(timed_out)) {
+                if (tid == 0) flag_error(err, ERR_TIMEOUT);
+                return false;
+            }
+            return true;
+        },
+        [&](int jj, T ky, T vy) {
+            if (jj == jf) {
+                patch[tid] = ky;
+                patch[D + tid] = vy;
+            }
+        });
+    if (jf == 0 && tid < D) {
+        patch[tid] = kn[tid];
+        patch[D + tid] = vn[tid];
+    }
+    fence_proxy_async_global();  // this CTA's writes, before its later bulk reads
+    __syncthreads();
+    return ok;
 }
 
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -342,6 +380,33 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
         if (!mbar_wait(&sm->bar[2], 0) && tid == 0) flag_error(p.err, ERR_TIMEOUT);
         __syncthreads();
     }
+    // [pooler | append scratch | patch rows: key, value | the appender's first tiles]
+    auto patch_rows = [&]() {
+        return reinterpret_cast<T*>(
+            smem_raw + ((D * D * sizeof(T) + append_scratch_floats(D, p.J_cap) * 4 + 127) & ~(size_t)127));
+    };
+    // Fused step, usual case: the appending CTA holds only the right-edge row
+    // of the first scored level (the only row the append changes), so it
+    // appends at once and needs no copy of that row. The first scored level
+    // is the highest level with more than k nodes (every level above keeps
+    // all of its candidates), else the tokens.
+    bool chained = false;
+    if (appender && !bad_len) {
+        int jt = 1;
+        while (jt < p.J_cap && sm->nlev[jt] > b) jt++;
+        int jf = 0;
+        for (int x = jt; x >= 1 && jf == 0; x--)
+            if (sm->nlev[x] > p.k) jf = x;
+        if (sm->nlev[jf] - 1 <= (CS - 1) * MY) {
+            const bool ok = fused_append<T, D>(AppendDims{p.cap, p.J_cap, p.b}, sm->lv, u, Lraw,
+                                               reinterpret_cast<const T*>(a.k_new) + u * D,
+                                               reinterpret_cast<const T*>(a.v_new) + u * D, smem_raw, patch_rows(), jf,
+                                               &sm->bar[2], p.err);
+            appended = ok;
+            if (!ok) bad = true;
+            chained = true;
+        }
+    }
     if (!bad_len) {
         int j = 1;
         while (j < p.J_cap && sm->nlev[j] > b) j++;  // top level
@@ -372,70 +437,57 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
         // last rows of every level
         int per = (ncand + CS - 1) / CS;
         int r0 = max(0, ncand - (CS - rank) * per), r1 = max(0, ncand - (CS - 1 - rank) * per);
-        if (app && ncand >= 1 && ncand - 1 <= (CS - 1) * MY) {
+        if (app && ncand >= 1 && ncand - 1 <= (CS - 1) * MY) {  // same test as the appender's early append
             // fused step: the appending CTA takes only the right-edge row (it
             // appends first), the others share the rest
             const int per1 = (ncand - 1 + CS - 2) / (CS - 1);
             r0 = rank == CS - 1 ? ncand - 1 : min(ncand - 1, rank * per1);
             r1 = rank == CS - 1 ? ncand : min(ncand - 1, r0 + per1);
         }
-        // Fused step. The appending CTA holds the last rows of this level,
-        // the only ones the append changes: its tiles are requested now, like
-        // every CTA's, into a place after the pooler and the append scratch
-        // (when they fit), and the refreshed right-edge row is written over
-        // the copied one once the tile has landed. The other CTAs read the
-        // right edge only after the first selection barrier, which this CTA
-        // reaches after the append.
-        // [pooler | append scratch | patch rows: key, value | first tiles]
-        auto patch_rows = [&]() {
-            return reinterpret_cast<T*>(
-                smem_raw + ((D * D * sizeof(T) + append_scratch_floats(D, p.J_cap) * 4 + 127) & ~(size_t)127));
-        };
+        // Fused step, other case (a first level too large for the one-row
+        // split): the appending CTA holds the last rows of this level; its
+        // tiles are requested now into a place after the pooler and the append
+        // scratch (when they fit), it appends, and the refreshed right-edge
+        // row is written over the copied one once the tile has landed. The
+        // other CTAs read the right edge only after the first selection
+        // barrier, which this CTA reaches after the append.
         const size_t tiles_off = ((reinterpret_cast<unsigned char*>(patch_rows() + 2 * D) - smem_raw) + 127) & ~(size_t)127;
         const bool early = appender && tiles_off + 2 * (size_t)(r1 - r0) * D * sizeof(T) <= (size_t)a.region0;
         if (early) {
             Kt = reinterpret_cast<T*>(smem_raw + tiles_off);
             Vt = Kt + (size_t)(r1 - r0) * D;
         }
-        if (tid == 0 && (!appender || early)) {
-            issue(0, j, r0, r1);
-            issue(1, j, r0, r1);
-        }
         int patch_row = -1;  // row of this CTA's first tiles to overwrite
-        if (appender) {
-            const int jf = j;
-            const T* kn = reinterpret_cast<const T*>(a.k_new) + u * D;
-            const T* vn = reinterpret_cast<const T*>(a.v_new) + u * D;
-            const bool ok = append_token<T, D>(
-                p, sm->lv, u, Lraw, kn, vn, reinterpret_cast<const T*>(smem_raw),
-                reinterpret_cast<float*>(smem_raw + D * D * sizeof(T)),
-                [&]() {
-                    const int timed_out = !mbar_wait(&sm->bar[2], 0);
-                    if (__syncthreads_or(timed_out)) {
-                        if (tid == 0) flag_error(p.err, ERR_TIMEOUT);
-                        return false;
-                    }
-                    return true;
-                },
-                [&](int jj, T ky, T vy) {
-                    if (jj == jf) {
-                        patch_rows()[tid] = ky;
-                        patch_rows()[D + tid] = vy;
-                    }
-                });
-            if (jf == 0 && tid < D) {  // the first scored level is the tokens: the new one
-                patch_rows()[tid] = kn[tid];
-                patch_rows()[D + tid] = vn[tid];
+        if (chained) {
+            // the one row is the refreshed right edge: written here, not copied
+            // (empty requests complete the tile barriers' phases)
+            if (tid < D) {
+                Kt[(size_t)(ncand - 1 - r0) * D + tid] = patch_rows()[tid];
+                Vt[(size_t)(ncand - 1 - r0) * D + tid] = patch_rows()[D + tid];
             }
-            appended = ok;
-            if (!ok) bad = true;
-            fence_proxy_async_global();  // this CTA's writes, before its own bulk reads
-            __syncthreads();             // pooler, scratch and patch rows in place
-            if (early)
-                patch_row = ncand - 1 - r0;
-            else if (tid == 0) {
+            if (tid == 0) {
+                issue(0, j, r0, r0);
+                issue(1, j, r0, r0);
+            }
+            __syncthreads();
+        } else {
+            if (tid == 0 && (!appender || early)) {
                 issue(0, j, r0, r1);
                 issue(1, j, r0, r1);
+            }
+            if (appender) {
+                const bool ok = fused_append<T, D>(AppendDims{p.cap, p.J_cap, p.b}, sm->lv, u, Lraw,
+                                                   reinterpret_cast<const T*>(a.k_new) + u * D,
+                                                   reinterpret_cast<const T*>(a.v_new) + u * D, smem_raw, patch_rows(),
+                                                   j, &sm->bar[2], p.err);
+                appended = ok;
+                if (!ok) bad = true;
+                if (early)
+                    patch_row = ncand - 1 - r0;
+                else if (tid == 0) {
+                    issue(0, j, r0, r1);
+                    issue(1, j, r0, r1);
+                }
             }
         }
         for (;;) {

@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(D) append_one_kernel(TreeParams p, const T* __
     load_levels(p, lv, threadIdx.x);
     __syncthreads();
     const bool ok = append_token<T, D>(
-        p, lv, u, P, k_new + u * D, v_new + u * D, Wt, scratch,
+        AppendDims{p.cap, p.J_cap, p.b}, lv, u, P, k_new + u * D, v_new + u * D, Wt, scratch,
         [&]() {
             const int timed_out = !mbar_wait(&wbar, 0);
             if (__syncthreads_or(timed_out)) {  // same decision in every thread

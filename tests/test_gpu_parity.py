@@ -262,8 +262,14 @@ def test_append_matches_rebuild_bitwise(bf16):
     check_units(inc, w, K, V, Wp, pos, q, gout, gsel, grows, free_exact=not bf16)
 
 
-@pytest.mark.parametrize("bf16", [False, True])
-def test_fused_append_decode(bf16):
+@pytest.mark.parametrize("bf16,branching,k,start,steps", [
+    (False, 4, 2, [30, 61], 40),
+    (True, 4, 2, [30, 61], 40),
+    # first scored level of 960 candidates: the appending CTA keeps a share of
+    # the rows and refreshes the right-edge row in its tile after the append
+    (True, 64, 16, [61400, 61439], 3),
+])
+def test_fused_append_decode(bf16, branching, k, start, steps):
     """recsa_append_decode (one launch per step) leaves the node arrays and
     returns the selections and row counts of recsa_append then recsa_decode,
     bit for bit, across node and level boundaries (sequence 1 grows from 61
@@ -271,9 +277,7 @@ def test_fused_append_decode(bf16):
     splits the first level's rows differently over the cluster, so the
     per-CTA softmax sums are added in another order. The last step also
     matches the oracle."""
-    w = small(batch=2, n_kv_heads=2, group=4, head_dim=128, branching=4, k=2, bf16=bf16)
-    start = [30, 61]
-    steps = 40
+    w = small(batch=2, n_kv_heads=2, group=4, head_dim=128, branching=branching, k=k, bf16=bf16)
     cap = max(start) + steps
     K, V, runs = synth.cache_arrays(w, cap)
     Kd, Vd = parity.to_dev(K, bf16), parity.to_dev(V, bf16)
