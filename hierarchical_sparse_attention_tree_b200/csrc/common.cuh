@@ -133,22 +133,11 @@ __device__ __forceinline__ long long key_id(unsigned long long key) {
     return (long long)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
 }
 
-__device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int m) {
-    return __shfl_xor_sync(0xffffffffu, v, m);
-}
-
 __device__ __forceinline__ long long ceil_div_ll(long long a, long long b) { return (a + b - 1) / b; }
 
 // Number of nodes of level j over L tokens.
 __device__ __forceinline__ long long level_rows(const TreeParams& p, int j, long long L) {
     return j == 0 ? L : ceil_div_ll(L, p.span[j]);
-}
-
-// Top level J over L >= 1 tokens: the first level with at most b nodes.
-__device__ __forceinline__ int top_level(const TreeParams& p, long long L) {
-    int j = 1;
-    while (j < p.J_cap && level_rows(p, j, L) > p.b) j++;
-    return j;
 }
 
 __device__ __forceinline__ void flag_error(int* err, int bits) { atomicOr(err, bits); }
@@ -227,53 +216,6 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
 // Orders this thread's generic-proxy global accesses with async-proxy ones.
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// The two halves of this lane's PPL rotation pairs, (x_i, x_{i+D/2}) for
-// i = lane*PPL + e, as floats.
-template <typename T, int PPL, int HD>
-__device__ __forceinline__ void load_pairs(const T* row, int lane, float* a, float* b);
-
-template <>
-__device__ __forceinline__ void load_pairs<__nv_bfloat16, 2, 64>(const __nv_bfloat16* row, int lane, float* a,
-                                                                  float* b) {
-    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(row + lane * 2);
-    const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(row + 64 + lane * 2);
-    a[0] = __low2float(x); a[1] = __high2float(x);
-    b[0] = __low2float(y); b[1] = __high2float(y);
-}
-template <>
-__device__ __forceinline__ void load_pairs<__nv_bfloat16, 1, 32>(const __nv_bfloat16* row, int lane, float* a,
-                                                                  float* b) {
-    a[0] = __bfloat162float(row[lane]);
-    b[0] = __bfloat162float(row[32 + lane]);
-}
-template <>
-__device__ __forceinline__ void load_pairs<float, 2, 64>(const float* row, int lane, float* a, float* b) {
-    const float2 x = *reinterpret_cast<const float2*>(row + lane * 2);
-    const float2 y = *reinterpret_cast<const float2*>(row + 64 + lane * 2);
-    a[0] = x.x; a[1] = x.y;
-    b[0] = y.x; b[1] = y.y;
-}
-template <>
-__device__ __forceinline__ void load_pairs<float, 1, 32>(const float* row, int lane, float* a, float* b) {
-    a[0] = row[lane];
-    b[0] = row[32 + lane];
-}
-
-
-}  // namespace recsa
-
-
-namespace recsa {
-
-
-// Elements [i0, i0 + N) and [HD + i0, HD + i0 + N) of a row, as floats
-// (N = 4 or 8; 8- or 16-byte aligned vector loads).
-template <typename T, int N>
-__device__ __forceinline__ void load_half_rows(const T* row, int i0, int HD, float* a, float* b) {
-    load_vec<T, N>(row + i0, a);
-    load_vec<T, N>(row + HD + i0, b);
 }
 
 }  // namespace recsa

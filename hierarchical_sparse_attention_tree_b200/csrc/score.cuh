@@ -32,30 +32,6 @@ struct ScoreLayout {
     static_assert(G <= LPC && 32 % LPC == 0 && G <= 8, "scoring layout");
 };
 
-// Hint: bring RoPE table rows [row0, row0 + nrows) toward L1 (the table is
-// [npos][3][D/2] fp32). Threads tid, tid + nthr, ... each take 128-byte lines.
-template <int D>
-__device__ __forceinline__ void prefetch_rope_rows(const float* rope, int row0, int nrows, int tid, int nthr) {
-    constexpr int LINES = 3 * (D / 2) * 4 / 128;
-    static_assert(LINES * 128 == 3 * (D / 2) * 4, "whole lines per row");
-    const char* base = reinterpret_cast<const char*>(rope + (size_t)row0 * 3 * (D / 2));
-    for (int x = tid; x < nrows * LINES; x += nthr)
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(base + (size_t)x * 128));
-}
-
-// Hint: the query rotations of blocks [qa, qb] of a level with nc candidates
-// (RoPE rows nc - 1 - q*b).
-template <int D>
-__device__ __forceinline__ void prefetch_query_rotations(const float* rope, int nc, int b, int qa, int qb, int tid,
-                                                         int nthr) {
-    constexpr int LINES = 3 * (D / 2) * 4 / 128;
-    for (int x = tid; x < (qb - qa + 1) * LINES; x += nthr) {
-        const int q = qa + x / LINES, line = x - (x / LINES) * LINES;
-        const char* row = reinterpret_cast<const char*>(rope + (size_t)(nc - 1 - q * b) * 3 * (D / 2));
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(row + line * 128));
-    }
-}
-
 // Rotated query (all G heads, this lane's PL pairs) at angle `angle`.
 template <int D, int G>
 __device__ __forceinline__ void rotate_query(const float* rope, const float* qf, int angle, int gl,
