@@ -73,12 +73,12 @@ __host__ __device__ constexpr int dec_ncc() { return D / CPT; }
 template <int D>
 __host__ __device__ constexpr int dec_neg() { return DEC_THREADS / (D / CPT); }
 
-// Shared memory: [region0: K tile | V tile; at the end: entry-group partials,
-// then (rank 0) the cluster gather area][DecSmem][key: u64 MY][gkeys: u64
-// 2*CS*KMAX][qf G*D][lg MY*G (logits, then softmax weights)][cacc G*D][cml 2G]
+// Shared memory: [region0: K tile | V tile; at the end: entry-group partials]
+// [DecSmem][key: u64 MY][gkeys: u64 2*CS*KMAX][qf G*D][lg MY*G (logits, then
+// softmax weights)][cacc G*D][cml 2G][gat: (rank 0) the CTAs' states CS*(G*D + 2G)]
 __host__ __device__ inline size_t decode_smem_tail(int D, int G, int MY) {
     return sizeof(DecSmem) + (size_t)MY * 8 + (size_t)2 * DEC_CLUSTER * KMAX * 8 +
-           (size_t)(G * D + MY * G + G * D + 2 * G) * 4;
+           (size_t)(G * D + MY * G + G * D + 2 * G) * 4 + (size_t)DEC_CLUSTER * (G * D + 2 * G) * 4;
 }
 __host__ __device__ inline size_t decode_region0(int D, int G, int MY, int elem, int J_cap, bool fused) {
     // the appending CTA of a fused step first holds the pooler and the
@@ -90,8 +90,7 @@ __host__ __device__ inline size_t decode_region0(int D, int G, int MY, int elem,
     const size_t tiles = tiles0 > app ? tiles0 : app;
     const size_t eg = (size_t)(DEC_THREADS / (D / CPT)) * G * D * 4;
     const size_t eg_al = (eg + 127) & ~(size_t)127;
-    const size_t gat = (size_t)DEC_CLUSTER * (G * D + 2 * G) * 4;
-    const size_t need = eg_al + gat;
+    const size_t need = eg_al;
     const size_t r0 = tiles > need ? tiles : need;
     return (r0 + 127) & ~(size_t)127;
 }
@@ -235,7 +234,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
     T* Kt = reinterpret_cast<T*>(smem_raw);
     T* Vt = Kt + (size_t)MY * D;
     float* egacc = reinterpret_cast<float*>(smem_raw);  // [NEG][G][D], after the last tile
-    float* gat = reinterpret_cast<float*>(smem_raw + ((NEG * G * D * 4 + 127) & ~127));  // [CS][G*D + 2G]
     DecSmem* sm = reinterpret_cast<DecSmem*>(smem_raw + a.region0);
     unsigned long long* key = reinterpret_cast<unsigned long long*>(sm + 1);
     unsigned long long* gkeys = key + MY;  // [2][CS][KMAX]: the CTAs' top-k lists, by level parity
@@ -243,6 +241,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
     float* lg = qf + G * D;    // [MY][G] logits, then softmax weights
     float* cacc = lg + MY * G;
     float* cml = cacc + G * D;  // [G] max, [G] sum
+    float* gat = cml + 2 * G;   // [CS][G*D + 2G] (rank 0: every CTA's state)
 
     // set-up that does not read the tree (overlaps the previous kernel under
     // programmatic dependent launch)
@@ -627,8 +626,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
         cml[tid] = sm->M[tid];
         cml[G + tid] = s;
     }
-    cluster.sync();  // every CTA is done with its tiles: rank 0's gather area is free
-    {
+    __syncthreads();  // cacc and cml complete
+    {  // the gather area has a place of its own: no barrier needed before the push
         float* dst = cluster.map_shared_rank(gat, 0) + rank * (G * D + 2 * G);
         for (int idx = tid; idx < G * D + 2 * G; idx += DEC_THREADS) dst[idx] = idx < G * D ? cacc[idx] : cml[idx - G * D];
     }
