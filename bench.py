@@ -475,14 +475,20 @@ def main():
     e2e = None
     if not args.no_e2e:
         out_h = torch.empty((B, Hq, D), dtype=bf, pin_memory=True)
-        qb, kb, vb = torch.empty_like(q_d[0]), torch.empty_like(kn_d[0]), torch.empty_like(vn_d[0])
+        # each step's inputs arrive as one pinned host record [q | k_new | v_new]
+        # and cross PCIe in one copy; the kernels read them in place
+        nq, nkv = q_h[0].numel(), kn_h[0].numel()
+        rec_h = torch.cat([q_h.reshape(n_total, -1), kn_h.reshape(n_total, -1), vn_h.reshape(n_total, -1)],
+                          dim=1).pin_memory()
+        rec_d = torch.empty(nq + 2 * nkv, dtype=bf, device=dev)
+        qb = rec_d[:nq].view(q_d[0].shape)
+        kb = rec_d[nq:nq + nkv].view(kn_d[0].shape)
+        vb = rec_d[nq + nkv:].view(vn_d[0].shape)
 
         def e2e_step(s, ev=None):
             if ev is not None:
                 ev[0].record(stream)
-            qb.copy_(q_h[s], non_blocking=True)
-            kb.copy_(kn_h[s], non_blocking=True)
-            vb.copy_(vn_h[s], non_blocking=True)
+            rec_d.copy_(rec_h[s], non_blocking=True)
             layer.append_decode(kb, vb, qb, out)
             out_h.copy_(out, non_blocking=True)
             if ev is not None:

@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
                                    });
             const int kk = max(1, min(p.k, ncand));
             const int chunk = (nmy + W - 1) / W;  // rows per warp, as in the scoring
-            if (j > 0) {  // each warp's top keys, sorted (its own rows: a warp barrier suffices)
+            if (j > 0 && nmy > 1) {  // each warp's top keys, sorted (its own rows: a warp barrier suffices)
                 __syncwarp();
                 const int w_lo = warp * chunk, nw = max(0, min(nmy, w_lo + chunk) - w_lo);
                 unsigned long long* wl = sm->wl[warp];
@@ -532,15 +532,22 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
                 // this CTA's top keys, written to slot `rank` of every CTA's
                 // list area for this level
                 unsigned long long* gk = gkeys + (j & 1) * (DEC_CLUSTER * KMAX);
-                for (int t = tid; t < W * kk; t += DEC_THREADS) {
-                    const unsigned long long x = sm->wl[t / kk][t % kk];
-                    if (x == 0ull) continue;
-                    const int c = rank_in_lists<W>(&sm->wl[0][0], KMAX, kk, x);
-                    if (c < kk)
-                        for (int r = 0; r < CS; r++) cluster.map_shared_rank(gk, r)[rank * KMAX + c] = x;
+                if (nmy <= 1) {  // the list is this CTA's one key (or nothing): no sort, no merge
+                    for (int t = tid; t < CS * kk; t += DEC_THREADS) {
+                        const int r = t / kk, c = t - r * kk;
+                        cluster.map_shared_rank(gk, r)[rank * KMAX + c] = (c == 0 && nmy == 1) ? key[0] : 0ull;
+                    }
+                } else {
+                    for (int t = tid; t < W * kk; t += DEC_THREADS) {
+                        const unsigned long long x = sm->wl[t / kk][t % kk];
+                        if (x == 0ull) continue;
+                        const int c = rank_in_lists<W>(&sm->wl[0][0], KMAX, kk, x);
+                        if (c < kk)
+                            for (int r = 0; r < CS; r++) cluster.map_shared_rank(gk, r)[rank * KMAX + c] = x;
+                    }
+                    for (int t = nmy + tid; t < kk; t += DEC_THREADS)  // fewer rows than kk
+                        for (int r = 0; r < CS; r++) cluster.map_shared_rank(gk, r)[rank * KMAX + t] = 0ull;
                 }
-                for (int t = nmy + tid; t < kk; t += DEC_THREADS)  // fewer rows than kk
-                    for (int r = 0; r < CS; r++) cluster.map_shared_rank(gk, r)[rank * KMAX + t] = 0ull;
                 cluster.sync();
                 // global top-kk (the same in every CTA) and the kept ids in
                 // ascending order (ids are distinct)
