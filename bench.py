@@ -3,8 +3,8 @@
 
 Workload (default): one Qwen3-4B-shaped attention layer (32 query heads, 8 KV
 heads, head_dim 128, bf16), L = 524288 cached tokens per sequence, batch 4,
-branching 64, k = 16. One step = append one token to every sequence
-(recsa_append) + one decode query per sequence (recsa_decode). Inputs are
+branching 64, k = 16. One step = append one token to every sequence and
+one decode query per sequence, one launch (recsa_append_decode). Inputs are
 seeded synthetic data (Gaussian-mixture keys in token runs, N(0,1) values,
 queries aimed at a planted run, random pooler) resident in HBM before timing.
 
@@ -144,21 +144,37 @@ def dist_setup(n_gpus: int):
     return world, rank, local
 
 
-def barrier(world, local):
+def barrier(world, local, backend: str = "nccl"):
     if world > 1:
         import torch.distributed as dist
 
-        dist.barrier(device_ids=[local])
+        if backend == "nccl":
+            dist.barrier(device_ids=[local])
+        else:
+            dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's time: every rank's number is reduced with MAX."""
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_sequences(rank: int, batch: int) -> int:
+    """First generator sequence id of this rank's batch: ranks hold disjoint,
+    independent sequences (weak scaling, no collective on the data path)."""
+    return rank * batch
+
+
+def aggregate_rate(world: int, batch: int, steps: int, max_seconds: float) -> float:
+    """Whole-job query tokens per second: every rank's batch per step, over
+    the slowest rank's time."""
+    return world * batch * steps / max_seconds
 
 
 # --------------------------------------------------------- oracle baseline
@@ -340,7 +356,7 @@ def main():
     W_, K_ = args.warmup, args.steps
     n_total = 2 * (W_ + K_) + 25
     cap = L0 + n_total
-    seq_off = rank * B
+    seq_off = rank_sequences(rank, B)
     bf = torch.bfloat16
 
     # ---- inputs: host (pinned), then resident in HBM
@@ -423,7 +439,7 @@ def main():
     layer.check()
     step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     total_s = max_over_ranks(sum(step_ms) / 1e3, world)
-    value = world * B * K_ / total_s
+    value = aggregate_rate(world, B, K_, total_s)
     rows_np = rows.cpu().numpy()  # K and V rows each fused step's descent read
 
     # ---- for the record: the decode kernel alone (K launches on the current
@@ -508,7 +524,7 @@ def main():
         torch.cuda.synchronize(dev)
         barrier(world, local)
         e2e_s = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev2) / 1e3, world)
-        e2e = {"value": world * B * K_ / e2e_s, "unit": "query-tok/s",
+        e2e = {"value": aggregate_rate(world, B, K_, e2e_s), "unit": "query-tok/s",
                "h2d_bytes_per_step": int((q_h[0].numel() + kn_h[0].numel() + vn_h[0].numel()) * es),
                "d2h_bytes_per_step": int(out_h.numel() * es)}
         layer.check()
