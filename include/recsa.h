@@ -132,7 +132,9 @@ recsa_status recsa_append_decode(recsa_ctx* ctx, const void* k_new, const void* 
  * [B][C][H_kv][d], out [B][C][H_q][d] (device). sel_out (nullable, device
  * int32 [B][C][H_kv][J_cap][k]) as in recsa_decode. scratch: device memory
  * of recsa_prefill_scratch_bytes(cfg, C) bytes, 256-byte aligned. The chunk
- * is not appended: call recsa_append(k, v, C) afterwards. */
+ * is not appended: call recsa_append(k, v, C) afterwards. Built for bf16
+ * storage only (RECSA_ERR_UNSUPPORTED for fp32, or when k * b candidates
+ * per level exceed the kernel's shared memory). */
 size_t recsa_prefill_scratch_bytes(const recsa_config* cfg, int C);
 recsa_status recsa_prefill(recsa_ctx* ctx, const void* q, const void* k, const void* v, int C, void* out,
                            int* sel_out, void* scratch, size_t scratch_bytes, recsa_stream_t stream);
