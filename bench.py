@@ -66,13 +66,15 @@ def measured_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_traffic(kernel: str):
+def kernel_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
+    on the current kernel source for this workload (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)[kernel]
+        if d.get("workload") != workload:
+            return None
         src = b"".join(open(os.path.join(ROOT, f), "rb").read() for f in d["sources"])
         if hashlib.sha256(src).hexdigest()[:16] != d["source_sha"]:
             return None
@@ -580,7 +582,7 @@ def main():
                        "value_is": "decode query-tok/s; prefill tok/s under 'prefill'"},
             "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": achieved, "peak": hbm,
                          "unit": "GB/s", "frac": achieved / hbm, "peak_source": peak_src,
-                         "traffic": kernel_traffic("decode_kernel"),
+                         "traffic": kernel_traffic("decode_kernel", w.name),
                          "algorithmic_bytes_per_launch": dec_bytes_per_launch, "launch_ms": dec_avg_s * 1e3},
             "append_ms": sum(app_ms) / len(app_ms), "decode_ms": sum(dec_ms) / K_,
             "split_step_ms": sum(split_ms) / len(split_ms),
