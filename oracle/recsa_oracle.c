@@ -45,6 +45,12 @@
  *   R11 RoPE: rotate-half pairs (i, i + d/2), theta_i = base^(-2i/d).
  *   R12 node keys and values are rounded to the storage type once, when
  *      formed; child keys are read as stored.
+ *
+ * Parity unpinned: R6 at levels >= 1 (the query position there; level 0 is
+ * pinned by the dense equivalence), R7's absence of a subtree-size bias, and
+ * R8 are fixed only by these readings. Every other step is pinned by the
+ * tests against the dense closed form, exact subtree means, the read bound,
+ * an independent brute force and hand-derived examples.
  */
 #include "recsa_oracle.h"
 
