@@ -31,8 +31,9 @@ template <int D>
 cudaError_t launch_prefill_local(const TreeParams&, const void*, const void*, const void*, float*, int, int, int, int,
                                  cudaStream_t);
 template <typename T, int D, int G>
-cudaError_t launch_prefill_tree(const TreeParams&, const void*, void*, const float*, int*, int, int, int,
+cudaError_t launch_prefill_tree(const TreeParams&, const void*, void*, const float*, int*, long long*, int, int, int,
                                 cudaStream_t);
+size_t decode_smem_bytes(int D, int G, int elem, int k, int b, int J_cap, bool fused);
 size_t prefill_tree_smem_bytes(int D, int G, int elem, int k, int b);
 size_t dense_static_scratch_bytes();
 cudaError_t dense_static_scratch(float** out);
@@ -110,7 +111,7 @@ struct Layout {
     int J_cap, npos;
     long long rows[MAXJ + 1];
     size_t off_K[MAXJ + 1], off_V[MAXJ + 1], off_VS[MAXJ + 1], off_PK[MAXJ + 1], off_PV[MAXJ + 1];
-    size_t off_Wt, off_rope, off_len, off_err, off_stage, total;
+    size_t off_Wt, off_rope, off_len, off_stats, off_err, off_stage, total;
 };
 
 Layout layout_for(const recsa_config* c) {
@@ -135,6 +136,7 @@ Layout layout_for(const recsa_config* c) {
     l.off_Wt = o; o = align256(o + D * D * es);
     l.off_rope = o; o = align256(o + (size_t)l.npos * 3 * (D / 2) * 4);
     l.off_len = o; o = align256(o + units * 8);
+    l.off_stats = o; o = align256(o + units * 3 * 8);
     l.off_err = o; o = align256(o + 4);
     l.off_stage = o; o = align256(o + (size_t)c->batch * 8);
     l.total = o;
@@ -198,6 +200,14 @@ recsa_status recsa_init(recsa_ctx** out, const recsa_config* cfg, void* k_cache,
     if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return fail(RECSA_ERR_INVALID_ARG, "cache not 16-byte aligned");
     if (!aligned(workspace, 256)) return fail(RECSA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
     Layout l = layout_for(cfg);
+    {
+        const int G = cfg->n_q_heads / cfg->n_kv_heads, elem = cfg->dtype == RECSA_BF16 ? 2 : 4;
+        const size_t need = decode_smem_bytes(cfg->head_dim, G, elem, cfg->k, cfg->branching, l.J_cap, true);
+        if (need > 227 * 1024)
+            return fail(RECSA_ERR_UNSUPPORTED,
+                        "k * branching = %d candidates per level need %zu bytes of decode shared memory (> 227 KB)",
+                        cfg->k * cfg->branching, need);
+    }
     if (workspace_bytes < l.total)
         return fail(RECSA_ERR_CAPACITY, "workspace has %zu bytes, needs %zu", workspace_bytes, l.total);
 
@@ -225,6 +235,7 @@ recsa_status recsa_init(recsa_ctx** out, const recsa_config* cfg, void* k_cache,
     p.Wt = ws + l.off_Wt;
     p.rope = reinterpret_cast<float*>(ws + l.off_rope);
     p.len = reinterpret_cast<long long*>(ws + l.off_len);
+    p.stats = reinterpret_cast<long long*>(ws + l.off_stats);
     p.err = reinterpret_cast<int*>(ws + l.off_err);
     p.scale = (float)(1.0 / std::sqrt((double)D));
     c->len_stage = reinterpret_cast<long long*>(ws + l.off_stage);
@@ -244,6 +255,7 @@ recsa_status recsa_init(recsa_ctx** out, const recsa_config* cfg, void* k_cache,
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemcpyAsync((void*)p.rope, tab.data(), tab.size() * sizeof(float), cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(p.len, 0, (size_t)p.B * p.H * 8, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(p.stats, 0, (size_t)p.B * p.H * 3 * 8, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(p.err, 0, 4, s);
     if (e == cudaSuccess) {
         pooler_transpose_kernel<<<(D * D + 255) / 256, 256, 0, s>>>(pooler_w, cfg->dtype == RECSA_BF16, D,
@@ -354,7 +366,8 @@ size_t recsa_prefill_scratch_bytes(const recsa_config* cfg, int C) {
 }
 
 recsa_status recsa_prefill(recsa_ctx* ctx, const void* q, const void* k, const void* v, int C, void* out,
-                           int* sel_out, void* scratch, size_t scratch_bytes, recsa_stream_t stream) {
+                           int* sel_out, long long* rows_out, void* scratch, size_t scratch_bytes,
+                           recsa_stream_t stream) {
     if (!ctx || !q || !k || !v || !out || !scratch) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
     const recsa_config& c = ctx->cfg;
     if (c.dtype != RECSA_BF16) return fail(RECSA_ERR_UNSUPPORTED, "prefill is built for bf16 storage only");
@@ -381,11 +394,11 @@ recsa_status recsa_prefill(recsa_ctx* ctx, const void* q, const void* k, const v
         using T = __nv_bfloat16;
         if (c.head_dim == 64) {
             constexpr int DD = 64;
-            DISPATCH_G(ctx->G, e = launch_prefill_tree<T, DD, GG>(ctx->p, q, out, state, sel_out, c.batch, C,
+            DISPATCH_G(ctx->G, e = launch_prefill_tree<T, DD, GG>(ctx->p, q, out, state, sel_out, rows_out, c.batch, C,
                                                                   c.n_q_heads, s));
         } else {
             constexpr int DD = 128;
-            DISPATCH_G(ctx->G, e = launch_prefill_tree<T, DD, GG>(ctx->p, q, out, state, sel_out, c.batch, C,
+            DISPATCH_G(ctx->G, e = launch_prefill_tree<T, DD, GG>(ctx->p, q, out, state, sel_out, rows_out, c.batch, C,
                                                                   c.n_q_heads, s));
         }
     }
@@ -414,6 +427,23 @@ recsa_status recsa_level_arrays(const recsa_ctx* ctx, int level, void** keys, vo
     if (keys) *keys = ctx->p.K[level];
     if (values) *values = ctx->p.V[level];
     if (value_sums) *value_sums = ctx->p.VS[level];
+    return RECSA_OK;
+}
+
+recsa_status recsa_query_stats(recsa_ctx* ctx, int* depth, long long* k_rows, long long* v_rows,
+                               recsa_stream_t stream) {
+    if (!ctx) return fail(RECSA_ERR_INVALID_ARG, "NULL context");
+    const size_t units = (size_t)ctx->p.B * ctx->p.H;
+    std::vector<long long> st(units * 3);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemcpy(st.data(), ctx->p.stats, units * 3 * 8, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_query_stats");
+    for (size_t u = 0; u < units; u++) {
+        if (depth) depth[u] = (int)st[u * 3];
+        if (k_rows) k_rows[u] = st[u * 3 + 1];
+        if (v_rows) v_rows[u] = st[u * 3 + 2];
+    }
     return RECSA_OK;
 }
 

@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace recsa {
 
 constexpr int MAXJ = 32;  // levels kept above the tokens (b >= 2, capacity < 2^32)
@@ -32,6 +34,7 @@ struct TreeParams {
     const void* Wt;            // pooler, transposed, storage type: Wt[c * D + r] = W[r][c]
     const float* rope;         // [npos][3][D/2]: cos, sin, -sin of (p * theta_i), theta_i = base^(-2i/d)
     long long* len;            // [B*H] tokens held by each unit
+    long long* stats;          // [B*H][3] last decode: depth, K rows read, V rows read
     int* err;                  // device error word
     float scale;               // 1 / sqrt(D)
 };
@@ -141,6 +144,21 @@ __device__ __forceinline__ long long level_rows(const TreeParams& p, int j, long
 }
 
 __device__ __forceinline__ void flag_error(int* err, int bits) { atomicOr(err, bits); }
+
+// Raises a kernel's dynamic shared memory limit on the current device, once
+// per device and kernel (the attribute is per device; `done` is a bit mask
+// of devices 0..63, higher devices set it on every call).
+template <typename F>
+inline cudaError_t set_smem_limit(F kern, int bytes, std::atomic<unsigned long long>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
 
 }  // namespace recsa
 

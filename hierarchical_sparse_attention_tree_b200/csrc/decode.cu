@@ -656,20 +656,32 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
             }
             outp[idx] = from_f<T>(bad ? 0.f : s / lsum);
         }
-        if (tid == 0 && a.rows_out) {
-            a.rows_out[u * 2] = krows;
-            a.rows_out[u * 2 + 1] = vrows;
+        int J = 0;
+        if (!bad_len) {
+            J = 1;
+            while (J < p.J_cap && sm->nlev[J] > b) J++;
         }
-        if (a.sel_out) {
-            int J = 0;
-            if (!bad_len) {
-                J = 1;
-                while (J < p.J_cap && sm->nlev[J] > b) J++;
+        if (tid == 0) {
+            if (a.rows_out) {
+                a.rows_out[u * 2] = krows;
+                a.rows_out[u * 2 + 1] = vrows;
             }
+            p.stats[u * 3] = bad_len ? 0 : J + 1;
+            p.stats[u * 3 + 1] = krows;
+            p.stats[u * 3 + 2] = vrows;
+        }
+        if (a.sel_out)
             for (int i = tid; i < (p.J_cap - J) * p.k; i += DEC_THREADS)
                 a.sel_out[(u * p.J_cap + J) * p.k + i] = -1;
-        }
     }
+}
+
+// Dynamic shared memory of one decode CTA (fused: the appending CTA's
+// pooler and scratch included).
+size_t decode_smem_bytes(int D, int G, int elem, int k, int b, int J_cap, bool fused) {
+    const long long maxc = (long long)k * b > b ? (long long)k * b : b;
+    const int my = (int)((maxc + DEC_CLUSTER - 1) / DEC_CLUSTER);
+    return decode_region0(D, G, my, elem, J_cap, fused) + decode_smem_tail(D, G, my);
 }
 
 // k_new, v_new: null for a decode alone; else the fused step (append the
@@ -684,13 +696,10 @@ cudaError_t launch_decode(const TreeParams& p, const void* k_new, const void* v_
     a.region0 = (int)decode_region0(D, G, a.my_max, (int)sizeof(T), p.J_cap, fused);
     const size_t smem = a.region0 + decode_smem_tail(D, G, a.my_max);
     auto kern = decode_kernel<T, D, G>;
-    static bool attr_set = false;  // per instantiation
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
+    static std::atomic<unsigned long long> attr_done{0};  // per instantiation, per device
+    cudaError_t e = set_smem_limit(kern, 227 * 1024, attr_done);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(CS, p.B * p.H, 1);
     cfg.blockDim = dim3(DEC_THREADS, 1, 1);

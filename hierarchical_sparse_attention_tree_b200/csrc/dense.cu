@@ -1,5 +1,5 @@
-// Dense GQA flash-decode: the comparator the RecSA pages measure against
-// ("faster than dense attention ... at 524K on one H200 GPU", abstract).
+// Dense GQA flash-decode: the comparator for RecSA's speed claim (the RecSA
+// abstract reports end-to-end speedups over dense attention at 524K tokens).
 // Not part of the method. One query per sequence attends every cached token;
 // keys are used as stored (a dense cache holds keys already rotated).
 //

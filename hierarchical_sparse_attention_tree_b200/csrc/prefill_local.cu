@@ -3,8 +3,8 @@
 //
 // In a prefill chunk [s, s+C) the query of token t sees, after the tree's
 // entries, the chunk's tokens s..t exactly; those follow the level-0
-// candidates in the RoPE index order (RecSA abstract: "each entry's RoPE
-// position is its index among the candidates of its level"). Only index
+// candidates in the RoPE index order (kongchang.com article, "Position
+// Encoding": positions are ranks within a level's candidate list). Only index
 // differences enter a logit, so this part is ordinary causal attention with
 // the query at t - s and the keys at u - s, whatever the tree selected; its
 // softmax state (running max, sum, unnormalised output) is merged with the
@@ -220,7 +220,8 @@ cudaError_t launch_prefill_local(const TreeParams& p, const void* q, const void*
                        (float)(1.0 / sqrt((double)D))};
     const size_t smem = (size_t)3 * PL_TILE * (D + 8) * sizeof(__nv_bfloat16);
     auto kern = prefill_local_kernel<D>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<unsigned long long> attr_done{0};
+    cudaError_t e = set_smem_limit(kern, (int)smem, attr_done);
     if (e != cudaSuccess) return e;
     dim3 grid((C + PL_TILE - 1) / PL_TILE, B * Hq);
     kern<<<grid, PL_THREADS, smem, s>>>(p, a);

@@ -32,6 +32,7 @@ struct PrefillTreeArgs {
     void* out;           // [B][C][Hq][D]
     const float* state;  // [B][C][Hq][D + 2] local part: unnormalised acc, max, sum
     int* sel_out;        // nullable [B][C][H][J_cap][k]
+    long long* rows_out;  // nullable [B][C][H][2]: key rows scored, value rows (softmax entries)
     int C, Hq;
     int maxc;            // most candidates a level can have
     int sortn;           // power of two >= maxc
@@ -267,6 +268,7 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
     };
 
     int J = 0;
+    long long krows = 0, vrows = 0;
     if (!bad_len && S > 0) {
         J = 1;
         while (J < p.J_cap && sm->nlev[J] > b) J++;  // top level of the tree over S tokens
@@ -283,6 +285,8 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
             }
             const int kk = min(p.k, ncand);
             if (ncand > p.k) {
+                krows += ncand;
+                vrows += ncand - kk;
                 // score every candidate, tile by tile; the next tile is in
                 // flight while one is scored
                 const int nt = (ncand + PT_TILE - 1) / PT_TILE;
@@ -400,6 +404,8 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
         // order) the chunk's own tokens, already in the local state
         const int n0 = bad ? 0 : ncand_of(0, npar);
         const int P0 = n0 + t;
+        krows += n0;
+        vrows += n0;
         // keys and values of half-size tiles together, the next tile in flight
         constexpr int T0 = PT_TILE / 2;
         const int nt0 = (n0 + T0 - 1) / T0;
@@ -414,6 +420,11 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
             accumulate(tile(bi) + (size_t)T0 * D, r0, nmy, true);
             __syncthreads();
         }
+    }
+    if (a.rows_out && tid == 0) {  // the chunk's own tokens s..t are entries too
+        long long* r = a.rows_out + (((size_t)bseq * a.C + t) * p.H + h) * 2;
+        r[0] = krows;
+        r[1] = vrows + t + 1;
     }
     if (a.sel_out) {
         int* selrow = a.sel_out + (((size_t)bseq * a.C + t) * p.H + h) * p.J_cap * p.k;
@@ -465,14 +476,15 @@ __global__ void __launch_bounds__(PT_THREADS, 2) prefill_tree_kernel(TreeParams 
 
 template <typename T, int D, int G>
 cudaError_t launch_prefill_tree(const TreeParams& p, const void* q, void* out, const float* state, int* sel_out,
-                                int B, int C, int Hq, cudaStream_t s) {
-    PrefillTreeArgs a{q, out, state, sel_out, C, Hq, 0, 1};
+                                long long* rows_out, int B, int C, int Hq, cudaStream_t s) {
+    PrefillTreeArgs a{q, out, state, sel_out, rows_out, C, Hq, 0, 1};
     a.maxc = p.k * p.b > p.b ? p.k * p.b : p.b;
     while (a.sortn < a.maxc) a.sortn <<= 1;
     const size_t smem = prefill_tree_smem(D, G, (int)sizeof(T), a.maxc, a.sortn);
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     auto kern = prefill_tree_kernel<T, D, G>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    static std::atomic<unsigned long long> attr_done{0};
+    cudaError_t e = set_smem_limit(kern, 227 * 1024, attr_done);
     if (e != cudaSuccess) return e;
     dim3 grid(C, B * p.H);
     kern<<<grid, PT_THREADS, smem, s>>>(p, a);
@@ -487,7 +499,7 @@ size_t prefill_tree_smem_bytes(int D, int G, int elem, int k, int b) {
 
 #define RECSA_INST_PT(T, D, G)                                                                                   \
     template cudaError_t launch_prefill_tree<T, D, G>(const TreeParams&, const void*, void*, const float*, int*, \
-                                                      int, int, int, cudaStream_t);
+                                                      long long*, int, int, int, cudaStream_t);
 #define RECSA_INST_PT_G(T, D) RECSA_INST_PT(T, D, 1) RECSA_INST_PT(T, D, 2) RECSA_INST_PT(T, D, 4) RECSA_INST_PT(T, D, 8)
 RECSA_INST_PT_G(__nv_bfloat16, 64)
 RECSA_INST_PT_G(__nv_bfloat16, 128)

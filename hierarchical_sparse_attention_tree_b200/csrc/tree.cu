@@ -1,9 +1,9 @@
 // Tree build and append kernels.
 //
-// "RecSA ... builds a tree over the KV cache in which each node summarizes its
-// subtree with one key and one mean-pooled value. The keys come from one
-// pooler per layer, shared by all levels" (abstract, paraphrased); node value
-// = mean of every token value in the subtree ("Core Idea", mean pooling).
+// The tree over the KV cache (RecSA abstract): every node stands for its
+// subtree through a single key and a single value; the value is the average
+// of the subtree's token values (kongchang.com article, "Core Idea"), the key
+// comes from the layer's one pooler, which every level uses (abstract).
 //
 // Arithmetic contract, shared by every path that writes a node so that a tree
 // grown token by token is bit-identical to one built at once:
@@ -221,7 +221,8 @@ cudaError_t launch_build_level(const TreeParams& p, int j, long long add, int fr
     const int threads = 256, wpb = threads / 32;
     size_t smem = (size_t)D * D * sizeof(T) + (size_t)wpb * D * sizeof(float);
     auto kern = build_level_kernel<T, D>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<unsigned long long> attr_done{0};
+    cudaError_t e = set_smem_limit(kern, (int)smem, attr_done);
     if (e != cudaSuccess) return e;
     long long gx = (max_nodes + wpb - 1) / wpb;
     if (gx < 1) gx = 1;
@@ -234,7 +235,8 @@ template <typename T, int D>
 cudaError_t launch_append_one(const TreeParams& p, const void* k_new, const void* v_new, cudaStream_t s) {
     size_t smem = (size_t)D * D * sizeof(T) + append_scratch_floats(D, p.J_cap) * sizeof(float);
     auto kern = append_one_kernel<T, D>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<unsigned long long> attr_done{0};
+    cudaError_t e = set_smem_limit(kern, (int)smem, attr_done);
     if (e != cudaSuccess) return e;
     kern<<<p.B * p.H, D, smem, s>>>(p, reinterpret_cast<const T*>(k_new), reinterpret_cast<const T*>(v_new));
     return cudaGetLastError();

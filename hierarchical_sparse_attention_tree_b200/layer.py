@@ -51,14 +51,17 @@ class RecsaLayer:
         self.ctx.append_decode(k_new, v_new, q, out, sel_out, rows_out, stream)
         return out
 
-    def prefill(self, q, k, v, out=None, sel_out=None, stream=None):
+    def prefill(self, q, k, v, out=None, sel_out=None, rows_out=None, stream=None):
         if out is None:
             out = torch.empty_like(q)
         need = self.ctx.prefill_scratch_bytes(q.shape[1])
         if self._scratch is None or self._scratch.numel() < need:
             self._scratch = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
-        self.ctx.prefill(q, k, v, out, sel_out, self._scratch, stream)
+        self.ctx.prefill(q, k, v, out, sel_out, self._scratch, rows_out, stream)
         return out
+
+    def query_stats(self, stream=None):
+        return self.ctx.query_stats(stream)
 
     def lengths(self):
         return self.ctx.lengths()

@@ -21,7 +21,7 @@ _TORCH_DTYPE = {F32: torch.float32, BF16: torch.bfloat16}
 EXPORTS = [
     "recsa_workspace_bytes", "recsa_init", "recsa_build_tree", "recsa_append", "recsa_decode", "recsa_append_decode",
     "recsa_prefill_scratch_bytes", "recsa_prefill", "recsa_get_lengths", "recsa_tree_shape", "recsa_level_arrays",
-    "recsa_check_device", "recsa_last_error", "recsa_destroy", "recsa_dense_decode_scratch_bytes",
+    "recsa_query_stats", "recsa_check_device", "recsa_last_error", "recsa_destroy", "recsa_dense_decode_scratch_bytes",
     "recsa_dense_decode", "recsa_dense_decode_static",
 ]
 
@@ -59,7 +59,8 @@ def lib():
             "recsa_decode": (i32, [vp, vp, vp, vp, vp, vp]),
             "recsa_append_decode": (i32, [vp, vp, vp, vp, vp, vp, vp, vp]),
             "recsa_prefill_scratch_bytes": (sz, [P(Config), i32]),
-            "recsa_prefill": (i32, [vp, vp, vp, vp, i32, vp, vp, vp, sz, vp]),
+            "recsa_prefill": (i32, [vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
+            "recsa_query_stats": (i32, [vp, P(i32), P(i64), P(i64), vp]),
             "recsa_get_lengths": (i32, [vp, P(i64)]),
             "recsa_tree_shape": (i32, [vp, P(i32), P(i64)]),
             "recsa_level_arrays": (i32, [vp, i32, P(vp), P(vp), P(vp)]),
@@ -168,11 +169,28 @@ class Context:
         _check(lib().recsa_append_decode(self.handle, _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(out), _ptr(sel_out),
                                          _ptr(rows_out), _stream(stream)))
 
-    def prefill(self, q, k, v, out, sel_out=None, scratch=None, stream=None):
+    def append_decode_ptrs(self, k_new: int, v_new: int, q: int, out: int, sel_out=None, rows_out=None,
+                           stream=None):
+        """recsa_append_decode on raw addresses: device memory, or pinned host
+        memory mapped into the device's address space (the kernel then reads
+        the inputs and writes the output over the bus)."""
+        vp = ctypes.c_void_p
+        _check(lib().recsa_append_decode(self.handle, vp(k_new), vp(v_new), vp(q), vp(out), _ptr(sel_out),
+                                         _ptr(rows_out), _stream(stream)))
+
+    def prefill(self, q, k, v, out, sel_out=None, scratch=None, rows_out=None, stream=None):
         C = q.shape[1]
         nbytes = 0 if scratch is None else scratch.numel() * scratch.element_size()
         _check(lib().recsa_prefill(self.handle, _ptr(q), _ptr(k), _ptr(v), C, _ptr(out), _ptr(sel_out),
-                                   _ptr(scratch), nbytes, _stream(stream)))
+                                   _ptr(rows_out), _ptr(scratch), nbytes, _stream(stream)))
+
+    def query_stats(self, stream=None):
+        """(depth, k_rows, v_rows) of the last decode, per (sequence, KV head)
+        unit, as lists of B * H_kv host integers."""
+        n = self.cfg.batch * self.cfg.n_kv_heads
+        d, kr, vr = (ctypes.c_int * n)(), (ctypes.c_longlong * n)(), (ctypes.c_longlong * n)()
+        _check(lib().recsa_query_stats(self.handle, d, kr, vr, _stream(stream)))
+        return list(d), list(kr), list(vr)
 
     def prefill_scratch_bytes(self, C: int) -> int:
         return lib().recsa_prefill_scratch_bytes(ctypes.byref(self.cfg), C)

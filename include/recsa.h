@@ -36,6 +36,10 @@
  *   append     k_new, v_new [B][n][H_kv][d]
  *   prefill    q, out [B][C][H_q][d]; k, v [B][C][H_kv][d]
  *
+ * Pointers documented as "device" may also be pinned host memory that is
+ * mapped into the device's address space (cudaHostAlloc memory under unified
+ * addressing): the kernels then read or write it over the bus.
+ *
  * Streams. Every call that launches work is asynchronous on the given
  * stream (a cudaStream_t; NULL = legacy default stream). Argument errors are
  * detected on the host, return a status and launch nothing;
@@ -93,15 +97,22 @@ recsa_status recsa_init(recsa_ctx** out, const recsa_config* cfg, void* k_cache,
 
 /* Sets sequence b's length to lengths[b] (host array of B entries, each in
  * [0, capacity]) and builds every tree level from the tokens already in the
- * cache ("builds a tree over the KV cache", abstract). */
+ * cache. The tree is the one the RecSA abstract keeps over the KV cache: node
+ * values are subtree means of the token values, node keys the layer's pooler
+ * applied to the mean of the children's keys (kongchang.com article, "Core
+ * Idea": mean pooling of values, learned pooling of keys). */
 recsa_status recsa_build_tree(recsa_ctx* ctx, const long long* lengths, recsa_stream_t stream);
 
 /* Appends n >= 1 tokens to every sequence: copies k_new / v_new
  * ([B][n][H_kv][d], device) into the cache after each sequence's current
- * tokens, then brings every node whose subtree gained tokens up to date
- * (right-edge nodes stay exact means; keys are recomputed by the pooler).
- * RECSA_ERR_CAPACITY (nothing launched) if any sequence would exceed the
- * capacity. */
+ * tokens, then brings every node whose subtree gained tokens up to date, so
+ * that the tree stays the one over the whole cache (RecSA abstract: the tree
+ * lives over the KV cache and grows with it; kongchang.com "Core Idea": node
+ * value = mean of its tokens, node key = pooler of its children's keys).
+ * Right-edge nodes stay exact means; their keys are recomputed by the pooler.
+ * A prefill chunk is appended with this call after recsa_prefill (the tree is
+ * updated after each chunk). RECSA_ERR_CAPACITY (nothing launched) if any
+ * sequence would exceed the capacity. */
 recsa_status recsa_append(recsa_ctx* ctx, const void* k_new, const void* v_new, int n, recsa_stream_t stream);
 
 /* One decode query per sequence (per-level top-k descent, shared softmax and
@@ -126,18 +137,26 @@ recsa_status recsa_append_decode(recsa_ctx* ctx, const void* k_new, const void* 
                                  int* sel_out, long long* rows_out, recsa_stream_t stream);
 
 /* Chunked causal prefill of C tokens per sequence (1 <= C <= max_chunk):
- * token t of the chunk attends the tree over the sequence's cached tokens
- * [0, s) plus the chunk's own tokens s..t exactly; those follow the level-0
- * candidates in the RoPE index order. q [B][C][H_q][d], k, v
+ * token t of the chunk runs the same descent as a decode query (RecSA
+ * abstract: top-down selection of at most k nodes per level, one softmax over
+ * the unselected summaries and the exact tokens, RoPE at candidate indices;
+ * kongchang.com "Core Idea" and "Position Encoding") over the tree of the
+ * sequence's cached tokens [0, s), and also attends the chunk's own tokens
+ * s..t exactly, which follow the level-0 candidates in the RoPE index order
+ * (causality inside the chunk is this library's reading: the pages do not
+ * spell out chunked prefill). q [B][C][H_q][d], k, v
  * [B][C][H_kv][d], out [B][C][H_q][d] (device). sel_out (nullable, device
- * int32 [B][C][H_kv][J_cap][k]) as in recsa_decode. scratch: device memory
+ * int32 [B][C][H_kv][J_cap][k]) as in recsa_decode. rows_out (nullable,
+ * device int64 [B][C][H_kv][2]): key rows scored and value rows (softmax
+ * entries, the chunk's own tokens included) per token and KV head. scratch: device memory
  * of recsa_prefill_scratch_bytes(cfg, C) bytes, 256-byte aligned. The chunk
  * is not appended: call recsa_append(k, v, C) afterwards. Built for bf16
  * storage only (RECSA_ERR_UNSUPPORTED for fp32, or when k * b candidates
  * per level exceed the kernel's shared memory). */
 size_t recsa_prefill_scratch_bytes(const recsa_config* cfg, int C);
 recsa_status recsa_prefill(recsa_ctx* ctx, const void* q, const void* k, const void* v, int C, void* out,
-                           int* sel_out, void* scratch, size_t scratch_bytes, recsa_stream_t stream);
+                           int* sel_out, long long* rows_out, void* scratch, size_t scratch_bytes,
+                           recsa_stream_t stream);
 
 /* Host-side view of the state, for tests and tools. */
 recsa_status recsa_get_lengths(const recsa_ctx* ctx, long long* lengths /* host [B] */);
@@ -147,8 +166,23 @@ recsa_status recsa_tree_shape(const recsa_ctx* ctx, int* j_cap, long long* rows 
  * in cfg->dtype, and the fp32 value sums [B][H_kv][rows[j]][d]. */
 recsa_status recsa_level_arrays(const recsa_ctx* ctx, int level, void** keys, void** values, float** value_sums);
 
+/* Per-unit statistics of the most recent recsa_decode or
+ * recsa_append_decode on this context, for checking the logarithmic read
+ * cost the RecSA abstract claims (a query reads O(log L) entries). Waits for
+ * `stream`, then fills, for every (sequence, KV head) unit u = b * H_kv + h:
+ *   depth[u]  levels the query descended, the tokens included (J + 1);
+ *   k_rows[u] key rows read (node keys and token keys; levels that keep all
+ *             of their at most k candidates are not read);
+ *   v_rows[u] value rows read, which is the number of softmax entries.
+ * Host arrays of B * H_kv entries each; any may be NULL. All zero before the
+ * first decode. RECSA_ERR_CUDA if the stream reports an error. */
+recsa_status recsa_query_stats(recsa_ctx* ctx, int* depth, long long* k_rows, long long* v_rows,
+                               recsa_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the device error word:
- * RECSA_ERR_DEVICE if a kernel flagged an inconsistent state. */
+ * RECSA_ERR_DEVICE if a kernel flagged an inconsistent state (bits: 1 a
+ * length out of range, 2 a tree shape inconsistent with the lengths, 4 a
+ * bounded wait for an asynchronous copy ran out, about a second). */
 recsa_status recsa_check_device(recsa_ctx* ctx, recsa_stream_t stream);
 
 const char* recsa_last_error(void);
@@ -178,7 +212,10 @@ recsa_status recsa_dense_decode(const void* k_cache, const void* v_cache, const 
  * shrinks to fit. The first call on each device looks up the array's device
  * address (with that device current), so make it before any stream capture.
  * All calls share the one array: calls whose kernels overlap on a device
- * (for example on two streams) race and corrupt each other's results. */
+ * (for example on two streams) race and corrupt each other's results. The
+ * looked-up address is kept for the life of the process: after
+ * cudaDeviceReset on a device (which unloads the library's device code
+ * there) do not call this entry point on that device again. */
 recsa_status recsa_dense_decode_static(const void* k_cache, const void* v_cache, const void* q, void* out, int batch,
                                        int n_kv_heads, int n_q_heads, int head_dim, long long length,
                                        long long l_stride, recsa_dtype dtype, recsa_stream_t stream);

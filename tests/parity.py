@@ -1,6 +1,9 @@
 """Helpers that compare the CUDA path with the fp64 oracle (tests only)."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -93,26 +96,50 @@ def q_unit(q: np.ndarray, b: int, h: int, G: int) -> np.ndarray:
     return synth.as_f32(np.ascontiguousarray(q[b, h * G:(h + 1) * G]))
 
 
+def first_tie_level(ref):
+    """Highest level whose oracle margin S_(k) - S_(k+1) is below NEAR_TIE
+    (the descent runs from level J down), or 0 if there is none. Selections
+    at that level and below may legitimately differ from the oracle's."""
+    for j in range(ref["J"], 0, -1):
+        if ref["margin"][j - 1] < NEAR_TIE:
+            return j
+    return 0
+
+
 def check_decode(gpu_out, gpu_sel, gpu_rows, ref, b, h, G, tol, report):
-    """Compares one unit's decode with an oracle result; near ties are counted
-    and skipped."""
-    if len(ref["margin"]) and ref["margin"].min() < NEAR_TIE:
-        report["near_ties"] += 1
-        return
+    """Compares one unit's decode with an oracle result. Levels above the
+    first near tie must select exactly what the oracle selects; at and below
+    it a different selection is counted as a near tie and the output is not
+    compared. Where every level agrees (near tie or not) the output and the
+    rows read are compared too."""
     J = ref["J"]
-    for j in range(1, J + 1):
+    tie = first_tie_level(ref)
+    if tie:
+        report["near_ties"] += 1
+    for j in range(J, 0, -1):
         got = [x for x in gpu_sel[b, h, j - 1].tolist() if x >= 0]
         want = [x for x in ref["sel"][j - 1].tolist() if x >= 0]
         if got != want:
+            if j <= tie:
+                report["near_tie_sel_diff"] += 1
+                return False
             report["sel_mismatch"] += 1
             report.setdefault("first_mismatch", (b, h, j, got, want))
-            return
+            return False
     assert (gpu_sel[b, h, J:] == -1).all()
     err = np.abs(gpu_out[b, h * G:(h + 1) * G] - ref["out"]).max()
     report["max_abs"] = max(report["max_abs"], float(err))
     assert err <= tol, (b, h, err)
     assert tuple(gpu_rows[b, h]) == expected_rows(ref), (gpu_rows[b, h], expected_rows(ref))
     report["checked"] += 1
+    return True
+
+
+def same_selection(ref_a, ref_b):
+    """True if two oracle results keep the same nodes at every level."""
+    if ref_a["J"] != ref_b["J"]:
+        return False
+    return all((ref_a["sel"][j] == ref_b["sel"][j]).all() for j in range(ref_a["J"]))
 
 
 def expected_rows(ref):
@@ -129,4 +156,27 @@ def expected_rows(ref):
 
 
 def new_report():
-    return {"checked": 0, "near_ties": 0, "sel_mismatch": 0, "max_abs": 0.0}
+    return {"queries": 0, "checked": 0, "near_ties": 0, "near_tie_sel_diff": 0, "sel_mismatch": 0,
+            "node_rounding_flips": 0, "max_abs": 0.0}
+
+
+def merge_reports(total, rep):
+    for key, v in rep.items():
+        if key == "max_abs":
+            total[key] = max(total[key], v)
+        elif isinstance(v, int):
+            total[key] = total.get(key, 0) + v
+    return total
+
+
+def record(test: str, config: str, mode: str, rep) -> None:
+    """Appends one parity count record (JSON line) to the file named by
+    RECSA_PARITY_REPORT, if set: near ties and free-running mismatches are
+    counted and kept, not only printed."""
+    path = os.environ.get("RECSA_PARITY_REPORT")
+    line = {"test": test, "config": config, "mode": mode,
+            **{k: v for k, v in rep.items() if k != "first_mismatch"}}
+    print(json.dumps(line))
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(line) + "\n")

@@ -35,13 +35,20 @@ def check_chunk(layer, w, K, V, Q, s, C, gout, gsel, tokens, rep):
                 qu = synth.as_f32(np.ascontiguousarray(Q[b][s + t, h * G:(h + 1) * G]))
                 ref = oracle.query(tK, tV, K[b, h], V[b, h], s, qu, w.head_dim, w.branching, w.k, G, w.rope_base,
                                    Kloc=K[b, h, s:s + t + 1], Vloc=V[b, h, s:s + t + 1])
-                if len(ref["margin"]) and ref["margin"].min() < parity.NEAR_TIE:
-                    rep["near_ties"] += 1
-                    continue
-                for j in range(1, ref["J"] + 1):
+                rep["queries"] += 1
+                tie = parity.first_tie_level(ref)
+                rep["near_ties"] += 1 if tie else 0
+                differs = False
+                for j in range(ref["J"], 0, -1):
                     got = [x for x in gsel[b, t, h, j - 1].tolist() if x >= 0]
                     want = [x for x in ref["sel"][j - 1].tolist() if x >= 0]
-                    assert got == want, (s, t, b, h, j, got, want)
+                    if got != want:
+                        assert j <= tie, (s, t, b, h, j, got, want)  # exact above the first near tie
+                        differs = True
+                        break
+                if differs:
+                    rep["near_tie_sel_diff"] += 1
+                    continue
                 assert (gsel[b, t, h, ref["J"]:] == -1).all()
                 err = np.abs(gout[b, t, h * G:(h + 1) * G] - ref["out"]).max()
                 rep["max_abs"] = max(rep["max_abs"], float(err))
@@ -81,6 +88,7 @@ def test_prefill_small_multichunk():
     """Several chunks (the last one ragged) over a tree that grows by appends."""
     w = small(batch=2, n_kv_heads=2, group=4, head_dim=128, branching=8, k=3)
     _, _, _, _, _, rep = run_prefill(w, 700, 128, lambda ci, C: sorted(set(range(0, C, 9)) | {C - 1}))
+    parity.record("test_prefill_small_multichunk", "bf16 700 tokens, chunks of 128, b=8 k=3", "staged", rep)
     assert rep["checked"] > 300, rep
 
 
@@ -88,6 +96,7 @@ def test_prefill_small_multichunk():
 def test_prefill_shapes(D, G):
     w = small(batch=1, n_kv_heads=2, group=G, head_dim=D, branching=4, k=2)
     _, _, _, _, _, rep = run_prefill(w, 300, 64, lambda ci, C: list(range(0, C, 5)) + [C - 1])
+    parity.record("test_prefill_shapes", f"bf16 d={D} G={G} 300 tokens, chunks of 64, b=4 k=2", "staged", rep)
     assert rep["checked"] > 100, rep
 
 
@@ -115,5 +124,5 @@ def test_prefill_131k_sampled():
     w = synth.WORKLOADS["prefill_131k"]
     _, _, _, _, _, rep = run_prefill(w, w.length, w.chunk, lambda ci, C: [0, 1, 517, 2048, C - 1],
                                      max_chunks_checked={0, 1, 31})
-    print("prefill_131k", rep)
+    parity.record("test_prefill_131k_sampled", w.name, "staged", rep)
     assert rep["checked"] >= 40, rep

@@ -59,3 +59,19 @@ def test_null_buffers_rejected():
     assert R.lib().recsa_build_tree(None, None, None) == R.ERR_INVALID_ARG
     assert R.lib().recsa_decode(None, None, None, None, None, None) == R.ERR_INVALID_ARG
     assert R.lib().recsa_dense_decode_scratch_bytes(4, 32, 128) == 4 * 32 * 256 * 130 * 4
+
+
+def test_query_stats_rejects_null_context():
+    assert R.lib().recsa_query_stats(None, None, None, None, None) == R.ERR_INVALID_ARG
+
+
+def test_decode_shared_memory_limit_checked_at_init():
+    """k * b candidates whose decode tiles cannot fit the 227 KB of shared
+    memory a CTA may use are refused when the context is created, before any
+    device call (the buffers below are never touched)."""
+    cfg = R.make_config(1, 8, 32, 128, 64, 64, 1 << 20)  # 4096 candidates per level
+    h = ctypes.c_void_p()
+    fake = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced
+    st = R.lib().recsa_init(ctypes.byref(h), ctypes.byref(cfg), fake, fake, fake, 0, fake, None)
+    assert st == R.ERR_UNSUPPORTED and not h.value
+    assert b"shared memory" in R.lib().recsa_last_error()
