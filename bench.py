@@ -311,9 +311,9 @@ def measure_prefill(wname, dev, flush, peaks, last_chunks=0, with_dense=True):
     # one warm-up chunk on a throw-away layer of the same shape
     warm = RecsaLayer(B, H, Hq, D, w.branching, w.k, 2 * C, torch.from_numpy(Wp).view(bf).to(dev), dtype=bf,
                       rope_base=w.rope_base, max_chunk=C, device=dev)
-    for s0 in (0, C):
+    for s0 in (0, C):  # the first chunk's queries, the tree growing over the sequence's first tokens
         sl = slice(s0, s0 + C)
-        warm.prefill(qd[:, sl].contiguous(), kd[:, sl].contiguous(), vd[:, sl].contiguous(), out)
+        warm.prefill(qd[:, :C].contiguous(), kd[:, sl].contiguous(), vd[:, sl].contiguous(), out)
         warm.append(kd[:, sl].contiguous(), vd[:, sl].contiguous())
     torch.cuda.synchronize(dev)
     warm.close()

@@ -28,13 +28,14 @@ cudaError_t launch_dense(const void*, const void*, const void*, void*, int, long
                          cudaStream_t);
 int dense_splits(long long units, long long L);
 template <int D>
-cudaError_t launch_prefill_local(const TreeParams&, const void*, const void*, const void*, float*, int, int, int, int,
-                                 cudaStream_t);
-template <typename T, int D, int G>
-cudaError_t launch_prefill_tree(const TreeParams&, const void*, void*, const float*, int*, long long*, int, int, int,
-                                cudaStream_t);
+cudaError_t launch_prefill_attn(const TreeParams&, const void*, const void*, const void*, float*, void*, void*, int,
+                                int, int, int, cudaStream_t);
+template <int D, int G>
+cudaError_t launch_prefill_tree_tc(const TreeParams&, const void*, void*, const float*, int*, long long*, int, int,
+                                   const long long*, void*, cudaStream_t);
+size_t prefill_tree_scratch_bytes(const TreeParams& p, int C, int Hq);
+bool prefill_tree_supported(int D, int b);
 size_t decode_smem_bytes(int D, int G, int elem, int k, int b, int J_cap, bool fused);
-size_t prefill_tree_smem_bytes(int D, int G, int elem, int k, int b);
 size_t dense_static_scratch_bytes();
 cudaError_t dense_static_scratch(float** out);
 }  // namespace recsa
@@ -360,9 +361,37 @@ recsa_status recsa_append_decode(recsa_ctx* ctx, const void* k_new, const void* 
     return RECSA_OK;
 }
 
+namespace {
+// Prefill scratch: [local softmax state: B C Hq (d + 2) fp32][rotated queries:
+// B C Hq d bf16][rotated keys: B C H d bf16][the tree part's arrays], each
+// 256-byte aligned.
+struct PrefillScratch {
+    size_t state, qr, kr, tree, total;
+};
+PrefillScratch prefill_scratch(const recsa_config* c, int C) {
+    PrefillScratch s{};
+    const size_t rows_q = (size_t)c->batch * C * c->n_q_heads, rows_k = (size_t)c->batch * C * c->n_kv_heads;
+    s.state = 0;
+    s.qr = align256(rows_q * (c->head_dim + 2) * sizeof(float));
+    s.kr = s.qr + align256(rows_q * c->head_dim * 2);
+    s.tree = s.kr + align256(rows_k * c->head_dim * 2);
+    const Layout l = layout_for(c);
+    TreeParams tp{};
+    tp.B = c->batch;
+    tp.H = c->n_kv_heads;
+    tp.D = c->head_dim;
+    tp.b = c->branching;
+    tp.k = c->k;
+    tp.J_cap = l.J_cap;
+    for (int j = 0; j <= l.J_cap; j++) tp.rows[j] = l.rows[j];
+    s.total = s.tree + align256(prefill_tree_scratch_bytes(tp, C, c->n_q_heads));
+    return s;
+}
+}  // namespace
+
 size_t recsa_prefill_scratch_bytes(const recsa_config* cfg, int C) {
     if (check_config(cfg) != RECSA_OK || C < 1) return 0;
-    return (size_t)cfg->batch * C * cfg->n_q_heads * (cfg->head_dim + 2) * sizeof(float);
+    return prefill_scratch(cfg, C).total;
 }
 
 recsa_status recsa_prefill(recsa_ctx* ctx, const void* q, const void* k, const void* v, int C, void* out,
@@ -381,25 +410,30 @@ recsa_status recsa_prefill(recsa_ctx* ctx, const void* q, const void* k, const v
     if (!aligned(scratch, 256)) return fail(RECSA_ERR_INVALID_ARG, "scratch not 256-byte aligned");
     const size_t need = recsa_prefill_scratch_bytes(&c, C);
     if (scratch_bytes < need) return fail(RECSA_ERR_CAPACITY, "scratch has %zu bytes, needs %zu", scratch_bytes, need);
-    if (prefill_tree_smem_bytes(c.head_dim, ctx->G, 2, c.k, c.branching) > 227 * 1024)
-        return fail(RECSA_ERR_UNSUPPORTED, "k * branching too large for the prefill kernel's shared memory");
+    if (!prefill_tree_supported(c.head_dim, c.branching))
+        return fail(RECSA_ERR_UNSUPPORTED, "prefill needs branching rounded up to 32 <= min(head_dim, 128)");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    float* state = static_cast<float*>(scratch);
+    const PrefillScratch ps = prefill_scratch(&c, C);
+    char* sc = static_cast<char*>(scratch);
+    float* state = reinterpret_cast<float*>(sc + ps.state);
     cudaError_t e;
     if (c.head_dim == 64)
-        e = launch_prefill_local<64>(ctx->p, q, k, v, state, c.batch, C, c.n_q_heads, c.n_kv_heads, s);
+        e = launch_prefill_attn<64>(ctx->p, q, k, v, state, sc + ps.qr, sc + ps.kr, c.batch, C, c.n_q_heads,
+                                    c.n_kv_heads, s);
     else
-        e = launch_prefill_local<128>(ctx->p, q, k, v, state, c.batch, C, c.n_q_heads, c.n_kv_heads, s);
+        e = launch_prefill_attn<128>(ctx->p, q, k, v, state, sc + ps.qr, sc + ps.kr, c.batch, C, c.n_q_heads,
+                                     c.n_kv_heads, s);
     if (e == cudaSuccess) {
-        using T = __nv_bfloat16;
+        void* tree = sc + ps.tree;
+        const long long* lens = ctx->len.data();
         if (c.head_dim == 64) {
             constexpr int DD = 64;
-            DISPATCH_G(ctx->G, e = launch_prefill_tree<T, DD, GG>(ctx->p, q, out, state, sel_out, rows_out, c.batch, C,
-                                                                  c.n_q_heads, s));
+            DISPATCH_G(ctx->G, e = launch_prefill_tree_tc<DD, GG>(ctx->p, q, out, state, sel_out, rows_out, C,
+                                                                  c.n_q_heads, lens, tree, s));
         } else {
             constexpr int DD = 128;
-            DISPATCH_G(ctx->G, e = launch_prefill_tree<T, DD, GG>(ctx->p, q, out, state, sel_out, rows_out, c.batch, C,
-                                                                  c.n_q_heads, s));
+            DISPATCH_G(ctx->G, e = launch_prefill_tree_tc<DD, GG>(ctx->p, q, out, state, sel_out, rows_out, C,
+                                                                  c.n_q_heads, lens, tree, s));
         }
     }
     if (e != cudaSuccess) return cuda_fail(e, "recsa_prefill");
