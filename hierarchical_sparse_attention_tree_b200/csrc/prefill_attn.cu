@@ -13,18 +13,22 @@
 //
 // Two launches. (1) rope_chunk_kernel rotates the chunk's queries and keys by
 // their offset in the chunk (fp32, the host fp64 table) and rounds them to
-// bf16 into scratch. (2) prefill_attn_kernel: one CTA of 128 threads per
-// (128-query tile, query head); thread t owns query row t. Per 128-key tile:
-// one thread issues S = Q K^T (tcgen05.mma kind::f16, M = N = 128, fp32 in
-// TMEM columns [0, 128)); every thread reads its row of S from TMEM, applies
-// the scale and the causal mask, and writes its probabilities as bf16 into a
-// 128-byte-swizzled shared tile; then O += P V (M = 128, N = d, V read as an
-// MN-major operand) accumulates in TMEM columns [128, 128 + d). K and V tiles
-// are double-buffered; the next tile's loads are issued as soon as its buffer
-// is free, and the next S product right after this tile's P V product. The
-// softmax keeps a reference maximum that moves only when a row's maximum
-// exceeds it by more than 8 (natural-log units); then the row of O in TMEM is
-// rescaled. Exact either way: numerator and denominator share the reference.
+// bf16 into scratch. (2) prefill_attn_kernel: one CTA of 256 threads per
+// (128-query tile, query head); threads t and t + 128 share query row t, each
+// owning half of the key columns of S and half of the output columns. Per
+// 128-key tile: one thread issues S = Q K^T (tcgen05.mma kind::f16,
+// M = N = 128, fp32 in TMEM columns [0, 128)); every thread reads its half
+// row of S from TMEM, scales it (log2 units) and masks it on the diagonal
+// tile, the two halves exchange their maxima, and each writes its
+// probabilities as bf16 into a 128-byte-swizzled shared tile; then O += P V
+// (M = 128, N = d, V read as an MN-major operand) accumulates in TMEM
+// columns [128, 128 + d). K and V tiles are double-buffered; each tile's key
+// load is issued as soon as its buffer's S product has completed, its value
+// load once the P V product that used the buffer has, and the next S product
+// right after this tile's P V product. The softmax keeps a reference maximum
+// that moves only when a row's maximum exceeds it by more than 2^8; then the
+// row of O in TMEM is rescaled. Exact either way: numerator and denominator
+// share the reference.
 #include "tc.cuh"
 
 #include <cudaTypedefs.h>
@@ -35,8 +39,8 @@
 namespace recsa {
 
 constexpr int PA_T = 128;        // queries per CTA = keys per tile
-constexpr int PA_THREADS = 128;  // one query row per thread
-constexpr float PA_RESCALE = 8.f;
+constexpr int PA_THREADS = 256;  // two threads per query row (halves of the key and output columns)
+constexpr float PA_RESCALE = 8.f;  // log2 units: the reference moves when a row's maximum exceeds it by 2^8
 
 struct PrefillAttnArgs {
     float* state;  // [B][C][Hq][D + 2]: unnormalised acc, reference max, sum
@@ -77,7 +81,8 @@ struct PaLayout {
     static constexpr uint32_t TILE = PA_T * 128;           // one 64-wide tile of 128 rows
     static constexpr uint32_t QB = DT * TILE, KB = DT * TILE, PB = 2 * TILE;
     static constexpr uint32_t OFF_K = QB, OFF_V = OFF_K + 2 * KB, OFF_P = OFF_V + 2 * KB, OFF_BAR = OFF_P + PB;
-    static constexpr uint32_t BYTES = OFF_BAR + 128 + 1024;  // barriers, TMEM address, alignment slack
+    static constexpr uint32_t BYTES = OFF_BAR + 128 + 4 * PA_T * 4 + 1024;  // barriers, TMEM address, row
+                                                                              // maxima and sums, alignment slack
 };
 
 template <int D>
@@ -86,6 +91,7 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
                         const __grid_constant__ CUtensorMap mv, PrefillAttnArgs a) {
     using LY = PaLayout<D>;
     constexpr int DT = LY::DT;
+    constexpr int HK = PA_T / 2, HDC = D / 2;  // this thread's keys of a tile / output columns
     extern __shared__ unsigned char smem_pa[];
     const uint32_t raw = smem_addr(smem_pa);
     unsigned char* sm = smem_pa + (((raw + 1023u) & ~1023u) - raw);  // 1024-byte aligned tiles
@@ -94,13 +100,16 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
     auto sV = [&](int bf) { return sm + LY::OFF_V + bf * LY::KB; };  // and value tiles
     unsigned char* sP = sm + LY::OFF_P;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + LY::OFF_BAR);  // 0 q, 1-2 k, 3-4 v, 5 s, 6 o, 7 drain
-    uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 8);  // TMEM base address
+    uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 8);          // TMEM base address
+    float* xmax = reinterpret_cast<float*>(tbase + 4);               // [2][128] row maxima of the two halves
+    float* xsum = xmax + 2 * PA_T;                                   // [2][128] row sums
 
     const int tid = threadIdx.x, warp = tid >> 5;
+    const int rr = tid & (PA_T - 1), half = tid >> 7;  // query row, half of the columns
     const int qt = a.n_tiles - 1 - (int)blockIdx.x;  // longest rows first
     const int hq = blockIdx.y % a.Hq, bseq = blockIdx.y / a.Hq, h = hq / a.G;
     const int nkt = qt + 1;
-    const int row = qt * PA_T + tid;  // this thread's query, offset in the chunk
+    const int row = qt * PA_T + rr;  // this thread's query, offset in the chunk
 
     if (tid == 0) {
         for (int i = 0; i < 8; i++) mbar_init(&bar[i], 1);
@@ -117,9 +126,11 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tbase;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_off, tO = tmem + lane_off + PA_T;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;  // warps w and w + 4 share TMEM lanes
+    const uint32_t tS = tmem + lane_off + half * HK, tO = tmem + lane_off + PA_T + half * HDC;
     constexpr uint32_t ID_S = idesc_bf16(PA_T, PA_T, 0, 0), ID_O = idesc_bf16(PA_T, D, 0, 1);
+    constexpr float LOG2E = 1.4426950408889634f;
+    const float sc2 = a.scale * LOG2E;  // logits in log2 units
 
     // thread 0's bookkeeping of loads issued / waited per K and V buffer
     uint32_t k_iss0 = 0, k_iss1 = 0, k_wt0 = 0, k_wt1 = 0, v_iss0 = 0, v_iss1 = 0, v_wt0 = 0, v_wt1 = 0;
@@ -127,11 +138,14 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
         mbar_arrive_expect_tx(b, DT * LY::TILE);
         for (int x = 0; x < DT; x++) tma_load_4d(dst + x * LY::TILE, m, x * 64, head, row0, bseq, b);
     };
-    auto load_kv = [&](int kt) {
+    auto load_k = [&](int kt) {
         const int bf = kt & 1;
         load_tile(&mk, sK(bf), h, kt * PA_T, &bar[1 + bf]);
-        load_tile(&mv, sV(bf), h, kt * PA_T, &bar[3 + bf]);
         (bf ? k_iss1 : k_iss0)++;
+    };
+    auto load_v = [&](int kt) {
+        const int bf = kt & 1;
+        load_tile(&mv, sV(bf), h, kt * PA_T, &bar[3 + bf]);
         (bf ? v_iss1 : v_iss0)++;
     };
     bool timeout = false;
@@ -159,8 +173,12 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
     if (tid == 0) {
         mbar_arrive_expect_tx(&bar[0], DT * LY::TILE);
         for (int x = 0; x < DT; x++) tma_load_4d(sQ + x * LY::TILE, &mq, x * 64, hq, qt * PA_T, bseq, &bar[0]);
-        load_kv(0);
-        if (nkt > 1) load_kv(1);
+        load_k(0);
+        load_v(0);
+        if (nkt > 1) {
+            load_k(1);
+            load_v(1);
+        }
         wait1(&bar[0], q_wt);
         wait1(&bar[1], k_wt0);
         tc_fence_after();
@@ -168,7 +186,7 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
         mma_commit(&bar[5]);
     }
 
-    float m_ref = -INFINITY, l = 0.f;
+    float m_ref = -INFINITY, l = 0.f;  // log2 units
     bool ok = true;
     for (int kt = 0; kt < nkt; kt++) {
         const int bf = kt & 1;
@@ -179,36 +197,46 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
             break;
         }
         tc_fence_after();
-        float s[PA_T];
+        // S(kt) has completed: the key buffer of tile kt + 1 (it held tile
+        // kt - 1) is free
+        if (tid == 0 && kt >= 1 && kt + 1 < nkt) load_k(kt + 1);
+        float s[HK];
 #pragma unroll
-        for (int c = 0; c < PA_T / 32; c++) tmem_ld32(tS + c * 32, s + c * 32);
+        for (int c = 0; c < HK / 32; c++) tmem_ld32(tS + c * 32, s + c * 32);
         tmem_wait_ld();
         float mx = -INFINITY;
-        const int key0 = kt * PA_T;
+        if (kt == qt) {  // the diagonal tile: causal mask (and the chunk's end)
+            const int key0 = kt * PA_T + half * HK;
 #pragma unroll
-        for (int j = 0; j < PA_T; j++) {
-            const int key = key0 + j;
-            const float x = (key > row || key >= a.C) ? -INFINITY : s[j] * a.scale;
-            s[j] = x;
-            mx = fmaxf(mx, x);
-        }
-        // the previous tile's P V product is done: P and O are free, and so
-        // are the K / V buffers of tile kt - 1, which take tile kt + 1
-        if (kt > 0) {
-            bad = !mbar_wait(&bar[6], (uint32_t)(kt - 1) & 1u);
-            if (__syncthreads_or(bad)) {
-                ok = false;
-                break;
+            for (int j = 0; j < HK; j++) {
+                const int key = key0 + j;
+                s[j] = (key > row || key >= a.C) ? -INFINITY : s[j] * sc2;
+                mx = fmaxf(mx, s[j]);
             }
-            tc_fence_after();
-            if (tid == 0 && kt + 1 < nkt) load_kv(kt + 1);
+        } else {
+#pragma unroll
+            for (int j = 0; j < HK; j++) {
+                s[j] *= sc2;
+                mx = fmaxf(mx, s[j]);
+            }
         }
-        float m_new = (mx > m_ref + PA_RESCALE) ? mx : m_ref;
+        xmax[half * PA_T + rr] = mx;
+        // the previous tile's P V product is done: P and O are free, and so
+        // is the value buffer of tile kt - 1, which takes tile kt + 1
+        if (kt > 0) bad = !mbar_wait(&bar[6], (uint32_t)(kt - 1) & 1u);
+        if (__syncthreads_or(bad)) {  // also publishes xmax
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        if (tid == 0 && kt >= 1 && kt + 1 < nkt) load_v(kt + 1);
+        mx = fmaxf(xmax[rr], xmax[PA_T + rr]);
+        const float m_new = (mx > m_ref + PA_RESCALE) ? mx : m_ref;
         const bool move = kt > 0 && m_new != m_ref;
-        const float alpha = move ? expf(m_ref - m_new) : 1.f;
+        const float alpha = move ? exp2f(m_ref - m_new) : 1.f;
         if (__any_sync(0xffffffffu, move)) {  // TMEM accesses are warp-wide
 #pragma unroll 1
-            for (int c = 0; c < D / 32; c++) {
+            for (int c = 0; c < HDC / 32; c++) {
                 float o[32];
                 tmem_ld32(tO + c * 32, o);
                 tmem_wait_ld();
@@ -222,11 +250,11 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
         m_ref = m_new;
         float ls = 0.f;
 #pragma unroll
-        for (int j = 0; j < PA_T; j += 8) {
+        for (int j = 0; j < HK; j += 8) {
             float p[8];
 #pragma unroll
             for (int i = 0; i < 8; i++) {
-                p[i] = s[j + i] == -INFINITY ? 0.f : expf(s[j + i] - m_ref);
+                p[i] = exp2f(s[j + i] - m_ref);  // 0 for masked keys
                 ls += p[i];
             }
             uint4 pk;
@@ -236,7 +264,7 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
             pk.y = *reinterpret_cast<uint32_t*>(&h1);
             pk.z = *reinterpret_cast<uint32_t*>(&h2);
             pk.w = *reinterpret_cast<uint32_t*>(&h3);
-            *reinterpret_cast<uint4*>(sP + sw128_offset(tid, j, PA_T)) = pk;
+            *reinterpret_cast<uint4*>(sP + sw128_offset(rr, half * HK + j, PA_T)) = pk;
         }
         l += ls;
         fence_proxy_async_shared();  // P (generic writes) before the tensor core reads it
@@ -259,20 +287,23 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
         ok = !__syncthreads_or(bad);
     }
     if (ok) {  // every thread loads (TMEM loads are warp-wide); rows past the chunk store nothing
+        xsum[half * PA_T + rr] = l;
         tc_fence_after();
         float* st = a.state + (((size_t)bseq * a.C + row) * a.Hq + hq) * (D + 2);
 #pragma unroll 1
-        for (int c = 0; c < D / 32; c++) {
+        for (int c = 0; c < HDC / 32; c++) {
             float o[32];
             tmem_ld32(tO + c * 32, o);
             tmem_wait_ld();
             if (row < a.C)  // state rows are d + 2 floats: 8-byte aligned
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) *reinterpret_cast<float2*>(st + c * 32 + i) = make_float2(o[i], o[i + 1]);
+                for (int i = 0; i < 32; i += 2)
+                    *reinterpret_cast<float2*>(st + half * HDC + c * 32 + i) = make_float2(o[i], o[i + 1]);
         }
-        if (row < a.C) {
-            st[D] = m_ref;
-            st[D + 1] = l;
+        __syncthreads();
+        if (row < a.C && half == 0) {  // natural-log units for the merge
+            st[D] = m_ref / LOG2E;
+            st[D + 1] = xsum[rr] + xsum[PA_T + rr];
         }
     }
     if (!ok && tid == 0) {

@@ -271,43 +271,63 @@ __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
     lo = pack8(l);
 }
 
+// bf16 pair (packed in 32 bits) <-> two floats.
+__device__ __forceinline__ float2 bf2_f2(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t f2_bf2(float2 x) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(x.x, x.y);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
 // One 8-frequency chunk: rotates (xa, xb) = dims [f, f + 8) and [HD + f,
-// HD + f + 8) by the table's (cos, sin) and stores both halves split into
-// hi / lo at `row` of two K-major swizzled operands of `rows` rows.
-template <int D>
+// HD + f + 8) by the table's (cos, sin), in packed fp32 (the same arithmetic
+// as the decode path's scoring), and stores both halves at `row` of two
+// K-major swizzled operands of `rows` rows: hi = bf16(x) and, if LO,
+// lo = bf16(x - hi). cs: cos [2], sin [2], -sin [2] as float4.
+template <int D, bool LO>
 __device__ __forceinline__ void put_chunk(uint4 xa_raw, uint4 xb_raw, const float4* cs, int f,
                                           unsigned char* hi_base, unsigned char* lo_base, int row, int rows) {
     constexpr int HD = D / 2;
-    float xa[8], xb[8], ra[8], rb[8];
-    const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&xa_raw);
-    const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&xb_raw);
+    const uint32_t xa[4] = {xa_raw.x, xa_raw.y, xa_raw.z, xa_raw.w};
+    const uint32_t xb[4] = {xb_raw.x, xb_raw.y, xb_raw.z, xb_raw.w};
+    const float2 c2[4] = {make_float2(cs[0].x, cs[0].y), make_float2(cs[0].z, cs[0].w), make_float2(cs[1].x, cs[1].y),
+                          make_float2(cs[1].z, cs[1].w)};
+    const float2 s2[4] = {make_float2(cs[2].x, cs[2].y), make_float2(cs[2].z, cs[2].w), make_float2(cs[3].x, cs[3].y),
+                          make_float2(cs[3].z, cs[3].w)};
+    const float2 n2[4] = {make_float2(cs[4].x, cs[4].y), make_float2(cs[4].z, cs[4].w), make_float2(cs[5].x, cs[5].y),
+                          make_float2(cs[5].z, cs[5].w)};
+    uint32_t ha[4], la[4], hb[4], lb[4];
+    const float2 m1 = make_float2(-1.f, -1.f);
 #pragma unroll
     for (int i = 0; i < 4; i++) {
-        xa[2 * i] = __low2float(ha[i]);
-        xa[2 * i + 1] = __high2float(ha[i]);
-        xb[2 * i] = __low2float(hb[i]);
-        xb[2 * i + 1] = __high2float(hb[i]);
+        const float2 a = bf2_f2(xa[i]), b = bf2_f2(xb[i]);
+        const float2 ra = ffma2(a, c2[i], fmul2(b, n2[i]));
+        const float2 rb = ffma2(b, c2[i], fmul2(a, s2[i]));
+        ha[i] = f2_bf2(ra);
+        hb[i] = f2_bf2(rb);
+        if (LO) {
+            la[i] = f2_bf2(ffma2(bf2_f2(ha[i]), m1, ra));
+            lb[i] = f2_bf2(ffma2(bf2_f2(hb[i]), m1, rb));
+        }
     }
-    const float cc[8] = {cs[0].x, cs[0].y, cs[0].z, cs[0].w, cs[1].x, cs[1].y, cs[1].z, cs[1].w};
-    const float ss[8] = {cs[2].x, cs[2].y, cs[2].z, cs[2].w, cs[3].x, cs[3].y, cs[3].z, cs[3].w};
-#pragma unroll
-    for (int i = 0; i < 8; i++) rot_pair(xa[i], xb[i], cc[i], ss[i], ra[i], rb[i]);
-    uint4 h, l;
-    split8(ra, h, l);
-    *reinterpret_cast<uint4*>(hi_base + sw128_offset(row, f, rows)) = h;
-    *reinterpret_cast<uint4*>(lo_base + sw128_offset(row, f, rows)) = l;
-    split8(rb, h, l);
-    *reinterpret_cast<uint4*>(hi_base + sw128_offset(row, HD + f, rows)) = h;
-    *reinterpret_cast<uint4*>(lo_base + sw128_offset(row, HD + f, rows)) = l;
+    const uint32_t oa = sw128_offset(row, f, rows), ob = sw128_offset(row, HD + f, rows);
+    *reinterpret_cast<uint4*>(hi_base + oa) = make_uint4(ha[0], ha[1], ha[2], ha[3]);
+    *reinterpret_cast<uint4*>(hi_base + ob) = make_uint4(hb[0], hb[1], hb[2], hb[3]);
+    if (LO) {
+        *reinterpret_cast<uint4*>(lo_base + oa) = make_uint4(la[0], la[1], la[2], la[3]);
+        *reinterpret_cast<uint4*>(lo_base + ob) = make_uint4(lb[0], lb[1], lb[2], lb[3]);
+    }
 }
-// The table's (cos, sin) of frequencies [f, f + 8) of row `tab`.
+// The table's cos, sin and -sin of frequencies [f, f + 8) of row `tab`.
 template <int D>
 __device__ __forceinline__ void load_cs(const float* tab, int f, float4* cs) {
     constexpr int HD = D / 2;
-    cs[0] = __ldg(reinterpret_cast<const float4*>(tab + f));
-    cs[1] = __ldg(reinterpret_cast<const float4*>(tab + f + 4));
-    cs[2] = __ldg(reinterpret_cast<const float4*>(tab + HD + f));
-    cs[3] = __ldg(reinterpret_cast<const float4*>(tab + HD + f + 4));
+#pragma unroll
+    for (int x = 0; x < 3; x++) {
+        cs[2 * x] = __ldg(reinterpret_cast<const float4*>(tab + x * HD + f));
+        cs[2 * x + 1] = __ldg(reinterpret_cast<const float4*>(tab + x * HD + f + 4));
+    }
 }
 
 __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
@@ -427,30 +447,29 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
             if (MODE == MODE_VALUE && tid * 64 < b * D) prefetch_l2(vb + nrow * D + tid * 64);
         }
         // ---- operands: the rotated query and keys, split hi / lo
+        // (the largest-logit pass of the tokens needs only an approximate
+        // reference maximum: hi parts and one product)
+        constexpr bool LO = MODE != MODE_MAX;
         {
             const float* tab = p.rope + (size_t)(qok ? P : 0) * 3 * HD;
-            float4 cs[4], cn[4];
+            float4 cs[6], cn[6];
             load_cs<D>(tab, 0, cs);
+            const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int c = 0; c < NCH; c++) {
                 if (c + 1 < NCH) load_cs<D>(tab, (c + 1) * 8, cn);
-                if (qok) {
-                    put_chunk<D>(qa[c], qb[c], cs, c * 8, sAh, sAl, tid, 128);
-                } else {
-                    const uint4 z = make_uint4(0, 0, 0, 0);
-                    put_chunk<D>(z, z, cs, c * 8, sAh, sAl, tid, 128);
-                }
+                put_chunk<D, LO>(qok ? qa[c] : z, qok ? qb[c] : z, cs, c * 8, sAh, sAl, tid, 128);
 #pragma unroll
-                for (int i = 0; i < 4; i++) cs[i] = cn[i];
+                for (int i = 0; i < 6; i++) cs[i] = cn[i];
             }
         }
 #pragma unroll
         for (int x = 0; x < BU; x++) {
             const int unit = tid + x * TP_THREADS, o = unit / NCH, c = unit % NCH;
-            float4 cs[4];
+            float4 cs[6];
             load_cs<D>(p.rope + (size_t)o * 3 * HD, c * 8, cs);
             const uint4 z = make_uint4(0, 0, 0, 0);
-            put_chunk<D>(o < nchild ? ka[x] : z, o < nchild ? kbv[x] : z, cs, c * 8, sBh, sBl, o, NB);
+            put_chunk<D, LO>(o < nchild ? ka[x] : z, o < nchild ? kbv[x] : z, cs, c * 8, sBh, sBl, o, NB);
         }
         if (MODE == MODE_VALUE) cp_async_wait_all();
         fence_proxy_async_shared();
@@ -460,7 +479,7 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int pass = 0; pass < 3; pass++) {
+            for (int pass = 0; pass < (MODE == MODE_MAX ? 1 : 3); pass++) {
                 const uint32_t ab = smem_addr(pass == 2 ? sAl : sAh), bb = smem_addr(pass == 1 ? sBl : sBh);
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ks++) {
@@ -496,12 +515,22 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
         if (MODE == MODE_SCORE) {
             // S = sum over the G heads (G consecutive lanes), written by the
             // G lanes in turn
+            // (each lane then writes a contiguous 1/G of the row, 16 bytes at a time)
             float* srow = a.S + (u * a.C + t) * (long long)a.maxc + (long long)r * b;
 #pragma unroll
-            for (int o = 0; o < NB; o++) {
-                float sv = lg[o];
-                for (int m = 1; m < G; m <<= 1) sv += __shfl_xor_sync(0xffffffffu, sv, m);
-                if (valid && o < nchild && (o % G) == g) srow[o] = sv;
+            for (int o = 0; o < NB; o++)
+                for (int m = 1; m < G; m <<= 1) lg[o] += __shfl_xor_sync(0xffffffffu, lg[o], m);
+            const int per = NB / G;
+            if (valid) {
+#pragma unroll
+                for (int o0 = 0; o0 < NB; o0 += 4) {
+                    if (o0 >= g * per && o0 < (g + 1) * per) {
+                        if (o0 + 4 <= nchild)
+                            *reinterpret_cast<float4*>(srow + o0) = make_float4(lg[o0], lg[o0 + 1], lg[o0 + 2], lg[o0 + 3]);
+                        else
+                            for (int i = o0; i < nchild; i++) srow[i] = lg[i];
+                    }
+                }
             }
         }
         if (MODE == MODE_VALUE) {
@@ -520,6 +549,8 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
             }
             const unsigned mk = valid ? a.mkey[orow] : 0u;
             const float mref = mk ? key_float(mk) : 0.f;
+            constexpr float LOG2E = 1.4426950408889634f;
+            const float mref2 = mref * LOG2E;
             float lsum = 0.f;
 #pragma unroll
             for (int o0 = 0; o0 < NB; o0 += 8) {
@@ -528,7 +559,7 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
                 for (int i = 0; i < 8; i++) {
                     const int o = o0 + i;
                     const bool kept = (keep[o >> 6] >> (o & 63)) & 1ull;
-                    w[i] = (mk != 0u && o < nchild && !kept) ? expf(lg[o] - mref) : 0.f;
+                    w[i] = (mk != 0u && o < nchild && !kept) ? exp2f(fmaf(lg[o], LOG2E, -mref2)) : 0.f;
                     lsum += w[i];
                 }
                 uint4 hi, lo;
