@@ -191,13 +191,32 @@ size_t recsa_workspace_bytes(const recsa_config* cfg) {
     return layout_for(cfg).total;
 }
 
-recsa_status recsa_init(recsa_ctx** out, const recsa_config* cfg, void* k_cache, void* v_cache, void* workspace,
-                        size_t workspace_bytes, const void* pooler_w, recsa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+struct PageArgs {
+    const int* table;
+    int page_size, max_pages;
+    long long num_pages;
+};
+
+recsa_status init_ctx(recsa_ctx** out, const recsa_config* cfg, void* k_cache, void* v_cache, void* workspace,
+                      size_t workspace_bytes, const void* pooler_w, recsa_stream_t stream, const PageArgs* pg) {
     if (!out) return fail(RECSA_ERR_INVALID_ARG, "out is NULL");
     *out = nullptr;
     recsa_status st = check_config(cfg);
     if (st != RECSA_OK) return st;
     if (!k_cache || !v_cache || !workspace || !pooler_w) return fail(RECSA_ERR_INVALID_ARG, "NULL buffer");
+    if (pg) {
+        if (!pg->table) return fail(RECSA_ERR_INVALID_ARG, "NULL page table");
+        if (pg->page_size < cfg->branching || pg->page_size % cfg->branching)
+            return fail(RECSA_ERR_INVALID_ARG, "page_size %d must be a multiple of branching %d", pg->page_size,
+                        cfg->branching);
+        if (pg->max_pages < 1 || (long long)pg->max_pages * pg->page_size < cfg->capacity)
+            return fail(RECSA_ERR_INVALID_ARG, "max_pages * page_size must cover the capacity");
+        if (pg->num_pages < 1 || pg->num_pages >= (1LL << 31))
+            return fail(RECSA_ERR_INVALID_ARG, "num_pages out of range");
+    }
     if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return fail(RECSA_ERR_INVALID_ARG, "cache not 16-byte aligned");
     if (!aligned(workspace, 256)) return fail(RECSA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
     Layout l = layout_for(cfg);
@@ -223,6 +242,12 @@ recsa_status recsa_init(recsa_ctx** out, const recsa_config* cfg, void* k_cache,
     p.B = cfg->batch; p.H = cfg->n_kv_heads; p.G = c->G; p.D = D; p.b = cfg->branching; p.k = cfg->k;
     p.J_cap = l.J_cap; p.npos = l.npos; p.cap = cfg->capacity;
     p.K[0] = k_cache; p.V[0] = v_cache;
+    if (pg) {
+        p.pages = pg->table;
+        p.page_size = pg->page_size;
+        p.max_pages = pg->max_pages;
+        p.num_pages = pg->num_pages;
+    }
     for (int j = 0; j <= MAXJ; j++) p.span[j] = span_sat(cfg->branching, j);
     p.rows[0] = cfg->capacity;
     for (int j = 1; j <= l.J_cap; j++) {
@@ -269,6 +294,21 @@ recsa_status recsa_init(recsa_ctx** out, const recsa_config* cfg, void* k_cache,
     }
     *out = c;
     return RECSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+recsa_status recsa_init(recsa_ctx** out, const recsa_config* cfg, void* k_cache, void* v_cache, void* workspace,
+                        size_t workspace_bytes, const void* pooler_w, recsa_stream_t stream) {
+    return init_ctx(out, cfg, k_cache, v_cache, workspace, workspace_bytes, pooler_w, stream, nullptr);
+}
+
+recsa_status recsa_init_paged(recsa_ctx** out, const recsa_config* cfg, void* k_pool, void* v_pool,
+                              long long num_pages, int page_size, const int* page_table, int max_pages,
+                              void* workspace, size_t workspace_bytes, const void* pooler_w, recsa_stream_t stream) {
+    const PageArgs pg{page_table, page_size, max_pages, num_pages};
+    return init_ctx(out, cfg, k_pool, v_pool, workspace, workspace_bytes, pooler_w, stream, &pg);
 }
 
 void recsa_destroy(recsa_ctx* ctx) { delete ctx; }

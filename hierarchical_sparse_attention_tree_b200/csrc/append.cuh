@@ -55,6 +55,7 @@ __device__ __forceinline__ float pool_product_half(const T* Wt, const float* x, 
 struct AppendDims {
     long long cap;
     int J_cap, b;
+    const TokenMap* tok;  // where the token rows live (in shared memory)
 };
 
 // Shared memory it needs besides the pooler: km [D], part [2][D] and pre
@@ -83,8 +84,8 @@ __device__ __forceinline__ bool append_token(const AppendDims& p, const LevelRef
     float* part = scratch + D;
     float* pre = scratch + 3 * D;
     T kn = from_f<T>(0.f), vn = from_f<T>(0.f);
-    T* K0 = reinterpret_cast<T*>(lv[0].K) + u * p.cap * D;
-    T* V0 = reinterpret_cast<T*>(lv[0].V) + u * p.cap * D;
+    T* K0 = reinterpret_cast<T*>(lv[0].K);
+    T* V0 = reinterpret_cast<T*>(lv[0].V);
     // per level j: prefix sums of the right edge and, if a child of level
     // j-1 completed at this token, that child's stored key and value sum
     auto load_level = [&](int j, float& pk, float& pv, float& ko, float& vo) {
@@ -99,8 +100,9 @@ __device__ __forceinline__ bool append_token(const AppendDims& p, const LevelRef
         if (rm == 0) {
             const long long c = qm - 1;  // completed child of level j-1
             if (j == 1) {
-                ko = to_f(K0[c * D + t]);
-                vo = to_f(V0[c * D + t]);
+                const long long rc = token_row(*p.tok, u, c);
+                ko = to_f(K0[rc * D + t]);
+                vo = to_f(V0[rc * D + t]);
             } else {
                 const long long row = u * lv[j - 1].rows + c;
                 ko = to_f(reinterpret_cast<const T*>(lv[j - 1].K)[row * D + t]);
@@ -127,8 +129,9 @@ __device__ __forceinline__ bool append_token(const AppendDims& p, const LevelRef
             load_level(j, r4[0], r4[1], r4[2], r4[3]);
             for (int x = 0; x < 4; x++) pre[((size_t)(j - 1) * 4 + x) * D + t] = r4[x];
         }
-        K0[P * D + t] = kn;
-        V0[P * D + t] = vn;
+        const long long rp = token_row(*p.tok, u, P);
+        K0[rp * D + t] = kn;
+        V0[rp * D + t] = vn;
     }
     if (!wait_w()) return false;  // no node has been written
 

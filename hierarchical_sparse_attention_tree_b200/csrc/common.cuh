@@ -33,11 +33,40 @@ struct TreeParams {
     float* PV[MAXJ + 1];       // right-edge value prefix sums [B*H][D] (j >= 1)
     const void* Wt;            // pooler, transposed, storage type: Wt[c * D + r] = W[r][c]
     const float* rope;         // [npos][3][D/2]: cos, sin, -sin of (p * theta_i), theta_i = base^(-2i/d)
+    const int* pages;          // paged token cache: [B][max_pages] pool page of each page of tokens (null: contiguous)
+    int page_size, max_pages;  // tokens per page (a multiple of b), pages per sequence
+    long long num_pages;       // pages in the pool
     long long* len;            // [B*H] tokens held by each unit
     long long* stats;          // [B*H][3] last decode: depth, K rows read, V rows read
     int* err;                  // device error word
     float scale;               // 1 / sqrt(D)
 };
+
+// Where the token rows live. Contiguous: unit u's rows at base + (u * cap + t) * D.
+// Paged: a pool [pages][H][page_size][D]; token t of unit u = (sequence
+// u / H, KV head u % H) is row t % page_size of page pages[seq * max_pages +
+// t / page_size]. Rows t .. t + n - 1 are contiguous while they stay in one
+// page (a node's children always do: the page size is a multiple of b).
+struct TokenMap {
+    const int* pages;
+    int page_size, max_pages, H;
+    long long cap, num_pages;
+    int* err;
+};
+// A page id outside the pool is reported in the error word (shape bit) and
+// replaced by page 0, so that no access leaves the pool.
+__device__ __forceinline__ long long token_row(const TokenMap& m, long long u, long long t) {
+    if (!m.pages) return u * m.cap + t;
+    long long pg = m.pages[(u / m.H) * m.max_pages + t / m.page_size];
+    if (pg < 0 || pg >= m.num_pages) {
+        atomicOr(m.err, 2);
+        pg = 0;
+    }
+    return (pg * m.H + u % m.H) * m.page_size + t % m.page_size;
+}
+__device__ __forceinline__ TokenMap token_map(const TreeParams& p) {
+    return TokenMap{p.pages, p.page_size, p.max_pages, p.H, p.cap, p.num_pages, p.err};
+}
 
 // One level's addresses and sizes together. Kernels that index the levels
 // with a runtime j copy these into shared memory once: kernel parameters

@@ -51,8 +51,16 @@ struct DecodeArgs {
     int region0;          // bytes of the K/V tile region (reused for the warp merge)
 };
 
+// Where a paged cache keeps this unit's tokens (set up once per CTA).
+struct DecPages {
+    const int* row;  // the sequence's page table row
+    int psize, nheads, head, npages;
+};
+
 struct DecSmem {
     uint64_t bar[3];                     // [0]: key tile, [1]: value tile, [2]: pooler (append)
+    DecPages pg;                         // paged cache (row null: contiguous)
+    TokenMap tok;                        // where the token rows live (for the append)
     unsigned long long wl[DEC_WARPS][KMAX];  // per-warp top-k lists, sorted, zero padded
     unsigned long long picked[KMAX];     // global top-k keys, best first
     unsigned long long thresh;           // the k-th best key
@@ -156,7 +164,19 @@ __device__ __forceinline__ int rank_in_lists(const unsigned long long* lists, in
 // out of line: it runs a few times per launch, on one thread.
 template <typename T, int D>
 __device__ __noinline__ void issue_rows(T* dst, const T* base, const int* par, int n_j, int b, int r0, int r1,
-                                        uint64_t* bar, int* err) {
+                                        uint64_t* bar, int* err, const DecPages* pg) {
+    // pg set (level 0 of a paged cache): base is the pool and each piece
+    // (part of one parent's children, which lie in one page) is translated;
+    // else base is the unit's first row
+    auto src = [&](int id0) {
+        if (!pg) return base + (size_t)id0 * D;
+        int page = pg->row[id0 / pg->psize];
+        if (page < 0 || page >= pg->npages) {
+            flag_error(err, ERR_SHAPE);
+            page = 0;
+        }
+        return base + (((size_t)page * pg->nheads + pg->head) * pg->psize + id0 % pg->psize) * D;
+    };
     const int pr = r0 / b, o0 = r0 - pr * b;
     uint32_t total = 0;
     for (int r = r0, q = pr, o = o0; r < r1; q++, o = 0) {
@@ -165,14 +185,16 @@ __device__ __noinline__ void issue_rows(T* dst, const T* base, const int* par, i
         if (id0 >= 0 && id0 + n <= n_j) total += (uint32_t)(n * D * sizeof(T));
         r += n;
     }
-    fence_proxy_async_shared();
-    fence_proxy_async_global();  // global writes of a fused append seen by the bulk reads
+    if (r1 > r0) {  // (an empty request only completes the barrier's phase: nothing to order)
+        fence_proxy_async_shared();
+        fence_proxy_async_global();  // global writes of a fused append seen by the bulk reads
+    }
     mbar_arrive_expect_tx(bar, total);
     for (int r = r0, q = pr, o = o0; r < r1; q++, o = 0) {
         const int n = min(b - o, r1 - r);
         const int id0 = par[q] * b + o;
         if (id0 >= 0 && id0 + n <= n_j)
-            bulk_g2s(dst + (size_t)(r - r0) * D, base + (size_t)id0 * D, (uint32_t)(n * D * sizeof(T)), bar);
+            bulk_g2s(dst + (size_t)(r - r0) * D, src(id0), (uint32_t)(n * D * sizeof(T)), bar);
         else
             flag_error(err, ERR_SHAPE);
         r += n;
@@ -183,12 +205,14 @@ __device__ __noinline__ void issue_rows(T* dst, const T* base, const int* par, i
 // token of unit u at position P, leaves the refreshed node of level jf (the
 // first scored level; jf = 0: the token itself) in patch[0..D) (key) and
 // patch[D..2D) (value), and makes its global writes visible to later bulk
-// reads. Every thread of the block calls it. False if the pooler copy (on
-// wbar, into the start of smem) did not arrive.
+// reads (fence = false: the caller fences later, before this CTA's next
+// bulk read and before other CTAs may read the appended rows). Every thread
+// of the block calls it. False if the pooler copy (on wbar, into the start
+// of smem) did not arrive.
 template <typename T, int D>
 __device__ __noinline__ bool fused_append(AppendDims dims, const LevelRef* lv, long long u, long long P, const T* kn,
                                           const T* vn, unsigned char* smem, T* patch, int jf, uint64_t* wbar,
-                                          int* err) {
+                                          int* err, bool fence) {
     const int tid = threadIdx.x;
     const bool ok = append_token<T, D>(
         dims, lv, u, P, kn, vn, reinterpret_cast<const T*>(smem), reinterpret_cast<float*>(smem + D * D * sizeof(T)),
@@ -210,7 +234,7 @@ __device__ __noinline__ bool fused_append(AppendDims dims, const LevelRef* lv, l
         patch[tid] = kn[tid];
         patch[D + tid] = vn[tid];
     }
-    fence_proxy_async_global();  // this CTA's writes, before its later bulk reads
+    if (fence) fence_proxy_async_global();  // this CTA's writes, before its later bulk reads
     __syncthreads();
     return ok;
 }
@@ -250,6 +274,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
     const bool app = a.k_new != nullptr;
     const bool appender = app && rank == CS - 1;
     if (tid == 0) {
+        sm->pg = DecPages{p.pages ? p.pages + (u / p.H) * p.max_pages : nullptr, p.page_size, p.H, (int)(u % p.H),
+                          (int)p.num_pages};
+        sm->tok = token_map(p);
         mbar_init(&sm->bar[0], 1);
         mbar_init(&sm->bar[1], 1);
         mbar_init(&sm->bar[2], 1);
@@ -260,9 +287,33 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
         }
     }
     asm volatile("griddepcontrol.launch_dependents;");
+    {  // the RoPE table is constant: every CTA brings its share of it into L2
+       // now, so that no scoring step waits for it in DRAM
+        const long long lines = ((long long)p.npos * 3 * (D / 2) * 4 + 127) / 128;
+        const long long nct = (long long)gridDim.y * CS, ci = (long long)blockIdx.y * CS + rank;
+        const long long per = (lines + nct - 1) / nct;
+        const long long l0 = ci * per + tid;
+        if (tid < per && l0 < lines) asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(p.rope) + l0 * 128));
+    }
     load_levels(p, sm->lv, tid);  // visible after the set-up barrier below
     if (tid < 8) sm->M[tid] = -INFINITY;
     grid_dependency_wait();  // from here on, every earlier kernel's writes are visible
+    if (appender) {
+        // the append reads every level's right-edge prefix sums and the new
+        // token's rows; their addresses do not depend on the length, so they
+        // are brought into L1 now, together with the length and the query
+        constexpr int LPR = D * 4 / 128;  // 128-byte lines of one fp32 row
+        const int nl = 2 * p.J_cap * LPR;
+        if (tid < nl) {
+            const int jj = tid / (2 * LPR) + 1, x = tid % (2 * LPR);
+            const float* row = (x < LPR ? p.PK[jj] : p.PV[jj]) + u * D;
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const char*>(row) + (x % LPR) * 128));
+        } else if (tid < nl + 2 * (int)((D * sizeof(T) + 127) / 128)) {
+            const int x = tid - nl, per = (int)((D * sizeof(T) + 127) / 128);
+            const T* row = reinterpret_cast<const T*>(x < per ? a.k_new : a.v_new) + u * D;
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const char*>(row) + (x % per) * 128));
+        }
+    }
     const long long Lraw = p.len[u];  // both loads in flight together
     {
         const T* qg = reinterpret_cast<const T*>(a.q) + (u * G) * D;
@@ -304,10 +355,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
     // Thread 0: request rows [r0, r1) of level j's candidate list (children of
     // sm->par) into the key (which = 0) or value (which = 1) tile.
     auto issue = [&](int which, int j, int r0, int r1) {
-        issue_rows<T, D>(which == 0 ? Kt : Vt,
-                         reinterpret_cast<const T*>(which == 0 ? sm->lv[j].K : sm->lv[j].V) + (u * sm->lv[j].rows) * D,
-                         sm->par,
-                         sm->nlev[j], b, r0, r1, &sm->bar[which], p.err);
+        const bool paged = j == 0 && p.pages;
+        const T* lb = reinterpret_cast<const T*>(which == 0 ? sm->lv[j].K : sm->lv[j].V);
+        issue_rows<T, D>(which == 0 ? Kt : Vt, paged ? lb : lb + (u * sm->lv[j].rows) * D, sm->par, sm->nlev[j], b, r0,
+                         r1, &sm->bar[which], p.err, paged ? &sm->pg : nullptr);
     };
     auto wait_tile = [&](int which) {
         if (!mbar_wait(&sm->bar[which], phase[which])) {
@@ -389,7 +440,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
     // appends at once and needs no copy of that row. The first scored level
     // is the highest level with more than k nodes (every level above keeps
     // all of its candidates), else the tokens.
-    bool chained = false;
+    bool chained = false, fenced = false;
     if (appender && !bad_len) {
         int jt = 1;
         while (jt < p.J_cap && sm->nlev[jt] > b) jt++;
@@ -397,10 +448,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
         for (int x = jt; x >= 1 && jf == 0; x--)
             if (sm->nlev[x] > p.k) jf = x;
         if (sm->nlev[jf] - 1 <= (CS - 1) * MY) {
-            const bool ok = fused_append<T, D>(AppendDims{p.cap, p.J_cap, p.b}, sm->lv, u, Lraw,
+            const bool ok = fused_append<T, D>(AppendDims{p.cap, p.J_cap, p.b, &sm->tok}, sm->lv, u, Lraw,
                                                reinterpret_cast<const T*>(a.k_new) + u * D,
                                                reinterpret_cast<const T*>(a.v_new) + u * D, smem_raw, patch_rows(), jf,
-                                               &sm->bar[2], p.err);
+                                               &sm->bar[2], p.err, false);
             appended = ok;
             if (!ok) bad = true;
             chained = true;
@@ -475,10 +526,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
                 issue(1, j, r0, r1);
             }
             if (appender) {
-                const bool ok = fused_append<T, D>(AppendDims{p.cap, p.J_cap, p.b}, sm->lv, u, Lraw,
+                const bool ok = fused_append<T, D>(AppendDims{p.cap, p.J_cap, p.b, &sm->tok}, sm->lv, u, Lraw,
                                                    reinterpret_cast<const T*>(a.k_new) + u * D,
                                                    reinterpret_cast<const T*>(a.v_new) + u * D, smem_raw, patch_rows(),
-                                                   j, &sm->bar[2], p.err);
+                                                   j, &sm->bar[2], p.err, true);
                 appended = ok;
                 if (!ok) bad = true;
                 if (early)
@@ -547,6 +598,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
                     }
                     for (int t = nmy + tid; t < kk; t += DEC_THREADS)  // fewer rows than kk
                         for (int r = 0; r < CS; r++) cluster.map_shared_rank(gk, r)[rank * KMAX + t] = 0ull;
+                }
+                if (chained && !fenced) {  // the append's global writes, before anyone's bulk reads of them
+                    fence_proxy_async_global();
+                    fenced = true;
                 }
                 cluster.sync();
                 // global top-kk (the same in every CTA) and the kept ids in
@@ -634,28 +689,44 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
         cml[G + tid] = s;
     }
     __syncthreads();  // cacc and cml complete
-    {  // the gather area has a place of its own: no barrier needed before the push
-        float* dst = cluster.map_shared_rank(gat, 0) + rank * (G * D + 2 * G);
-        for (int idx = tid; idx < G * D + 2 * G; idx += DEC_THREADS) dst[idx] = idx < G * D ? cacc[idx] : cml[idx - G * D];
+    // Every CTA merges one slice of the output columns: each CTA sends slice r
+    // of its (unnormalised) output, with its maxima and sums, to CTA r (the
+    // gather area has a place of its own: no barrier is needed before it).
+    constexpr int SL = G * D / DEC_CLUSTER;  // output columns per CTA
+    constexpr int GST = SL + 2 * G;          // one source's record in the gather area
+    static_assert((G * D) % DEC_CLUSTER == 0, "output slices");
+    for (int x = tid; x < CS * GST; x += DEC_THREADS) {
+        const int r = x / GST, i = x - r * GST;
+        cluster.map_shared_rank(gat, r)[rank * GST + i] = i < SL ? cacc[r * SL + i] : cml[i - SL];
     }
-    cluster.sync();  // the gather area of rank 0 is complete
+    if (chained && !fenced) fence_proxy_async_global();
+    cluster.sync();  // every CTA's gather area is complete
     if (appended && tid == 0) p.len[u] = Lraw + 1;  // every CTA has read the old length
-    if (rank == 0) {
-        T* outp = reinterpret_cast<T*>(a.out) + (u * G) * D;
-        const int stride = G * D + 2 * G;
-        for (int idx = tid; idx < G * D; idx += DEC_THREADS) {
-            const int g = idx / D;
+    {
+        // per head: the common maximum, each source's factor, the denominator
+        float* fac = cacc;  // [CS][G] factors, then [G] reciprocal denominators (cacc is free now)
+        if (tid < G) {
             float M = -INFINITY;
-            for (int r = 0; r < CS; r++) M = fmaxf(M, gat[r * stride + G * D + g]);
-            float s = 0.f, lsum = 0.f;
+            for (int r = 0; r < CS; r++) M = fmaxf(M, gat[r * GST + SL + tid]);
+            float den = 0.f;
             for (int r = 0; r < CS; r++) {
-                const float mr = gat[r * stride + G * D + g];
+                const float mr = gat[r * GST + SL + tid];
                 const float f = (mr == -INFINITY) ? 0.f : expf(mr - M);
-                s += gat[r * stride + idx] * f;
-                lsum += gat[r * stride + G * D + G + g] * f;
+                fac[r * G + tid] = f;
+                den += gat[r * GST + SL + G + tid] * f;
             }
-            outp[idx] = from_f<T>(bad ? 0.f : s / lsum);
+            fac[CS * G + tid] = 1.f / den;
         }
+        __syncthreads();
+        T* outp = reinterpret_cast<T*>(a.out) + (u * G) * D + rank * SL;
+        for (int i = tid; i < SL; i += DEC_THREADS) {
+            const int g = (rank * SL + i) / D;
+            float s = 0.f;
+            for (int r = 0; r < CS; r++) s += gat[r * GST + i] * fac[r * G + g];
+            outp[i] = from_f<T>(bad ? 0.f : s * fac[CS * G + g]);
+        }
+    }
+    if (rank == 0) {
         int J = 0;
         if (!bad_len) {
             J = 1;

@@ -395,7 +395,8 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
         const long long S = p.len[u];
         const long long n_j = j == 0 ? S : ceil_div_ll(S, p.span[j]);
         const int nchild = (int)min((long long)b, n_j - (long long)par * b);
-        const long long crow = u * ustride + (long long)par * b;  // first child row
+        // first child row (a page of tokens at level 0 of a paged cache)
+        const long long crow = j == 0 ? token_row(token_map(p), u, (long long)par * b) : u * ustride + (long long)par * b;
         const bool valid = pr < npairs;
         int t = 0, r = 0, P = -1;
         if (valid) {
@@ -442,7 +443,8 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
         // the next tile's child rows into L2 while this one is computed
         if (ti + (int)gridDim.x < ntiles) {
             const int4 nt = L.tiles[ti + gridDim.x];
-            const long long nrow = (long long)nt.x * ustride + (long long)nt.y * b;
+            const long long nrow = j == 0 ? token_row(token_map(p), nt.x, (long long)nt.y * b)
+                                          : (long long)nt.x * ustride + (long long)nt.y * b;
             if (tid * 64 < b * D) prefetch_l2(kb + nrow * D + tid * 64);
             if (MODE == MODE_VALUE && tid * 64 < b * D) prefetch_l2(vb + nrow * D + tid * 64);
         }

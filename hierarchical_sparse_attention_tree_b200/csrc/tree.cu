@@ -54,8 +54,9 @@ __global__ void copy_tokens_kernel(TreeParams p, const T* __restrict__ k_new, co
         if (L + t >= p.cap) { flag_error(p.err, ERR_LENGTH); continue; }
         const uint4* ks = reinterpret_cast<const uint4*>(k_new + (r * D)) + piece;
         const uint4* vs = reinterpret_cast<const uint4*>(v_new + (r * D)) + piece;
-        T* kd = reinterpret_cast<T*>(p.K[0]) + (u * p.cap + L + t) * D;
-        T* vd = reinterpret_cast<T*>(p.V[0]) + (u * p.cap + L + t) * D;
+        const long long row = token_row(token_map(p), u, L + t);
+        T* kd = reinterpret_cast<T*>(p.K[0]) + row * D;
+        T* vd = reinterpret_cast<T*>(p.V[0]) + row * D;
         reinterpret_cast<uint4*>(kd)[piece] = *ks;
         reinterpret_cast<uint4*>(vd)[piece] = *vs;
     }
@@ -89,12 +90,14 @@ __global__ void __launch_bounds__(256) build_level_kernel(TreeParams p, int j, l
         return;
     }
 
+    const bool right_edge = (m == n_j - 1);
     const long long c_lo = m * p.b;
     const long long c_hi = min(c_lo + (long long)p.b, n_prev);
-    const bool right_edge = (m == n_j - 1);
-    const T* Kc = reinterpret_cast<const T*>(p.K[j - 1]) + (u * p.rows[j - 1]) * D + lane * DPL;
-    const T* Vc = reinterpret_cast<const T*>(p.V[0]) + (u * p.cap) * D + lane * DPL;  // j == 1
-    const float* Sc = (j >= 2) ? p.VS[j - 1] + (u * p.rows[j - 1]) * D + lane * DPL : nullptr;
+    // child rows c_lo .. c_hi - 1, indexed from c_lo (one page of tokens at j = 1)
+    const long long crow = j == 1 ? token_row(token_map(p), u, c_lo) : u * p.rows[j - 1] + c_lo;
+    const T* Kc = reinterpret_cast<const T*>(p.K[j - 1]) + (crow - c_lo) * D + lane * DPL;
+    const T* Vc = reinterpret_cast<const T*>(p.V[0]) + (crow - c_lo) * D + lane * DPL;  // j == 1
+    const float* Sc = (j >= 2) ? p.VS[j - 1] + (crow - c_lo) * D + lane * DPL : nullptr;
 
     float ks[DPL], vs[DPL];
 #pragma unroll
@@ -183,6 +186,7 @@ __global__ void __launch_bounds__(D) append_one_kernel(TreeParams p, const T* __
     float* scratch = reinterpret_cast<float*>(smem_a + D * D * sizeof(T));  // append_scratch_floats
     __shared__ uint64_t wbar;
     __shared__ LevelRef lv[MAXJ + 1];
+    __shared__ TokenMap tok;
     const long long u = blockIdx.x;
     // the next kernel on the stream (a decode) may start its own set-up now
     asm volatile("griddepcontrol.launch_dependents;");
@@ -192,6 +196,7 @@ __global__ void __launch_bounds__(D) append_one_kernel(TreeParams p, const T* __
         return;
     }
     if (threadIdx.x == 0) {
+        tok = token_map(p);
         mbar_init(&wbar, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(&wbar, (uint32_t)(D * D * sizeof(T)));
@@ -200,7 +205,7 @@ __global__ void __launch_bounds__(D) append_one_kernel(TreeParams p, const T* __
     load_levels(p, lv, threadIdx.x);
     __syncthreads();
     const bool ok = append_token<T, D>(
-        AppendDims{p.cap, p.J_cap, p.b}, lv, u, P, k_new + u * D, v_new + u * D, Wt, scratch,
+        AppendDims{p.cap, p.J_cap, p.b, &tok}, lv, u, P, k_new + u * D, v_new + u * D, Wt, scratch,
         [&]() {
             const int timed_out = !mbar_wait(&wbar, 0);
             if (__syncthreads_or(timed_out)) {  // same decision in every thread

@@ -10,15 +10,26 @@ from . import recsa as _r
 
 class RecsaLayer:
     def __init__(self, batch, n_kv_heads, n_q_heads, head_dim, branching, k, capacity, pooler_w: torch.Tensor,
-                 dtype=torch.bfloat16, rope_base=1e6, max_chunk=0, device="cuda", stream=None):
+                 dtype=torch.bfloat16, rope_base=1e6, max_chunk=0, device="cuda", stream=None, page_size=0,
+                 num_pages=0, page_table=None):
+        """page_size > 0: a paged token cache, a pool of num_pages pages of
+        page_size tokens (k_cache, v_cache [num_pages][H_kv][page_size][d])
+        with page_table [B][max_pages] (int32; copied to the device)."""
         self.cfg = _r.make_config(batch, n_kv_heads, n_q_heads, head_dim, branching, k, capacity, dtype, rope_base,
                                   max_chunk)
         self.dtype, self.device = dtype, torch.device(device)
-        self.k_cache = torch.zeros(batch, n_kv_heads, capacity, head_dim, dtype=dtype, device=device)
+        self.page_size = page_size
+        if page_size:
+            self.k_cache = torch.zeros(num_pages, n_kv_heads, page_size, head_dim, dtype=dtype, device=device)
+            self.page_table = torch.as_tensor(page_table, dtype=torch.int32).to(device).contiguous()
+        else:
+            self.k_cache = torch.zeros(batch, n_kv_heads, capacity, head_dim, dtype=dtype, device=device)
+            self.page_table = None
         self.v_cache = torch.zeros_like(self.k_cache)
         self.workspace = torch.zeros(_r.workspace_bytes(self.cfg), dtype=torch.uint8, device=device)
         w = pooler_w.to(device=device, dtype=dtype).contiguous()
-        self.ctx = _r.Context(self.cfg, self.k_cache, self.v_cache, self.workspace, w, stream)
+        self.ctx = _r.Context(self.cfg, self.k_cache, self.v_cache, self.workspace, w, stream, self.page_table,
+                              page_size)
         torch.cuda.current_stream(self.device).synchronize() if stream is None else stream.synchronize()
         self._scratch = None
 
@@ -27,12 +38,34 @@ class RecsaLayer:
         return self.cfg.n_q_heads // self.cfg.n_kv_heads
 
     def load(self, K: torch.Tensor, V: torch.Tensor, lengths, stream=None):
-        """Copy tokens [B][H][L][d] into the cache and build the tree over
-        the first lengths[b] tokens of each sequence."""
+        """Copy tokens [B][H][L][d] into the cache (through the page table
+        when paged) and build the tree over the first lengths[b] tokens of
+        each sequence."""
         L = K.shape[2]
-        self.k_cache[:, :, :L].copy_(K, non_blocking=True)
-        self.v_cache[:, :, :L].copy_(V, non_blocking=True)
+        if self.page_size:
+            P = self.page_size
+            table = self.page_table.cpu()
+            for b in range(K.shape[0]):
+                for pg in range(-(-L // P)):
+                    n = min(P, L - pg * P)
+                    dst = int(table[b, pg])
+                    self.k_cache[dst, :, :n].copy_(K[b, :, pg * P:pg * P + n], non_blocking=True)
+                    self.v_cache[dst, :, :n].copy_(V[b, :, pg * P:pg * P + n], non_blocking=True)
+        else:
+            self.k_cache[:, :, :L].copy_(K, non_blocking=True)
+            self.v_cache[:, :, :L].copy_(V, non_blocking=True)
         self.ctx.build_tree(lengths, stream)
+
+    def tokens(self, b: int, L: int):
+        """Keys and values [H][L][d] of sequence b's first L tokens (read
+        back through the page table when paged)."""
+        if not self.page_size:
+            return self.k_cache[b, :, :L], self.v_cache[b, :, :L]
+        P = self.page_size
+        pages = [int(x) for x in self.page_table[b, :-(-L // P)].cpu()]
+        k = torch.cat([self.k_cache[pg] for pg in pages], dim=1)[:, :L]
+        v = torch.cat([self.v_cache[pg] for pg in pages], dim=1)[:, :L]
+        return k, v
 
     def append(self, k_new, v_new, stream=None):
         self.ctx.append(k_new, v_new, stream)

@@ -19,7 +19,7 @@ F32, BF16 = 0, 1
 _TORCH_DTYPE = {F32: torch.float32, BF16: torch.bfloat16}
 
 EXPORTS = [
-    "recsa_workspace_bytes", "recsa_init", "recsa_build_tree", "recsa_append", "recsa_decode", "recsa_append_decode",
+    "recsa_workspace_bytes", "recsa_init", "recsa_init_paged", "recsa_build_tree", "recsa_append", "recsa_decode", "recsa_append_decode",
     "recsa_prefill_scratch_bytes", "recsa_prefill", "recsa_get_lengths", "recsa_tree_shape", "recsa_level_arrays",
     "recsa_query_stats", "recsa_check_device", "recsa_last_error", "recsa_destroy", "recsa_dense_decode_scratch_bytes",
     "recsa_dense_decode", "recsa_dense_decode_static",
@@ -54,6 +54,7 @@ def lib():
         sig = {
             "recsa_workspace_bytes": (sz, [P(Config)]),
             "recsa_init": (i32, [P(vp), P(Config), vp, vp, vp, sz, vp, vp]),
+            "recsa_init_paged": (i32, [P(vp), P(Config), vp, vp, i64, i32, vp, i32, vp, sz, vp, vp]),
             "recsa_build_tree": (i32, [vp, P(i64), vp]),
             "recsa_append": (i32, [vp, vp, vp, i32, vp]),
             "recsa_decode": (i32, [vp, vp, vp, vp, vp, vp]),
@@ -135,12 +136,22 @@ class Context:
     by this object."""
 
     def __init__(self, cfg: Config, k_cache: torch.Tensor, v_cache: torch.Tensor, workspace: torch.Tensor,
-                 pooler_w: torch.Tensor, stream=None):
+                 pooler_w: torch.Tensor, stream=None, page_table: torch.Tensor | None = None, page_size: int = 0):
+        """Contiguous cache: k_cache, v_cache [B][H_kv][capacity][d]. Paged:
+        k_cache, v_cache are the page pools [num_pages][H_kv][page_size][d]
+        and page_table the device int32 [B][max_pages] table."""
         self.cfg = cfg
-        self._keep = (k_cache, v_cache, workspace)
+        self._keep = (k_cache, v_cache, workspace, page_table)
         h = ctypes.c_void_p()
-        _check(lib().recsa_init(ctypes.byref(h), ctypes.byref(cfg), _ptr(k_cache), _ptr(v_cache), _ptr(workspace),
-                                workspace.numel() * workspace.element_size(), _ptr(pooler_w), _stream(stream)))
+        if page_table is None:
+            _check(lib().recsa_init(ctypes.byref(h), ctypes.byref(cfg), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(pooler_w),
+                                    _stream(stream)))
+        else:
+            _check(lib().recsa_init_paged(ctypes.byref(h), ctypes.byref(cfg), _ptr(k_cache), _ptr(v_cache),
+                                          k_cache.shape[0], page_size, _ptr(page_table), page_table.shape[1],
+                                          _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                          _ptr(pooler_w), _stream(stream)))
         self.handle = h
 
     def close(self):

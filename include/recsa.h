@@ -95,6 +95,25 @@ size_t recsa_workspace_bytes(const recsa_config* cfg);
 recsa_status recsa_init(recsa_ctx** out, const recsa_config* cfg, void* k_cache, void* v_cache, void* workspace,
                         size_t workspace_bytes, const void* pooler_w, recsa_stream_t stream);
 
+/* recsa_init with a paged token cache: instead of K, V [B][H_kv][capacity]
+ * [d], the tokens live in a pool of pages shared by the sequences, K, V
+ * [num_pages][H_kv][page_size][d] (the caller's, borrowed). Token t of
+ * sequence b is row t % page_size of pool page page_table[b * max_pages +
+ * t / page_size]; page_table (device int32 [B][max_pages], borrowed) is
+ * read by the kernels at every call, so the caller assigns a page before the
+ * tokens that land in it are appended (for example a serving engine handing
+ * out pages on demand), and may change entries of pages not yet used.
+ * page_size must be a multiple of the branching factor (the children of a
+ * level-1 node, b consecutive tokens, then lie in one page) and max_pages *
+ * page_size must cover cfg->capacity. The tree levels stay in the workspace.
+ * A page id outside [0, num_pages) is reported by recsa_check_device (shape
+ * bit) and page 0 is read instead. Every other call is unchanged. This is
+ * the paged, variable-length cache of a serving engine; the pages (RecSA
+ * abstract: a tree over the KV cache) do not change what is computed. */
+recsa_status recsa_init_paged(recsa_ctx** out, const recsa_config* cfg, void* k_pool, void* v_pool,
+                              long long num_pages, int page_size, const int* page_table, int max_pages,
+                              void* workspace, size_t workspace_bytes, const void* pooler_w, recsa_stream_t stream);
+
 /* Sets sequence b's length to lengths[b] (host array of B entries, each in
  * [0, capacity]) and builds every tree level from the tokens already in the
  * cache. The tree is the one the RecSA abstract keeps over the KV cache: node

@@ -75,3 +75,18 @@ def test_decode_shared_memory_limit_checked_at_init():
     st = R.lib().recsa_init(ctypes.byref(h), ctypes.byref(cfg), fake, fake, fake, 0, fake, None)
     assert st == R.ERR_UNSUPPORTED and not h.value
     assert b"shared memory" in R.lib().recsa_last_error()
+
+
+def test_paged_init_checks_page_geometry():
+    """recsa_init_paged refuses a page size that is not a multiple of the
+    branching factor and a page table too small for the capacity, before any
+    device call (the buffers below are never touched)."""
+    cfg = R.make_config(1, 8, 32, 128, 64, 16, 4096)
+    h = ctypes.c_void_p()
+    fake = ctypes.c_void_p(1 << 20)
+    st = R.lib().recsa_init_paged(ctypes.byref(h), ctypes.byref(cfg), fake, fake, 64, 96, fake, 64, fake, 1 << 40,
+                                  fake, None)
+    assert st == R.ERR_INVALID_ARG and b"multiple of branching" in R.lib().recsa_last_error()
+    st = R.lib().recsa_init_paged(ctypes.byref(h), ctypes.byref(cfg), fake, fake, 64, 64, fake, 8, fake, 1 << 40,
+                                  fake, None)
+    assert st == R.ERR_INVALID_ARG and b"cover the capacity" in R.lib().recsa_last_error()
