@@ -57,6 +57,9 @@ def _load():
             lib.orc_build.argtypes = [vp, vp, i32, i64, i32, i32, vp, i32, i64, i32, vp, vp]
             lib.orc_pool_level.restype = i32
             lib.orc_pool_level.argtypes = [vp, i64, i32, i32, vp, i32, vp]
+            lib.orc_query_grad.restype = i32
+            lib.orc_query_grad.argtypes = [i32, i32, i32, i32, dbl, i64, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp,
+                                           vp]
             lib.orc_query.restype = i32
             lib.orc_query.argtypes = [i32, i32, i32, i32, dbl, i64, vp, vp, vp, vp, i32, vp, vp, i64, vp, vp, vp, vp,
                                       vp]
@@ -168,6 +171,30 @@ def query(tree_K, tree_V, Ktok, Vtok, T, q, d, b, k, G, rope_base, Kloc=None, Vl
     if J < 0:
         raise ValueError("oracle query rejected its arguments")
     return dict(out=out, sel=sel[:J], margin=margin[:J], k_rows=int(rows[0]), v_rows=int(rows[1]), J=J)
+
+
+def query_grad(tree_K, tree_V, Ktok, Vtok, T, q, dout, W, d, b, k, G, rope_base):
+    """Gradients of one decode query with the selections held fixed.
+    Returns dict(dq [G][d], dK [T][d], dV [T][d], dW [d][d]) in fp64."""
+    lib = _load()
+    kt, dt = _tok(Ktok)
+    vt, _ = _tok(Vtok)
+    Jt, _ = levels(T, b)
+    qf = np.ascontiguousarray(q, dtype=np.float32)
+    do = np.ascontiguousarray(dout, dtype=np.float64)
+    Wf = np.ascontiguousarray(W, dtype=np.float32)
+    dq = np.zeros((G, d))
+    dK = np.zeros((T, d))
+    dV = np.zeros((T, d))
+    dW = np.zeros((d, d))
+    Kp = [None] + [np.ascontiguousarray(x, dtype=np.float64) for x in tree_K[1:Jt + 1]]
+    Vp = [None] + [np.ascontiguousarray(x, dtype=np.float64) for x in tree_V[1:Jt + 1]]
+    J = lib.orc_query_grad(d, b, k, G, rope_base, T, _ptr_array(Kp), _ptr_array(Vp), kt.ctypes.data, vt.ctypes.data,
+                           dt, Wf.ctypes.data, qf.ctypes.data, do.ctypes.data, dq.ctypes.data, dK.ctypes.data,
+                           dV.ctypes.data, dW.ctypes.data)
+    if J < 0:
+        raise ValueError("oracle gradient rejected its arguments")
+    return dict(dq=dq, dK=dK, dV=dV, dW=dW, J=J)
 
 
 def query_tree(tree: Tree, Ktok, Vtok, q, k, G, rope_base, Kloc=None, Vloc=None, T=None):

@@ -354,3 +354,206 @@ int orc_query(int d, int b, int k, int G, double rope_base, long long T, const d
     free(sl);
     return J;
 }
+
+/* ----------------------------------------------------------- gradients */
+
+/* Gradient of one decode query's output (orc_query with no local tokens)
+ * with the selections held fixed (they are not differentiable): given
+ * dout [G][d], returns dq [G][d] (overwritten) and adds into dKtok, dVtok
+ * [T][d] and dW [d][d] the gradients with respect to the token keys and
+ * values and the pooler, through the direct token entries and through the
+ * summaries (a node value is the mean of its subtree's token values, a node
+ * key is W times the mean of its children's stored keys; storage rounding is
+ * taken as the identity). Written from the definitions, step by step:
+ *   logit l_e,g = <rope(q_g, P), rope(k_e, i)> / sqrt(d), p = softmax_e(l),
+ *   out_g = sum_e p_e,g v_e;
+ *   dv_e = sum_g p_e,g dout_g;  dl_e,g = p_e,g (<dout_g, v_e> - sum_f p_f,g <dout_g, v_f>);
+ *   dq_g = sum_e dl_e,g rope(k_e, i - P) / sqrt(d);  dk_e = sum_g dl_e,g rope(q_g, P - i) / sqrt(d);
+ * then, level by level from the top, the key gradient g_m of node m (its own
+ * entry gradient plus W^T g_parent / children(parent)) adds g_m mean_m^T to
+ * dW, and each token gets W^T g_parent / children(parent) for its level-1
+ * parent plus, for every ancestor a, dv_a / tokens(a).
+ * Returns J, or -1 on bad arguments / allocation failure. */
+int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, const double* const* Knode,
+                   const double* const* Vnode, const void* Ktok, const void* Vtok, int tok_dtype, const float* W,
+                   const float* q, const double* dout, double* dq, double* dKtok, double* dVtok, double* dW) {
+    if (d <= 0 || d % 2 || b < 2 || k < 1 || G < 1 || T < 1) return -1;
+    long long n[ORC_MAXLEV + 1];
+    int J = orc_levels(T, b, n);
+    int* sel = (int*)malloc(sizeof(int) * (size_t)(J * k + 1));
+    double* out = (double*)malloc(sizeof(double) * (size_t)(G * d));
+    if (!sel || !out) {
+        free(sel);
+        free(out);
+        return -1;
+    }
+    /* the forward's selections */
+    if (orc_query(d, b, k, G, rope_base, T, Knode, Vnode, Ktok, Vtok, tok_dtype, NULL, NULL, 0, q, out, sel, NULL,
+                  NULL) != J) {
+        free(sel);
+        free(out);
+        return -1;
+    }
+    double scale = 1.0 / sqrt((double)d);
+    long long max_cand = (long long)k * b > b ? (long long)k * b : b;
+    long long max_ent = (long long)(J + 1) * max_cand + 1;
+    long long* cand = (long long*)malloc(sizeof(long long) * (size_t)max_cand);
+    long long* next = (long long*)malloc(sizeof(long long) * (size_t)max_cand);
+    int* e_lev = (int*)malloc(sizeof(int) * (size_t)max_ent);
+    long long* e_id = (long long*)malloc(sizeof(long long) * (size_t)max_ent);
+    long long* e_rank = (long long*)malloc(sizeof(long long) * (size_t)max_ent);
+    long long* e_pos = (long long*)malloc(sizeof(long long) * (size_t)max_ent);
+    double* lg = (double*)malloc(sizeof(double) * (size_t)(max_ent * G));
+    double* kv = (double*)malloc(sizeof(double) * (size_t)d);
+    double* vv = (double*)malloc(sizeof(double) * (size_t)d);
+    double* qd = (double*)malloc(sizeof(double) * (size_t)d);
+    double* r1 = (double*)malloc(sizeof(double) * (size_t)d);
+    double* r2 = (double*)malloc(sizeof(double) * (size_t)d);
+    /* per-level node gradients (entries) and the top-down sums */
+    double** dKn = (double**)calloc((size_t)J + 2, sizeof(double*));
+    double** dVn = (double**)calloc((size_t)J + 2, sizeof(double*));
+    int ok = cand && next && e_lev && e_id && e_rank && e_pos && lg && kv && vv && qd && r1 && r2 && dKn && dVn;
+    for (int j = 1; ok && j <= J; j++) {
+        dKn[j] = (double*)calloc((size_t)(n[j] * d), sizeof(double));
+        dVn[j] = (double*)calloc((size_t)(n[j] * d), sizeof(double));
+        ok = dKn[j] && dVn[j];
+    }
+    long long n_ent = 0;
+    if (ok) {
+        /* the entries: unselected candidates of every level, then the tokens
+         * under the selected level-1 nodes (as the forward) */
+        long long nc = n[J];
+        for (long long i = 0; i < nc; i++) cand[i] = i;
+        for (int j = J; j >= 1; j--) {
+            long long kk = nc < k ? nc : k;
+            for (long long i = 0; i < nc; i++) {
+                int chosen = 0;
+                for (long long r = 0; r < kk; r++) chosen |= (sel[(j - 1) * k + r] == cand[i]);
+                if (chosen) continue;
+                e_lev[n_ent] = j;
+                e_id[n_ent] = cand[i];
+                e_rank[n_ent] = i;
+                e_pos[n_ent] = nc - 1;
+                n_ent++;
+            }
+            long long nn = 0;
+            for (long long r = 0; r < kk; r++) {
+                long long m = sel[(j - 1) * k + r];
+                long long c_lo = m * b, c_hi = (m + 1) * b < n[j - 1] ? (m + 1) * b : n[j - 1];
+                for (long long c = c_lo; c < c_hi; c++) next[nn++] = c;
+            }
+            memcpy(cand, next, sizeof(long long) * (size_t)nn);
+            nc = nn;
+        }
+        for (long long i = 0; i < nc; i++) {
+            e_lev[n_ent] = 0;
+            e_id[n_ent] = cand[i];
+            e_rank[n_ent] = i;
+            e_pos[n_ent] = nc - 1;
+            n_ent++;
+        }
+        /* logits and softmax per head */
+        for (long long e = 0; e < n_ent; e++) {
+            for (int i = 0; i < d; i++)
+                kv[i] = e_lev[e] ? Knode[e_lev[e]][e_id[e] * d + i] : tok_at(Ktok, tok_dtype, e_id[e] * d + i);
+            rope(kv, e_rank[e], d, rope_base, r1);
+            for (int g = 0; g < G; g++) {
+                for (int i = 0; i < d; i++) qd[i] = (double)q[g * d + i];
+                rope(qd, e_pos[e], d, rope_base, r2);
+                double dot = 0.0;
+                for (int i = 0; i < d; i++) dot += r2[i] * r1[i];
+                lg[e * G + g] = dot * scale;
+            }
+        }
+        for (int g = 0; g < G; g++) {
+            double mx = -HUGE_VAL, den = 0.0, Dg = 0.0;
+            for (long long e = 0; e < n_ent; e++) mx = lg[e * G + g] > mx ? lg[e * G + g] : mx;
+            for (long long e = 0; e < n_ent; e++) den += exp(lg[e * G + g] - mx);
+            /* p_e, <dout, v_e> and their weighted sum D */
+            for (long long e = 0; e < n_ent; e++) {
+                double p = exp(lg[e * G + g] - mx) / den, a = 0.0;
+                for (int i = 0; i < d; i++) {
+                    vv[i] = e_lev[e] ? Vnode[e_lev[e]][e_id[e] * d + i] : tok_at(Vtok, tok_dtype, e_id[e] * d + i);
+                    a += dout[g * d + i] * vv[i];
+                }
+                Dg += p * a;
+            }
+            for (int i = 0; i < d; i++) dq[g * d + i] = 0.0;
+            for (long long e = 0; e < n_ent; e++) {
+                double p = exp(lg[e * G + g] - mx) / den, a = 0.0;
+                for (int i = 0; i < d; i++) {
+                    vv[i] = e_lev[e] ? Vnode[e_lev[e]][e_id[e] * d + i] : tok_at(Vtok, tok_dtype, e_id[e] * d + i);
+                    a += dout[g * d + i] * vv[i];
+                }
+                double dl = p * (a - Dg);
+                /* dq: the key rotated by i - P; dk: the query rotated by P - i */
+                for (int i = 0; i < d; i++)
+                    kv[i] = e_lev[e] ? Knode[e_lev[e]][e_id[e] * d + i] : tok_at(Ktok, tok_dtype, e_id[e] * d + i);
+                rope(kv, e_rank[e] - e_pos[e], d, rope_base, r1);
+                for (int i = 0; i < d; i++) qd[i] = (double)q[g * d + i];
+                rope(qd, e_pos[e] - e_rank[e], d, rope_base, r2);
+                double* dk = e_lev[e] ? dKn[e_lev[e]] + e_id[e] * d : dKtok + e_id[e] * d;
+                double* dv = e_lev[e] ? dVn[e_lev[e]] + e_id[e] * d : dVtok + e_id[e] * d;
+                for (int i = 0; i < d; i++) {
+                    dq[g * d + i] += dl * scale * r1[i];
+                    dk[i] += dl * scale * r2[i];
+                    dv[i] += p * dout[g * d + i];
+                }
+            }
+        }
+        /* top-down through the tree: hk = W^T g / children (to the children's
+         * keys), hv = dv / tokens accumulated over the ancestors (to every
+         * token of the subtree); dW += g mean^T */
+        double* hk_up = NULL;
+        double* hv_up = NULL;
+        for (int j = J; j >= 1 && ok; j--) {
+            double* hk = (double*)calloc((size_t)(n[j] * d), sizeof(double));
+            double* hv = (double*)calloc((size_t)(n[j] * d), sizeof(double));
+            if (!hk || !hv) {
+                free(hk);
+                free(hv);
+                ok = 0;
+                break;
+            }
+            long long span = ipow_sat(b, j);
+            for (long long m = 0; m < n[j]; m++) {
+                long long c_lo = m * b, c_hi = (m + 1) * b < n[j - 1] ? (m + 1) * b : n[j - 1];
+                long long t_lo = m * span, t_hi = (m + 1) * span < T ? (m + 1) * span : T;
+                for (int i = 0; i < d; i++) {
+                    qd[i] = dKn[j][m * d + i] + (hk_up ? hk_up[(m / b) * d + i] : 0.0); /* g_m */
+                    hv[m * d + i] = dVn[j][m * d + i] / (double)(t_hi - t_lo) + (hv_up ? hv_up[(m / b) * d + i] : 0.0);
+                    double s = 0.0;
+                    for (long long c = c_lo; c < c_hi; c++)
+                        s += (j == 1) ? tok_at(Ktok, tok_dtype, c * d + i) : Knode[j - 1][c * d + i];
+                    kv[i] = s / (double)(c_hi - c_lo); /* mean of the children's keys */
+                }
+                for (int r = 0; r < d; r++)
+                    for (int c = 0; c < d; c++) dW[r * d + c] += qd[r] * kv[c];
+                for (int c = 0; c < d; c++) {
+                    double s = 0.0;
+                    for (int r = 0; r < d; r++) s += (double)W[r * d + c] * qd[r];
+                    hk[m * d + c] = s / (double)(c_hi - c_lo);
+                }
+            }
+            free(hk_up);
+            free(hv_up);
+            hk_up = hk;
+            hv_up = hv;
+        }
+        if (ok && hk_up)
+            for (long long t = 0; t < T; t++)
+                for (int i = 0; i < d; i++) {
+                    dKtok[t * d + i] += hk_up[(t / b) * d + i];
+                    dVtok[t * d + i] += hv_up[(t / b) * d + i];
+                }
+        free(hk_up);
+        free(hv_up);
+    }
+    for (int j = 1; j <= J; j++) {
+        if (dKn) free(dKn[j]);
+        if (dVn) free(dVn[j]);
+    }
+    free(dKn); free(dVn); free(sel); free(out); free(cand); free(next); free(e_lev); free(e_id); free(e_rank);
+    free(e_pos); free(lg); free(kv); free(vv); free(qd); free(r1); free(r2);
+    return ok ? J : -1;
+}

@@ -64,6 +64,16 @@ int orc_query(int d, int b, int k, int G, double rope_base, long long T, const d
               const void* Vloc, long long nloc, const float* q, double* out, int* sel, double* margin,
               long long* rows);
 
+/* Gradients of one decode query (no local tokens) with the selections
+ * held fixed: dq [G][d] is overwritten; the gradients with respect to the
+ * token keys and values (dKtok, dVtok [T][d], through the entries and the
+ * summaries) and the pooler (dW [d][d], row-major like W) are added into
+ * the given arrays. dout [G][d] is the output gradient. Storage rounding is
+ * taken as the identity. Returns J, or -1. */
+int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, const double* const* Knode,
+                   const double* const* Vnode, const void* Ktok, const void* Vtok, int tok_dtype, const float* W,
+                   const float* q, const double* dout, double* dq, double* dKtok, double* dVtok, double* dW);
+
 #ifdef __cplusplus
 }
 #endif
