@@ -9,6 +9,7 @@
 #include <vector>
 
 #include "../../include/recsa.h"
+#include "backward.cuh"
 #include "common.cuh"
 
 namespace recsa {
@@ -590,6 +591,110 @@ recsa_status recsa_dense_decode_static(const void* k_cache, const void* v_cache,
                 DISPATCH_G(G, e = launch_dense<T, DD, GG>(k_cache, v_cache, q, out, units, length, l_stride, scratch,
                                                          max_splits < 256 ? max_splits : 256, s)));
     if (e != cudaSuccess) return cuda_fail(e, "recsa_dense_decode_static");
+    return RECSA_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------ backward
+
+namespace {
+// Backward scratch: [node-key accumulators, levels 1..J_cap][node-value
+// accumulators, levels 1..J_cap] (fp32, [B*H][rows[j]][d] each; the prefix
+// the tree pass clears) then the per-call plan, logits, <dout, v> and
+// softmax statistics.
+struct BwdLayout {
+    size_t gK[MAXJ + 1], gV[MAXJ + 1], nodes_end, plan, lg, ag, st, total;
+    int E_cap;
+};
+BwdLayout bwd_layout(const recsa_config* c) {
+    BwdLayout b{};
+    const Layout l = layout_for(c);
+    const size_t units = (size_t)c->batch * c->n_kv_heads, D = c->head_dim;
+    const size_t G = (size_t)(c->n_q_heads / c->n_kv_heads);
+    size_t o = 0;
+    for (int j = 1; j <= l.J_cap; j++) { b.gK[j] = o; o = align256(o + units * (size_t)l.rows[j] * D * 4); }
+    for (int j = 1; j <= l.J_cap; j++) { b.gV[j] = o; o = align256(o + units * (size_t)l.rows[j] * D * 4); }
+    b.nodes_end = o;
+    long long maxc = (long long)c->k * c->branching;
+    if (maxc < c->branching) maxc = c->branching;
+    b.E_cap = (int)((l.J_cap + 1) * maxc);
+    b.plan = o; o = align256(o + units * PLAN_INTS * 4);
+    b.lg = o; o = align256(o + units * (size_t)b.E_cap * G * 4);
+    b.ag = o; o = align256(o + units * (size_t)b.E_cap * G * 4);
+    b.st = o; o = align256(o + units * G * 3 * 4);
+    b.total = o;
+    return b;
+}
+BwdArgs bwd_args(const recsa_ctx* ctx, void* scratch) {
+    const BwdLayout l = bwd_layout(&ctx->cfg);
+    char* base = static_cast<char*>(scratch);
+    BwdArgs a{};
+    for (int j = 1; j <= ctx->p.J_cap; j++) {
+        a.gK[j] = reinterpret_cast<float*>(base + l.gK[j]);
+        a.gV[j] = reinterpret_cast<float*>(base + l.gV[j]);
+    }
+    a.plan = reinterpret_cast<int*>(base + l.plan);
+    a.lg = reinterpret_cast<float*>(base + l.lg);
+    a.ag = reinterpret_cast<float*>(base + l.ag);
+    a.st = reinterpret_cast<float*>(base + l.st);
+    a.E_cap = l.E_cap;
+    return a;
+}
+}  // namespace
+
+extern "C" {
+
+size_t recsa_backward_scratch_bytes(const recsa_config* cfg) {
+    if (check_config(cfg) != RECSA_OK) return 0;
+    return bwd_layout(cfg).total;
+}
+
+recsa_status recsa_decode_backward(recsa_ctx* ctx, const void* q, const void* dout, const int* sel, float* dq,
+                                   float* dk, float* dv, void* scratch, size_t scratch_bytes, recsa_stream_t stream) {
+    if (!ctx || !q || !dout || !sel || !dq || !dk || !dv || !scratch) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    if (!aligned(q, 16) || !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16))
+        return fail(RECSA_ERR_INVALID_ARG, "q/dout/dq/dk/dv not 16-byte aligned");
+    if (!aligned(scratch, 256)) return fail(RECSA_ERR_INVALID_ARG, "scratch not 256-byte aligned");
+    const recsa_config& c = ctx->cfg;
+    if (scratch_bytes < bwd_layout(&c).total)
+        return fail(RECSA_ERR_INVALID_ARG, "scratch of %zu bytes, %zu needed", scratch_bytes, bwd_layout(&c).total);
+    for (int b = 0; b < c.batch; b++)
+        if (ctx->len[b] < 1) return fail(RECSA_ERR_INVALID_ARG, "sequence %d holds no tokens", b);
+    BwdArgs a = bwd_args(ctx, scratch);
+    a.q = q;
+    a.dout = dout;
+    a.sel = sel;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    DISPATCH_TD(c.dtype, c.head_dim, DISPATCH_G(ctx->G, e = launch_decode_backward<T, DD, GG>(ctx->p, a, s)));
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_decode_backward");
+    return RECSA_OK;
+}
+
+recsa_status recsa_tree_backward(recsa_ctx* ctx, float* dk, float* dv, float* dw, void* scratch,
+                                 size_t scratch_bytes, recsa_stream_t stream) {
+    if (!ctx || !dk || !dv || !dw || !scratch) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    if (!aligned(dk, 16) || !aligned(dv, 16) || !aligned(dw, 16))
+        return fail(RECSA_ERR_INVALID_ARG, "dk/dv/dw not 16-byte aligned");
+    if (!aligned(scratch, 256)) return fail(RECSA_ERR_INVALID_ARG, "scratch not 256-byte aligned");
+    const recsa_config& c = ctx->cfg;
+    const BwdLayout l = bwd_layout(&c);
+    if (scratch_bytes < l.total) return fail(RECSA_ERR_INVALID_ARG, "scratch of %zu bytes, %zu needed", scratch_bytes, l.total);
+    BwdArgs a = bwd_args(ctx, scratch);
+    a.dk = dk;
+    a.dv = dv;
+    a.dw = dw;
+    long long maxL = 0;
+    for (int b = 0; b < c.batch; b++) maxL = ctx->len[b] > maxL ? ctx->len[b] : maxL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (maxL > 0) DISPATCH_TD(c.dtype, c.head_dim, e = launch_tree_backward<T, DD>(ctx->p, a, maxL, s));
+    if (e == cudaSuccess) e = cudaMemsetAsync(scratch, 0, l.nodes_end, s);
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_tree_backward");
     return RECSA_OK;
 }
 

@@ -1,0 +1,33 @@
+// Arguments of the decode-backward kernels, shared by their launchers and
+// the C ABI's host code.
+#pragma once
+
+#include "common.cuh"
+
+namespace recsa {
+
+constexpr int PLAN_INTS = 72;          // valid, J, items, pad, then off[j], nc[j] for j = 0..MAXJ
+
+struct BwdArgs {
+    const void* q;     // [B][Hq][D], storage type
+    const void* dout;  // [B][Hq][D], storage type
+    const int* sel;    // [B*H][J_cap][k], the forward's selections
+    float* dq;         // [B][Hq][D]
+    float* dk;         // token gradients, the cache's row layout, [rows][D]
+    float* dv;
+    float* dw;         // [D][D], dW[r][c] for W[r][c]
+    float* gK[MAXJ + 1];  // node-key gradient accumulators [B*H][rows[j]][D] (j >= 1)
+    float* gV[MAXJ + 1];  // node-value gradient accumulators
+    int* plan;         // [B*H][PLAN_INTS]
+    float* lg;         // [B*H][E_cap][G] logits (-inf: not an entry)
+    float* ag;         // [B*H][E_cap][G] <dout_g, v_e>
+    float* st;         // [B*H][G][3] softmax maximum, denominator, sum_e p_e <dout, v_e>
+    int E_cap;
+};
+
+template <typename T, int D, int G>
+cudaError_t launch_decode_backward(const TreeParams& p, const BwdArgs& a, cudaStream_t s);
+template <typename T, int D>
+cudaError_t launch_tree_backward(const TreeParams& p, const BwdArgs& a, long long max_len, cudaStream_t s);
+
+}  // namespace recsa

@@ -93,6 +93,41 @@ class RecsaLayer:
         self.ctx.prefill(q, k, v, out, sel_out, self._scratch, rows_out, stream)
         return out
 
+    # ------------------------------------------------------------ gradients
+
+    def zero_grad(self):
+        """Allocates (first call) or clears the fp32 gradients: dk, dv shaped
+        like the cache, dw [d][d], and the node accumulators."""
+        if getattr(self, "dk", None) is None:
+            self.dk = torch.zeros(self.k_cache.shape, dtype=torch.float32, device=self.device)
+            self.dv = torch.zeros_like(self.dk)
+            self.dw = torch.zeros(self.cfg.head_dim, self.cfg.head_dim, dtype=torch.float32, device=self.device)
+            self._bwd_scratch = torch.zeros(max(self.ctx.backward_scratch_bytes(), 256), dtype=torch.uint8,
+                                            device=self.device)
+        else:
+            self.dk.zero_()
+            self.dv.zero_()
+            self.dw.zero_()
+            self._bwd_scratch.zero_()
+
+    def decode_backward(self, q, dout, sel, dq=None, stream=None):
+        """Gradients of the last decode's output with its selections sel
+        [B][H_kv][J_cap][k] held fixed: returns dq [B][H_q][d] (fp32) and adds
+        the token entries' gradients into self.dk, self.dv and the summaries'
+        into the node accumulators (carried down by tree_backward)."""
+        if getattr(self, "dk", None) is None:
+            self.zero_grad()
+        if dq is None:
+            dq = torch.empty(q.shape, dtype=torch.float32, device=self.device)
+        self.ctx.decode_backward(q, dout, sel, dq, self.dk, self.dv, self._bwd_scratch, stream)
+        return dq
+
+    def tree_backward(self, stream=None):
+        """Carries the node accumulators into self.dk, self.dv and self.dw."""
+        if getattr(self, "dk", None) is None:
+            self.zero_grad()
+        self.ctx.tree_backward(self.dk, self.dv, self.dw, self._bwd_scratch, stream)
+
     def query_stats(self, stream=None):
         return self.ctx.query_stats(stream)
 

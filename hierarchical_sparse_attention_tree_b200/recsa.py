@@ -22,7 +22,8 @@ EXPORTS = [
     "recsa_workspace_bytes", "recsa_init", "recsa_init_paged", "recsa_build_tree", "recsa_append", "recsa_decode", "recsa_append_decode",
     "recsa_prefill_scratch_bytes", "recsa_prefill", "recsa_get_lengths", "recsa_tree_shape", "recsa_level_arrays",
     "recsa_query_stats", "recsa_check_device", "recsa_last_error", "recsa_destroy", "recsa_dense_decode_scratch_bytes",
-    "recsa_dense_decode", "recsa_dense_decode_static",
+    "recsa_dense_decode", "recsa_dense_decode_static", "recsa_backward_scratch_bytes", "recsa_decode_backward",
+    "recsa_tree_backward",
 ]
 
 
@@ -58,6 +59,9 @@ def lib():
             "recsa_build_tree": (i32, [vp, P(i64), vp]),
             "recsa_append": (i32, [vp, vp, vp, i32, vp]),
             "recsa_decode": (i32, [vp, vp, vp, vp, vp, vp]),
+            "recsa_backward_scratch_bytes": (sz, [P(Config)]),
+            "recsa_decode_backward": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+            "recsa_tree_backward": (i32, [vp, vp, vp, vp, vp, sz, vp]),
             "recsa_append_decode": (i32, [vp, vp, vp, vp, vp, vp, vp, vp]),
             "recsa_prefill_scratch_bytes": (sz, [P(Config), i32]),
             "recsa_prefill": (i32, [vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
@@ -194,6 +198,18 @@ class Context:
         nbytes = 0 if scratch is None else scratch.numel() * scratch.element_size()
         _check(lib().recsa_prefill(self.handle, _ptr(q), _ptr(k), _ptr(v), C, _ptr(out), _ptr(sel_out),
                                    _ptr(rows_out), _ptr(scratch), nbytes, _stream(stream)))
+
+    def backward_scratch_bytes(self) -> int:
+        return lib().recsa_backward_scratch_bytes(ctypes.byref(self.cfg))
+
+    def decode_backward(self, q, dout, sel, dq, dk, dv, scratch, stream=None):
+        _check(lib().recsa_decode_backward(self.handle, _ptr(q), _ptr(dout), _ptr(sel), _ptr(dq), _ptr(dk), _ptr(dv),
+                                           _ptr(scratch), scratch.numel() * scratch.element_size(),
+                                           _stream(stream)))
+
+    def tree_backward(self, dk, dv, dw, scratch, stream=None):
+        _check(lib().recsa_tree_backward(self.handle, _ptr(dk), _ptr(dv), _ptr(dw), _ptr(scratch),
+                                         scratch.numel() * scratch.element_size(), _stream(stream)))
 
     def query_stats(self, stream=None):
         """(depth, k_rows, v_rows) of the last decode, per (sequence, KV head)

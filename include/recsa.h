@@ -198,6 +198,53 @@ recsa_status recsa_level_arrays(const recsa_ctx* ctx, int level, void** keys, vo
 recsa_status recsa_query_stats(recsa_ctx* ctx, int* depth, long long* k_rows, long long* v_rows,
                                recsa_stream_t stream);
 
+/* ---------------------------------------------------------------------
+ * Gradients of decode queries (the training side of the method). The RecSA
+ * abstract's output is one softmax over the summaries of the candidates not
+ * kept and the exact tokens under the kept level-1 nodes; a summary's value
+ * is the mean of its subtree's token values and its key the pooler W applied
+ * to the mean of its children's keys (kongchang.com article, "Core Idea"),
+ * so the gradient of a query's output reaches q, every cached token's key
+ * and value, and W. The top-k choice is discrete and held fixed: the caller
+ * passes the selections its recsa_decode returned. Rounding of stored node
+ * keys and values to the storage type is taken as the identity.
+ *
+ * Two stages, so that any number of queries can be summed before the part
+ * whose cost grows with the cache:
+ *   recsa_decode_backward  per query: dq, and the gradients of the softmax
+ *                          entries (tokens: added into dk, dv; summaries:
+ *                          added into node accumulators held in `scratch`);
+ *   recsa_tree_backward    once: carries the node accumulators down the
+ *                          tree into every token's dk, dv and into dw, then
+ *                          clears them.
+ * `scratch`: device memory of recsa_backward_scratch_bytes(cfg) bytes,
+ * 256-byte aligned, ZEROED by the caller before its first use; every
+ * recsa_tree_backward leaves it zeroed again. Gradient arrays are fp32:
+ *   dk, dv  one row of d per cache row, in the cache's own layout (contiguous
+ *           [B][H_kv][capacity][d]; paged [num_pages][H_kv][page_size][d]);
+ *           both calls ADD into them;
+ *   dw      [d][d], dw[r][c] = dLoss/dW[r][c] (W row-major as given to
+ *           recsa_init); recsa_tree_backward ADDS into it.
+ * Asynchronous on `stream`; the context's tree and lengths must be the ones
+ * the forward used (no append in between). */
+size_t recsa_backward_scratch_bytes(const recsa_config* cfg);
+
+/* q [B][H_q][d] (the forward's query) and dout [B][H_q][d] (dLoss/dout),
+ * both in cfg->dtype, device, 16-byte aligned; sel [B][H_kv][J_cap][k]
+ * int32 device, as recsa_decode's sel_out wrote it. dq [B][H_q][d] fp32 is
+ * overwritten. A unit whose selections are not a valid descent over its
+ * tree is skipped (its dq is zero) and flagged in the device error word
+ * (bit 2, read by recsa_check_device). RECSA_ERR_INVALID_ARG (nothing
+ * launched) for NULL or misaligned pointers, a short scratch or an empty
+ * sequence. */
+recsa_status recsa_decode_backward(recsa_ctx* ctx, const void* q, const void* dout, const int* sel, float* dq,
+                                   float* dk, float* dv, void* scratch, size_t scratch_bytes, recsa_stream_t stream);
+
+/* Carries the node accumulators in `scratch` into dk, dv and dw (see
+ * above), level by level from the top, and clears them. */
+recsa_status recsa_tree_backward(recsa_ctx* ctx, float* dk, float* dv, float* dw, void* scratch,
+                                 size_t scratch_bytes, recsa_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the device error word:
  * RECSA_ERR_DEVICE if a kernel flagged an inconsistent state (bits: 1 a
  * length out of range, 2 a tree shape inconsistent with the lengths, 4 a

@@ -90,3 +90,17 @@ def test_paged_init_checks_page_geometry():
     st = R.lib().recsa_init_paged(ctypes.byref(h), ctypes.byref(cfg), fake, fake, 64, 64, fake, 8, fake, 1 << 40,
                                   fake, None)
     assert st == R.ERR_INVALID_ARG and b"cover the capacity" in R.lib().recsa_last_error()
+
+
+def test_backward_scratch_and_null_arguments():
+    """The backward scratch holds two fp32 rows per tree node (about 2/b of
+    the fp32 token gradients) plus small per-call arrays; NULL arguments
+    are rejected on the host."""
+    cfg = R.make_config(4, 8, 32, 128, 64, 16, 524288)
+    n = R.lib().recsa_backward_scratch_bytes(ctypes.byref(cfg))
+    nodes = 4 * 8 * (8192 + 128 + 2) * 128 * 4 * 2
+    assert nodes <= n < nodes + 16 * 2 ** 20
+    bad = R.make_config(1, 8, 32, 96, 64, 16, 1024)
+    assert R.lib().recsa_backward_scratch_bytes(ctypes.byref(bad)) == 0
+    assert R.lib().recsa_decode_backward(None, None, None, None, None, None, None, None, 0, None) == R.ERR_INVALID_ARG
+    assert R.lib().recsa_tree_backward(None, None, None, None, None, 0, None) == R.ERR_INVALID_ARG
