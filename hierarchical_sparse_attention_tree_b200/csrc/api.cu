@@ -604,7 +604,7 @@ namespace {
 // the tree pass clears) then the per-call plan, logits, <dout, v> and
 // softmax statistics.
 struct BwdLayout {
-    size_t gK[MAXJ + 1], gV[MAXJ + 1], nodes_end, plan, lg, ag, st, total;
+    size_t gK[MAXJ + 1], gV[MAXJ + 1], nodes_end, plan, ubase, lg, ag, st, total;
     int E_cap;
 };
 BwdLayout bwd_layout(const recsa_config* c) {
@@ -620,6 +620,7 @@ BwdLayout bwd_layout(const recsa_config* c) {
     if (maxc < c->branching) maxc = c->branching;
     b.E_cap = (int)((l.J_cap + 1) * maxc);
     b.plan = o; o = align256(o + units * PLAN_INTS * 4);
+    b.ubase = o; o = align256(o + (units + 1) * 4);
     b.lg = o; o = align256(o + units * (size_t)b.E_cap * G * 4);
     b.ag = o; o = align256(o + units * (size_t)b.E_cap * G * 4);
     b.st = o; o = align256(o + units * G * 3 * 4);
@@ -635,6 +636,7 @@ BwdArgs bwd_args(const recsa_ctx* ctx, void* scratch) {
         a.gV[j] = reinterpret_cast<float*>(base + l.gV[j]);
     }
     a.plan = reinterpret_cast<int*>(base + l.plan);
+    a.ubase = reinterpret_cast<int*>(base + l.ubase);
     a.lg = reinterpret_cast<float*>(base + l.lg);
     a.ag = reinterpret_cast<float*>(base + l.ag);
     a.st = reinterpret_cast<float*>(base + l.st);

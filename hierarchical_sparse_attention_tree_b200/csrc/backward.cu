@@ -33,6 +33,8 @@
 // Lanes hold rotate-half pairs: lane l keeps elements l*NP .. l*NP+NP-1 of
 // each half (NP = D / 64), so every rotation is lane-local and a warp reads
 // each half of a row as one contiguous piece.
+#include <algorithm>
+
 #include "backward.cuh"
 
 namespace recsa {
@@ -41,6 +43,7 @@ constexpr int BWD_THREADS = 256;
 constexpr int BWD_WARPS = BWD_THREADS / 32;
 constexpr int BWD_ITEMS_PER_CTA = 64;  // entry kernels: candidates per CTA
 constexpr int BWD_NODES_PER_PASS = BWD_WARPS;
+constexpr int BWD_BATCH = 4;           // entries a warp has in flight at once
 __device__ __forceinline__ int* plan_off(int* pl) { return pl + 4; }
 __device__ __forceinline__ int* plan_nc(int* pl) { return pl + 4 + (MAXJ + 1); }
 
@@ -188,13 +191,6 @@ __device__ __forceinline__ bool kept(const TreeParams& p, const int* sel, int j,
     return f;
 }
 
-// Shared by the two entry kernels: the unit's plan and this warp's view of
-// the query heads and output gradients.
-struct BwdUnit {
-    int off[MAXJ + 1], nc[MAXJ + 1];
-    int J, items, valid;
-};
-
 template <typename T, int D>
 __device__ __forceinline__ const T* entry_row(const TreeParams& p, const TokenMap& tok, int j, long long u,
                                               long long m, bool value) {
@@ -220,92 +216,189 @@ __device__ __forceinline__ void rot_pairs(const float* tab, int lane, const floa
     }
 }
 
+// The unit a warp is working on: its plan (level offsets and candidate
+// counts copied to the warp's slot of shared memory), its selections and
+// this lane's pairs of its query heads and output gradients; reloaded
+// whenever the warp's item range crosses into another unit.
 template <int D, int G>
+struct UnitView {
+    long long u;
+    int ubeg, uend, J;
+    int* off;  // shared memory, MAXJ + 1 each
+    int* nc;
+    const int* sel;
+    float ql[G][D / 64], qh[G][D / 64], dl[G][D / 64], dh[G][D / 64];
+};
+
+template <typename T, int D, int G>
 __device__ __forceinline__ void load_unit(const TreeParams& p, const BwdArgs& a, long long u, int lane,
-                                          BwdUnit* su, float (*ql)[D / 64], float (*qh)[D / 64], float (*dl)[D / 64],
-                                          float (*dh)[D / 64], bool is_bf16) {
-    constexpr int NP = D / 64;
+                                          UnitView<D, G>& v) {
+    const int* pl = a.plan + u * PLAN_INTS;
+    v.u = u;
+    v.ubeg = a.ubase[u];
+    v.uend = a.ubase[u + 1];
+    v.J = pl[1];
+    v.sel = a.sel + u * p.J_cap * p.k;
+    __syncwarp();
+    for (int y = lane; y <= MAXJ; y += 32) {
+        v.off[y] = pl[4 + y];
+        v.nc[y] = pl[4 + MAXJ + 1 + y];
+    }
 #pragma unroll
     for (int g = 0; g < G; g++) {
         const long long row = (u * G + g) * D;
-        if (is_bf16) {
-            load_pairs<__nv_bfloat16, D>(reinterpret_cast<const __nv_bfloat16*>(a.q) + row, lane, ql[g], qh[g]);
-            load_pairs<__nv_bfloat16, D>(reinterpret_cast<const __nv_bfloat16*>(a.dout) + row, lane, dl[g], dh[g]);
-        } else {
-            load_pairs<float, D>(reinterpret_cast<const float*>(a.q) + row, lane, ql[g], qh[g]);
-            load_pairs<float, D>(reinterpret_cast<const float*>(a.dout) + row, lane, dl[g], dh[g]);
-        }
+        load_pairs<T, D>(reinterpret_cast<const T*>(a.q) + row, lane, v.ql[g], v.qh[g]);
+        load_pairs<T, D>(reinterpret_cast<const T*>(a.dout) + row, lane, v.dl[g], v.dh[g]);
     }
-    (void)NP;
-    (void)su;
+    __syncwarp();
 }
 
-__device__ __forceinline__ void read_plan(const BwdArgs& a, long long u, BwdUnit* su, int tid) {
-    const int* pl = a.plan + u * PLAN_INTS;
-    if (tid <= MAXJ) {
-        su->off[tid] = pl[4 + tid];
-        su->nc[tid] = pl[4 + MAXJ + 1 + tid];
+// Items xg .. xg + nb - 1 of the current unit (nb <= NI): lane t < nb works
+// out item t (level, rank, node, query position, kept or not) and the warp
+// receives all of them, so the item's row loads can all be in flight at once.
+template <int NI>
+struct Batch {
+    int j[NI], i[NI], m[NI], P[NI];  // node ids fit in int: capacity < 2^31
+    bool skip[NI];  // a kept node (not an entry), or past the batch
+};
+template <int NI, int D, int G>
+__device__ __forceinline__ void batch_items(const TreeParams& p, const UnitView<D, G>& v, int xg, int nb, int lane,
+                                            Batch<NI>& bt) {
+    int mj = 0, mi = 0, mm = 0, mP = 0, mk = 1;
+    if (lane < nb) {
+        const Item it = plan_item(p, v.sel, v.off, v.nc, v.J, xg + lane - v.ubeg);
+        mj = it.j;
+        mi = (int)it.i;
+        mm = (int)it.m;
+        mP = (int)it.P;
+        mk = it.j >= 1 && kept(p, v.sel, it.j, it.m, v.nc[it.j]);
     }
-    if (tid == 0) {
-        su->valid = pl[0];
-        su->J = pl[1];
-        su->items = pl[2];
+#pragma unroll
+    for (int t = 0; t < NI; t++) {
+        bt.j[t] = __shfl_sync(0xffffffffu, mj, t);
+        bt.i[t] = __shfl_sync(0xffffffffu, mi, t);
+        bt.m[t] = __shfl_sync(0xffffffffu, mm, t);
+        bt.P[t] = __shfl_sync(0xffffffffu, mP, t);
+        bt.skip[t] = __shfl_sync(0xffffffffu, mk, t) != 0;
     }
+}
+
+// The items of all units form one list (unit u's items at ubase[u] ..
+// ubase[u + 1]); every warp of the grid takes one contiguous slice of it,
+// so the work is balanced whatever the units' sizes.
+struct Slice {
+    int x0, x1;
+};
+__device__ __forceinline__ Slice warp_slice(const BwdArgs& a, long long units) {
+    const int total = a.ubase[units];
+    const long long warps = (long long)gridDim.x * BWD_WARPS;
+    const long long gw = (long long)blockIdx.x * BWD_WARPS + (threadIdx.x >> 5);
+    const long long per = (total + warps - 1) / warps;
+    Slice sl;
+    sl.x0 = (int)min((long long)total, gw * per);
+    sl.x1 = (int)min((long long)total, sl.x0 + per);
+    return sl;
+}
+// The unit holding global item x (binary search over ubase).
+__device__ __forceinline__ long long unit_of(const BwdArgs& a, long long units, int x) {
+    long long lo = 0, hi = units - 1;
+    while (lo < hi) {
+        const long long mid = (lo + hi + 1) >> 1;
+        if (a.ubase[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Prefix sums of the units' item counts (one CTA).
+__global__ void __launch_bounds__(1024) bwd_scan_kernel(TreeParams p, BwdArgs a) {
+    __shared__ int part[1024];
+    const long long units = (long long)p.B * p.H;
+    const int tid = threadIdx.x;
+    const long long per = (units + 1023) / 1024;
+    const long long u0 = tid * per, u1 = min(units, u0 + per);
+    int s = 0;
+    for (long long u = u0; u < u1; u++) s += a.plan[u * PLAN_INTS + 2];
+    part[tid] = s;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {  // inclusive scan
+        const int v = tid >= o ? part[tid - o] : 0;
+        __syncthreads();
+        part[tid] += v;
+        __syncthreads();
+    }
+    int base = tid ? part[tid - 1] : 0;
+    for (long long u = u0; u < u1; u++) {
+        a.ubase[u] = base;
+        base += a.plan[u * PLAN_INTS + 2];
+    }
+    if (tid == 1023) a.ubase[units] = part[1023];
 }
 
 // --------------------------------------------------- entry logits, <dout, v>
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(BWD_THREADS) bwd_score_kernel(TreeParams p, BwdArgs a) {
-    constexpr int NP = D / 64;
-    __shared__ BwdUnit su;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const long long u = blockIdx.y;
-    read_plan(a, u, &su, tid);
-    __syncthreads();
-    const int x0 = blockIdx.x * BWD_ITEMS_PER_CTA;
-    if (!su.valid || x0 >= su.items) return;
-    float ql[G][NP], qh[G][NP], dl[G][NP], dh[G][NP];
-    load_unit<D, G>(p, a, u, lane, &su, ql, qh, dl, dh, sizeof(T) == 2);
+__global__ void __launch_bounds__(BWD_THREADS, 2) bwd_score_kernel(TreeParams p, BwdArgs a) {
+    constexpr int NP = D / 64, NI = G >= 8 ? 2 : BWD_BATCH;
+    __shared__ int s_plan[BWD_WARPS][2][MAXJ + 1];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long units = (long long)p.B * p.H;
+    const Slice sl = warp_slice(a, units);
+    if (sl.x0 >= sl.x1) return;
     const TokenMap tok = token_map(p);
-    const int* sel = a.sel + u * p.J_cap * p.k;
-    const int x1 = min(x0 + BWD_ITEMS_PER_CTA, su.items);
-    for (int x = x0 + warp; x < x1; x += BWD_WARPS) {
-        const Item it = plan_item(p, sel, su.off, su.nc, su.J, x);
-        float* lgx = a.lg + (u * a.E_cap + x) * G;
-        float* agx = a.ag + (u * a.E_cap + x) * G;
-        if (it.j >= 1 && kept(p, sel, it.j, it.m, su.nc[it.j])) {
-            if (lane < G) {
-                lgx[lane] = -INFINITY;
-                agx[lane] = 0.f;
-            }
-            continue;
-        }
-        float klo[NP], khi[NP], vlo[NP], vhi[NP];
-        load_pairs<T, D>(entry_row<T, D>(p, tok, it.j, u, it.m, false), lane, klo, khi);
-        load_pairs<T, D>(entry_row<T, D>(p, tok, it.j, u, it.m, true), lane, vlo, vhi);
-        const float* tab = p.rope + (it.P - it.i) * 3 * (D / 2);
-        float lgv[G], agv[G];
+    UnitView<D, G> v;
+    v.off = s_plan[warp][0];
+    v.nc = s_plan[warp][1];
+    v.uend = 0;
+    for (int xg = sl.x0; xg < sl.x1;) {
+        if (xg >= v.uend) load_unit<T, D, G>(p, a, unit_of(a, units, xg), lane, v);
+        const long long u = v.u;
+        const int nb = min(NI, min(sl.x1, v.uend) - xg);
+        Batch<NI> bt;
+        batch_items<NI>(p, v, xg, nb, lane, bt);
+        float klo[NI][NP], khi[NI][NP], vlo[NI][NP], vhi[NI][NP];
 #pragma unroll
-        for (int g = 0; g < G; g++) {
-            float rl[NP], rh[NP];
-            rot_pairs<D>(tab, lane, ql[g], qh[g], false, rl, rh);
-            float s = 0.f, t = 0.f;
-#pragma unroll
-            for (int i = 0; i < NP; i++) {
-                s += rl[i] * klo[i] + rh[i] * khi[i];
-                t += dl[g][i] * vlo[i] + dh[g][i] * vhi[i];
+        for (int t = 0; t < NI; t++)
+            if (!bt.skip[t]) {
+                load_pairs<T, D>(entry_row<T, D>(p, tok, bt.j[t], u, bt.m[t], false), lane, klo[t], khi[t]);
+                load_pairs<T, D>(entry_row<T, D>(p, tok, bt.j[t], u, bt.m[t], true), lane, vlo[t], vhi[t]);
             }
-            lgv[g] = warp_sum(s) * p.scale;
-            agv[g] = warp_sum(t);
-        }
-        if (lane == 0) {
+#pragma unroll
+        for (int t = 0; t < NI; t++) {
+            if (t >= nb) break;
+            const int x = xg + t - v.ubeg;
+            float* lgx = a.lg + (u * a.E_cap + x) * G;
+            float* agx = a.ag + (u * a.E_cap + x) * G;
+            if (bt.skip[t]) {
+                if (lane < G) {
+                    lgx[lane] = -INFINITY;
+                    agx[lane] = 0.f;
+                }
+                continue;
+            }
+            const float* tab = p.rope + (bt.P[t] - bt.i[t]) * 3 * (D / 2);
+            float lgv[G], agv[G];
 #pragma unroll
             for (int g = 0; g < G; g++) {
-                lgx[g] = lgv[g];
-                agx[g] = agv[g];
+                float rl[NP], rh[NP];
+                rot_pairs<D>(tab, lane, v.ql[g], v.qh[g], false, rl, rh);
+                float s = 0.f, w = 0.f;
+#pragma unroll
+                for (int i = 0; i < NP; i++) {
+                    s += rl[i] * klo[t][i] + rh[i] * khi[t][i];
+                    w += v.dl[g][i] * vlo[t][i] + v.dh[g][i] * vhi[t][i];
+                }
+                lgv[g] = warp_sum(s) * p.scale;
+                agv[g] = warp_sum(w);
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int g = 0; g < G; g++) {
+                    lgx[g] = lgv[g];
+                    agx[g] = agv[g];
+                }
             }
         }
+        xg += nb;
     }
 }
 
@@ -376,149 +469,163 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_stats_kernel(TreeParams p, Bw
 
 // --------------------------------------------------- entry gradients
 
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(BWD_THREADS) bwd_entry_kernel(TreeParams p, BwdArgs a) {
+// Adds a warp's dq partial of unit u into dq and clears it.
+template <int D, int G>
+__device__ __forceinline__ void flush_dq(float* dq, long long u, int lane, float (*aql)[D / 64],
+                                         float (*aqh)[D / 64]) {
     constexpr int NP = D / 64;
-    __shared__ BwdUnit su;
-    __shared__ float dqs[BWD_WARPS][G][D];
-    __shared__ float sts[G][3];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const long long u = blockIdx.y;
-    read_plan(a, u, &su, tid);
-    if (tid < G * 3) sts[tid / 3][tid % 3] = a.st[u * G * 3 + tid];
-    __syncthreads();
-    const int x0 = blockIdx.x * BWD_ITEMS_PER_CTA;
-    if (!su.valid || x0 >= su.items) return;
-    float ql[G][NP], qh[G][NP], dl[G][NP], dh[G][NP];
-    load_unit<D, G>(p, a, u, lane, &su, ql, qh, dl, dh, sizeof(T) == 2);
-    float aql[G][NP], aqh[G][NP];  // this warp's dq partial
+#pragma unroll
+    for (int g = 0; g < G; g++) {
+        float* row = dq + (u * G + g) * D;
+#pragma unroll
+        for (int i = 0; i < NP; i++) {
+            if (aql[g][i] != 0.f) atomicAdd(row + lane * NP + i, aql[g][i]);
+            if (aqh[g][i] != 0.f) atomicAdd(row + D / 2 + lane * NP + i, aqh[g][i]);
+            aql[g][i] = aqh[g][i] = 0.f;
+        }
+    }
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(BWD_THREADS, 2) bwd_entry_kernel(TreeParams p, BwdArgs a) {
+    constexpr int NP = D / 64, NI = G >= 8 ? 1 : BWD_BATCH;
+    __shared__ int s_plan[BWD_WARPS][2][MAXJ + 1];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long units = (long long)p.B * p.H;
+    const Slice sl = warp_slice(a, units);
+    if (sl.x0 >= sl.x1) return;
+    const TokenMap tok = token_map(p);
+    UnitView<D, G> v;
+    v.off = s_plan[warp][0];
+    v.nc = s_plan[warp][1];
+    v.uend = 0;
+    v.u = -1;
+    float st[G][3];
+    float aql[G][NP], aqh[G][NP];  // this warp's dq partial of unit v.u
 #pragma unroll
     for (int g = 0; g < G; g++)
 #pragma unroll
         for (int i = 0; i < NP; i++) aql[g][i] = aqh[g][i] = 0.f;
-    const TokenMap tok = token_map(p);
-    const int* sel = a.sel + u * p.J_cap * p.k;
-    const int x1 = min(x0 + BWD_ITEMS_PER_CTA, su.items);
-    for (int x = x0 + warp; x < x1; x += BWD_WARPS) {
-        const float* lgx = a.lg + (u * a.E_cap + x) * G;
-        const float* agx = a.ag + (u * a.E_cap + x) * G;
-        float pg[G], dlg[G];
-        bool any = false;
+    for (int xg = sl.x0; xg < sl.x1;) {
+        if (xg >= v.uend) {
+            if (v.u >= 0) flush_dq<D, G>(a.dq, v.u, lane, aql, aqh);
+            load_unit<T, D, G>(p, a, unit_of(a, units, xg), lane, v);
 #pragma unroll
-        for (int g = 0; g < G; g++) {
-            const float l = lgx[g];
-            pg[g] = l == -INFINITY ? 0.f : expf(l - sts[g][0]) / sts[g][1];
-            dlg[g] = pg[g] * (agx[g] - sts[g][2]);
-            any |= l != -INFINITY;
+            for (int g = 0; g < G; g++)
+#pragma unroll
+                for (int c = 0; c < 3; c++) st[g][c] = a.st[(v.u * G + g) * 3 + c];
         }
-        if (!any) continue;  // a kept node: not an entry
-        const Item it = plan_item(p, sel, su.off, su.nc, su.J, x);
-        float klo[NP], khi[NP];
-        load_pairs<T, D>(entry_row<T, D>(p, tok, it.j, u, it.m, false), lane, klo, khi);
-        const float* tab = p.rope + (it.P - it.i) * 3 * (D / 2);
-        float gkl[NP], gkh[NP], gvl[NP], gvh[NP], rkl[NP], rkh[NP];
+        const long long u = v.u;
+        const int nb = min(NI, min(sl.x1, v.uend) - xg);
+        Batch<NI> bt;
+        batch_items<NI>(p, v, xg, nb, lane, bt);
+        float klo[NI][NP], khi[NI][NP], lgt[NI][G], agt[NI][G];
 #pragma unroll
-        for (int i = 0; i < NP; i++) gkl[i] = gkh[i] = gvl[i] = gvh[i] = 0.f;
-        rot_pairs<D>(tab, lane, klo, khi, true, rkl, rkh);  // R(i - P) k
+        for (int t = 0; t < NI; t++)
+            if (!bt.skip[t]) {
+                const int x = xg + t - v.ubeg;
+                load_pairs<T, D>(entry_row<T, D>(p, tok, bt.j[t], u, bt.m[t], false), lane, klo[t], khi[t]);
 #pragma unroll
-        for (int g = 0; g < G; g++) {
-            float rl[NP], rh[NP];
-            rot_pairs<D>(tab, lane, ql[g], qh[g], false, rl, rh);  // R(P - i) q
-            const float c = dlg[g] * p.scale;
-#pragma unroll
-            for (int i = 0; i < NP; i++) {
-                gkl[i] += c * rl[i];
-                gkh[i] += c * rh[i];
-                gvl[i] += pg[g] * dl[g][i];
-                gvh[i] += pg[g] * dh[g][i];
-                aql[g][i] += c * rkl[i];
-                aqh[g][i] += c * rkh[i];
+                for (int g = 0; g < G; g++) {
+                    lgt[t][g] = a.lg[(u * a.E_cap + x) * G + g];
+                    agt[t][g] = a.ag[(u * a.E_cap + x) * G + g];
+                }
             }
+#pragma unroll
+        for (int t = 0; t < NI; t++) {
+            if (bt.skip[t]) continue;
+            float pg[G], dlg[G];
+#pragma unroll
+            for (int g = 0; g < G; g++) {
+                pg[g] = expf(lgt[t][g] - st[g][0]) / st[g][1];
+                dlg[g] = pg[g] * (agt[t][g] - st[g][2]);
+            }
+            const float* tab = p.rope + (bt.P[t] - bt.i[t]) * 3 * (D / 2);
+            float gkl[NP], gkh[NP], gvl[NP], gvh[NP], rkl[NP], rkh[NP];
+#pragma unroll
+            for (int i = 0; i < NP; i++) gkl[i] = gkh[i] = gvl[i] = gvh[i] = 0.f;
+            rot_pairs<D>(tab, lane, klo[t], khi[t], true, rkl, rkh);  // R(i - P) k
+#pragma unroll
+            for (int g = 0; g < G; g++) {
+                float rl[NP], rh[NP];
+                rot_pairs<D>(tab, lane, v.ql[g], v.qh[g], false, rl, rh);  // R(P - i) q
+                const float c = dlg[g] * p.scale;
+#pragma unroll
+                for (int i = 0; i < NP; i++) {
+                    gkl[i] += c * rl[i];
+                    gkh[i] += c * rh[i];
+                    gvl[i] += pg[g] * v.dl[g][i];
+                    gvh[i] += pg[g] * v.dh[g][i];
+                    aql[g][i] += c * rkl[i];
+                    aqh[g][i] += c * rkh[i];
+                }
+            }
+            float* rk;
+            float* rv;
+            if (bt.j[t] >= 1) {
+                rk = a.gK[bt.j[t]] + (u * p.rows[bt.j[t]] + bt.m[t]) * D;
+                rv = a.gV[bt.j[t]] + (u * p.rows[bt.j[t]] + bt.m[t]) * D;
+            } else {
+                const long long row = token_row(tok, u, bt.m[t]);
+                rk = a.dk + row * D;
+                rv = a.dv + row * D;
+            }
+            add_pairs<D>(rk, lane, gkl, gkh);
+            add_pairs<D>(rv, lane, gvl, gvh);
         }
-        float* rk;
-        float* rv;
-        if (it.j >= 1) {
-            rk = a.gK[it.j] + (u * p.rows[it.j] + it.m) * D;
-            rv = a.gV[it.j] + (u * p.rows[it.j] + it.m) * D;
-        } else {
-            const long long row = token_row(tok, u, it.m);
-            rk = a.dk + row * D;
-            rv = a.dv + row * D;
-        }
-        add_pairs<D>(rk, lane, gkl, gkh);
-        add_pairs<D>(rv, lane, gvl, gvh);
+        xg += nb;
     }
-    // dq: this CTA's partial, summed over its warps, added once per element
-#pragma unroll
-    for (int g = 0; g < G; g++)
-#pragma unroll
-        for (int i = 0; i < NP; i++) {
-            dqs[warp][g][lane * NP + i] = aql[g][i];
-            dqs[warp][g][D / 2 + lane * NP + i] = aqh[g][i];
-        }
-    __syncthreads();
-    for (int e = tid; e < G * D; e += BWD_THREADS) {
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < BWD_WARPS; w++) s += dqs[w][e / D][e % D];
-        atomicAdd(a.dq + u * G * D + e, s);
-    }
+    if (v.u >= 0) flush_dq<D, G>(a.dq, v.u, lane, aql, aqh);
 }
 
 // ------------------------------------------------------- propagation
 
-// Shared memory of the propagation kernels: W (fp32, W[r][c] at r * D + c)
-// and the staged (g, mean) pairs of one pass of nodes.
-template <int D>
+// Shared memory of the propagation kernel: W in the storage type (W[r][c]
+// at r * D + c), this CTA's dW partial (fp32, [D][D]) and the staged
+// (g, mean) rows of one pass of nodes.
+template <typename T, int D>
 struct PropSmem {
-    float W[D * D];
+    float dw[D * D];
     float g[BWD_NODES_PER_PASS][D];
     float mean[BWD_NODES_PER_PASS][D];
+    T W[D * D];
 };
 
-// Each thread owns D*D/256 consecutive elements of one row of dW:
-// row r = tid % D, columns [cb * CW, (cb + 1) * CW) with cb = tid / D.
-template <int D>
-__device__ __forceinline__ void accumulate_dw(const PropSmem<D>& sm, int tid, float* acc) {
-    constexpr int CW = D * D / BWD_THREADS;
-    const int r = tid % D, cb = tid / D;
-#pragma unroll 1
-    for (int w = 0; w < BWD_NODES_PER_PASS; w++) {
-        const float gr = sm.g[w][r];
-        if (gr == 0.f) continue;
-        const float4* mrow = reinterpret_cast<const float4*>(&sm.mean[w][cb * CW]);
-#pragma unroll
-        for (int c = 0; c < CW / 4; c++) {
-            const float4 mv = mrow[c];
-            acc[4 * c] += gr * mv.x;
-            acc[4 * c + 1] += gr * mv.y;
-            acc[4 * c + 2] += gr * mv.z;
-            acc[4 * c + 3] += gr * mv.w;
-        }
-    }
-}
-
-template <int D>
-__device__ __forceinline__ void flush_dw(float* dw, int tid, const float* acc) {
-    constexpr int CW = D * D / BWD_THREADS;
-    const int r = tid % D, cb = tid / D;
-#pragma unroll
-    for (int c = 0; c < CW; c++)
-        if (acc[c] != 0.f) atomicAdd(dw + r * D + cb * CW + c, acc[c]);
-}
-
+// Each thread owns D*D/256 consecutive elements of one row of dW: row
+// r = tid % D, columns [cb * CW, (cb + 1) * CW) with cb = tid / D. The
+// partial stays in shared memory between passes; a pass adds the outer
+// products of its staged rows.
 template <typename T, int D>
-__device__ __forceinline__ void load_w(const TreeParams& p, PropSmem<D>& sm, int tid) {
-    const T* wt = reinterpret_cast<const T*>(p.Wt);  // Wt[c * D + r] = W[r][c]
-    for (int i = tid; i < D * D; i += BWD_THREADS) {
-        const int c = i / D, r = i % D;
-        sm.W[r * D + c] = to_f(wt[i]);
+__device__ __forceinline__ void accumulate_dw(PropSmem<T, D>& sm, int tid) {
+    constexpr int CW = D * D / BWD_THREADS;
+    const int r = tid % D, cb = tid / D;
+    float gr[BWD_NODES_PER_PASS];
+    bool any = false;
+#pragma unroll
+    for (int w = 0; w < BWD_NODES_PER_PASS; w++) {
+        gr[w] = sm.g[w][r];
+        any |= gr[w] != 0.f;
+    }
+    if (!any) return;
+    float4* dst = reinterpret_cast<float4*>(&sm.dw[r * D + cb * CW]);
+#pragma unroll 4
+    for (int c = 0; c < CW / 4; c++) {
+        float4 acc = dst[c];
+#pragma unroll
+        for (int w = 0; w < BWD_NODES_PER_PASS; w++) {
+            const float4 mv = reinterpret_cast<const float4*>(&sm.mean[w][cb * CW])[c];
+            acc.x += gr[w] * mv.x;
+            acc.y += gr[w] * mv.y;
+            acc.z += gr[w] * mv.z;
+            acc.w += gr[w] * mv.w;
+        }
+        dst[c] = acc;
     }
 }
 
 // h = W^T g / n on this lane's pairs; g is the warp's staged row.
-template <int D>
-__device__ __forceinline__ void wt_times(const PropSmem<D>& sm, const float* g, int lane, float inv_n, float* hlo,
+template <typename T, int D>
+__device__ __forceinline__ void wt_times(const PropSmem<T, D>& sm, const float* g, int lane, float inv_n, float* hlo,
                                          float* hhi) {
     constexpr int NP = D / 64;
 #pragma unroll
@@ -526,10 +633,12 @@ __device__ __forceinline__ void wt_times(const PropSmem<D>& sm, const float* g, 
 #pragma unroll 4
     for (int r = 0; r < D; r++) {
         const float gr = g[r];
+        float wl[NP], wh[NP];
+        load_pairs<T, D>(sm.W + r * D, lane, wl, wh);
 #pragma unroll
         for (int i = 0; i < NP; i++) {
-            hlo[i] += sm.W[r * D + lane * NP + i] * gr;
-            hhi[i] += sm.W[r * D + D / 2 + lane * NP + i] * gr;
+            hlo[i] += wl[i] * gr;
+            hhi[i] += wh[i] * gr;
         }
     }
 #pragma unroll
@@ -539,40 +648,43 @@ __device__ __forceinline__ void wt_times(const PropSmem<D>& sm, const float* g, 
     }
 }
 
-// Level j (1..J_cap): one warp per node, BWD_NODES_PER_PASS nodes per pass,
-// `passes` passes per CTA. At level 1 the warp also adds h and s into the
-// gradients of the node's tokens.
+// Level j (1..J_cap), persistent: the grid walks chunks of
+// BWD_NODES_PER_PASS consecutive nodes of one unit (one node per warp) with
+// a grid stride. Per node: g = acc_K + parent h, s = acc_V / tokens + parent
+// s, h = W^T g / children, and the mean of the stored child keys (for dW).
+// Level j > 1 writes h and s in place for the level below; level 1 adds them
+// into the node's tokens' dk and dv in the same pass that reads the tokens'
+// keys for the mean.
 template <typename T, int D>
-__global__ void __launch_bounds__(BWD_THREADS) bwd_prop_kernel(TreeParams p, BwdArgs a, int j, int passes) {
+__global__ void __launch_bounds__(BWD_THREADS, 2)
+    bwd_prop_kernel(TreeParams p, BwdArgs a, int j, long long chunks_per_unit) {
     constexpr int NP = D / 64;
-    constexpr int CW = D * D / BWD_THREADS;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    PropSmem<D>& sm = *reinterpret_cast<PropSmem<D>*>(smem_raw);
+    PropSmem<T, D>& sm = *reinterpret_cast<PropSmem<T, D>*>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const long long u = blockIdx.y;
-    const long long L = p.len[u];
-    const long long nj = L >= 1 ? level_rows(p, j, L) : 0;
-    const long long m_first = (long long)blockIdx.x * passes * BWD_NODES_PER_PASS;
-    if (m_first >= nj) return;
-    load_w<T, D>(p, sm, tid);
-    float acc[CW];
-#pragma unroll
-    for (int c = 0; c < CW; c++) acc[c] = 0.f;
+    {
+        const T* wt = reinterpret_cast<const T*>(p.Wt);  // Wt[c * D + r] = W[r][c]
+        for (int i = tid; i < D * D; i += BWD_THREADS) {
+            sm.W[(i % D) * D + i / D] = wt[i];
+            sm.dw[i] = 0.f;
+        }
+    }
     const TokenMap tok = token_map(p);
     const bool top = j == p.J_cap;
-    for (int pass = 0; pass < passes; pass++) {
-        const long long m = m_first + (long long)pass * BWD_NODES_PER_PASS + warp;
-        __syncthreads();  // W loaded / the previous pass's rows consumed
-        float glo[NP], ghi[NP], slo[NP], shi[NP], mlo[NP], mhi[NP];
+    const long long total = (long long)p.B * p.H * chunks_per_unit;
+    for (long long ch = blockIdx.x; ch < total; ch += gridDim.x) {
+        const long long u = ch / chunks_per_unit;
+        const long long m = (ch % chunks_per_unit) * BWD_NODES_PER_PASS + warp;
+        const long long L = p.len[u];
+        const bool live = L >= 1 && m < level_rows(p, j, L);
+        __syncthreads();  // W loaded / the previous pass's staged rows consumed
+        float glo[NP], ghi[NP], slo[NP], shi[NP];
 #pragma unroll
-        for (int i = 0; i < NP; i++) glo[i] = ghi[i] = slo[i] = shi[i] = mlo[i] = mhi[i] = 0.f;
-        long long nch = 0;
-        const bool live = m < nj;
+        for (int i = 0; i < NP; i++) glo[i] = ghi[i] = slo[i] = shi[i] = 0.f;
+        long long nch = 1;
         if (live) {
-            float* gk = a.gK[j] + (u * p.rows[j] + m) * D;
-            float* gv = a.gV[j] + (u * p.rows[j] + m) * D;
-            load_pairs<float, D>(gk, lane, glo, ghi);
-            load_pairs<float, D>(gv, lane, slo, shi);
+            load_pairs<float, D>(a.gK[j] + (u * p.rows[j] + m) * D, lane, glo, ghi);
+            load_pairs<float, D>(a.gV[j] + (u * p.rows[j] + m) * D, lane, slo, shi);
             const float inv_t = 1.f / (float)n_tokens(p, j, m, L);
 #pragma unroll
             for (int i = 0; i < NP; i++) {
@@ -580,10 +692,10 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_prop_kernel(TreeParams p, Bwd
                 shi[i] *= inv_t;
             }
             if (!top) {  // the parent's h and s (already propagated)
-                const long long par = u * p.rows[j + 1] + m / p.b;
+                const long long par = (u * p.rows[j + 1] + m / p.b) * D;
                 float hl[NP], hh[NP], sl[NP], sh[NP];
-                load_pairs<float, D>(a.gK[j + 1] + par * D, lane, hl, hh);
-                load_pairs<float, D>(a.gV[j + 1] + par * D, lane, sl, sh);
+                load_pairs<float, D>(a.gK[j + 1] + par, lane, hl, hh);
+                load_pairs<float, D>(a.gV[j + 1] + par, lane, sl, sh);
 #pragma unroll
                 for (int i = 0; i < NP; i++) {
                     glo[i] += hl[i];
@@ -593,17 +705,72 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_prop_kernel(TreeParams p, Bwd
                 }
             }
             nch = n_children(p, j, m, L);
-            // mean of the stored child keys
-#pragma unroll 8
-            for (long long c = 0; c < nch; c++) {
-                float kl[NP], kh[NP];
-                const T* row = j == 1 ? reinterpret_cast<const T*>(p.K[0]) + token_row(tok, u, m * p.b + c) * D
-                                      : reinterpret_cast<const T*>(p.K[j - 1]) + (u * p.rows[j - 1] + m * p.b + c) * D;
-                load_pairs<T, D>(row, lane, kl, kh);
+        }
+        store_pairs<D>(sm.g[warp], lane, glo, ghi);
+        __syncwarp();
+        float mlo[NP], mhi[NP];
 #pragma unroll
-                for (int i = 0; i < NP; i++) {
-                    mlo[i] += kl[i];
-                    mhi[i] += kh[i];
+        for (int i = 0; i < NP; i++) mlo[i] = mhi[i] = 0.f;
+        if (live) {
+            float hlo[NP], hhi[NP];
+            wt_times<T, D>(sm, sm.g[warp], lane, 1.f / (float)nch, hlo, hhi);
+            if (j > 1) {
+                // mean of the stored child keys, then h and s in place for the children
+                const T* kb = reinterpret_cast<const T*>(p.K[j - 1]) + (u * p.rows[j - 1] + m * p.b) * D;
+#pragma unroll 8
+                for (long long c = 0; c < nch; c++) {
+                    float kl[NP], kh[NP];
+                    load_pairs<T, D>(kb + c * D, lane, kl, kh);
+#pragma unroll
+                    for (int i = 0; i < NP; i++) {
+                        mlo[i] += kl[i];
+                        mhi[i] += kh[i];
+                    }
+                }
+                store_pairs<D>(a.gK[j] + (u * p.rows[j] + m) * D, lane, hlo, hhi);
+                store_pairs<D>(a.gV[j] + (u * p.rows[j] + m) * D, lane, slo, shi);
+            } else {
+                // the node's tokens (contiguous rows: a node never straddles
+                // a page): their keys for the mean, dk += h, dv += s
+                const long long row0 = token_row(tok, u, m * p.b);
+                const T* kb = reinterpret_cast<const T*>(p.K[0]) + row0 * D;
+                float* dkb = a.dk + row0 * D;
+                float* dvb = a.dv + row0 * D;
+                constexpr int U = 4;  // rows in flight per lane and array
+                long long c = 0;
+                for (; c + U <= nch; c += U) {
+                    float kl[U][NP], kh[U][NP], xl[U][NP], xh[U][NP], yl[U][NP], yh[U][NP];
+#pragma unroll
+                    for (int x = 0; x < U; x++) {
+                        load_pairs<T, D>(kb + (c + x) * D, lane, kl[x], kh[x]);
+                        load_pairs<float, D>(dkb + (c + x) * D, lane, xl[x], xh[x]);
+                        load_pairs<float, D>(dvb + (c + x) * D, lane, yl[x], yh[x]);
+                    }
+#pragma unroll
+                    for (int x = 0; x < U; x++) {
+#pragma unroll
+                        for (int i = 0; i < NP; i++) {
+                            mlo[i] += kl[x][i];
+                            mhi[i] += kh[x][i];
+                            xl[x][i] += hlo[i];
+                            xh[x][i] += hhi[i];
+                            yl[x][i] += slo[i];
+                            yh[x][i] += shi[i];
+                        }
+                        store_pairs<D>(dkb + (c + x) * D, lane, xl[x], xh[x]);
+                        store_pairs<D>(dvb + (c + x) * D, lane, yl[x], yh[x]);
+                    }
+                }
+                for (; c < nch; c++) {
+                    float kl[NP], kh[NP];
+                    load_pairs<T, D>(kb + c * D, lane, kl, kh);
+#pragma unroll
+                    for (int i = 0; i < NP; i++) {
+                        mlo[i] += kl[i];
+                        mhi[i] += kh[i];
+                    }
+                    add_pairs<D>(dkb + c * D, lane, hlo, hhi);
+                    add_pairs<D>(dvb + c * D, lane, slo, shi);
                 }
             }
             const float inv_c = 1.f / (float)nch;
@@ -613,70 +780,35 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_prop_kernel(TreeParams p, Bwd
                 mhi[i] *= inv_c;
             }
         }
-#pragma unroll
-        for (int i = 0; i < NP; i++) {
-            sm.g[warp][lane * NP + i] = glo[i];
-            sm.g[warp][D / 2 + lane * NP + i] = ghi[i];
-            sm.mean[warp][lane * NP + i] = mlo[i];
-            sm.mean[warp][D / 2 + lane * NP + i] = mhi[i];
-        }
-        __syncwarp();
-        if (live) {
-            float hlo[NP], hhi[NP];
-            wt_times<D>(sm, sm.g[warp], lane, 1.f / (float)nch, hlo, hhi);
-            if (j > 1) {  // in place: the children read h and s
-                float* gk = a.gK[j] + (u * p.rows[j] + m) * D;
-                float* gv = a.gV[j] + (u * p.rows[j] + m) * D;
-                store_pairs<D>(gk, lane, hlo, hhi);
-                store_pairs<D>(gv, lane, slo, shi);
-            } else {  // the node's tokens (contiguous rows: a node never straddles a page)
-                const long long row0 = token_row(tok, u, m * p.b);
-                constexpr int U = 4;  // rows in flight per lane and array
-                long long c = 0;
-                for (; c + U <= nch; c += U) {
-                    float kl[U][NP], kh[U][NP], vl[U][NP], vh[U][NP];
-#pragma unroll
-                    for (int x = 0; x < U; x++) {
-                        load_pairs<float, D>(a.dk + (row0 + c + x) * D, lane, kl[x], kh[x]);
-                        load_pairs<float, D>(a.dv + (row0 + c + x) * D, lane, vl[x], vh[x]);
-                    }
-#pragma unroll
-                    for (int x = 0; x < U; x++) {
-#pragma unroll
-                        for (int i = 0; i < NP; i++) {
-                            kl[x][i] += hlo[i];
-                            kh[x][i] += hhi[i];
-                            vl[x][i] += slo[i];
-                            vh[x][i] += shi[i];
-                        }
-                        store_pairs<D>(a.dk + (row0 + c + x) * D, lane, kl[x], kh[x]);
-                        store_pairs<D>(a.dv + (row0 + c + x) * D, lane, vl[x], vh[x]);
-                    }
-                }
-                for (; c < nch; c++) {
-                    add_pairs<D>(a.dk + (row0 + c) * D, lane, hlo, hhi);
-                    add_pairs<D>(a.dv + (row0 + c) * D, lane, slo, shi);
-                }
-            }
-        }
+        store_pairs<D>(sm.mean[warp], lane, mlo, mhi);
         __syncthreads();
-        accumulate_dw<D>(sm, tid, acc);
+        accumulate_dw<T, D>(sm, tid);
     }
-    flush_dw<D>(a.dw, tid, acc);
+    __syncthreads();
+    for (int i = tid; i < D * D; i += BWD_THREADS)
+        if (sm.dw[i] != 0.f) atomicAdd(a.dw + i, sm.dw[i]);
 }
 
 // ---------------------------------------------------------------- host
 
-size_t bwd_prop_smem(int D) { return D == 64 ? sizeof(PropSmem<64>) : sizeof(PropSmem<128>); }
-
 template <typename T, int D, int G>
 cudaError_t launch_decode_backward(const TreeParams& p, const BwdArgs& a, cudaStream_t s) {
     const long long units = (long long)p.B * p.H;
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     bwd_plan_kernel<<<(unsigned)((units + 3) / 4), 128, 0, s>>>(p, a);
-    const dim3 grid((unsigned)((a.E_cap + BWD_ITEMS_PER_CTA - 1) / BWD_ITEMS_PER_CTA), (unsigned)units);
-    bwd_score_kernel<T, D, G><<<grid, BWD_THREADS, 0, s>>>(p, a);
+    bwd_scan_kernel<<<1, 1024, 0, s>>>(p, a);
+    // one wave of resident CTAs (no more warps than items at the cap)
+    auto grid_for = [&](auto kern) {
+        int per_sm = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, BWD_THREADS, 0) != cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        const long long need = (units * a.E_cap + BWD_WARPS - 1) / BWD_WARPS;
+        return (unsigned)std::max(1LL, std::min(need, (long long)sms * per_sm));
+    };
+    bwd_score_kernel<T, D, G><<<grid_for(bwd_score_kernel<T, D, G>), BWD_THREADS, 0, s>>>(p, a);
     bwd_stats_kernel<D, G><<<(unsigned)units, BWD_THREADS, 0, s>>>(p, a);
-    bwd_entry_kernel<T, D, G><<<grid, BWD_THREADS, 0, s>>>(p, a);
+    bwd_entry_kernel<T, D, G><<<grid_for(bwd_entry_kernel<T, D, G>), BWD_THREADS, 0, s>>>(p, a);
     return cudaGetLastError();
 }
 
@@ -684,26 +816,21 @@ cudaError_t launch_decode_backward(const TreeParams& p, const BwdArgs& a, cudaSt
 template <typename T, int D>
 cudaError_t launch_tree_backward(const TreeParams& p, const BwdArgs& a, long long max_len, cudaStream_t s) {
     const long long units = (long long)p.B * p.H;
-    const size_t smem = sizeof(PropSmem<D>);
+    const size_t smem = sizeof(PropSmem<T, D>);
+    auto kern = bwd_prop_kernel<T, D>;
     static std::atomic<unsigned long long> attr_done{0};
-    cudaError_t e = set_smem_limit(bwd_prop_kernel<T, D>, (int)smem, attr_done);
+    cudaError_t e = set_smem_limit(kern, (int)smem, attr_done);
     if (e != cudaSuccess) return e;
-    int sms = 148;
-    {
-        int dev = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    }
-    const long long target = (long long)sms * 6;  // about two waves of three resident CTAs per SM
+    int sms = 148, dev = 0, per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, BWD_THREADS, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
     for (int j = p.J_cap; j >= 1; j--) {
         const long long nodes = (max_len + p.span[j] - 1) / p.span[j];
-        // enough nodes per CTA that the dW partials are flushed by about `target` CTAs
-        long long passes = (nodes * units + target * BWD_NODES_PER_PASS - 1) / (target * BWD_NODES_PER_PASS);
-        const long long most = (nodes + BWD_NODES_PER_PASS - 1) / BWD_NODES_PER_PASS;
-        if (passes > most) passes = most;
-        if (passes < 1) passes = 1;
-        const long long per = passes * BWD_NODES_PER_PASS;
-        const dim3 grid((unsigned)((nodes + per - 1) / per), (unsigned)units);
-        bwd_prop_kernel<T, D><<<grid, BWD_THREADS, smem, s>>>(p, a, j, (int)passes);
+        const long long chunks = (nodes + BWD_NODES_PER_PASS - 1) / BWD_NODES_PER_PASS;
+        const long long grid = std::max(1LL, std::min(chunks * units, (long long)sms * per_sm));
+        kern<<<(unsigned)grid, BWD_THREADS, smem, s>>>(p, a, j, chunks);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

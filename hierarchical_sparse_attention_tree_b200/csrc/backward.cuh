@@ -19,6 +19,7 @@ struct BwdArgs {
     float* gK[MAXJ + 1];  // node-key gradient accumulators [B*H][rows[j]][D] (j >= 1)
     float* gV[MAXJ + 1];  // node-value gradient accumulators
     int* plan;         // [B*H][PLAN_INTS]
+    int* ubase;        // [B*H + 1] first item of each unit in the list of all units' items
     float* lg;         // [B*H][E_cap][G] logits (-inf: not an entry)
     float* ag;         // [B*H][E_cap][G] <dout_g, v_e>
     float* st;         // [B*H][G][3] softmax maximum, denominator, sum_e p_e <dout, v_e>
