@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--prefill-workload", default="prefill_524k")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the chunked prefill (profiling): no decode, no baselines")
@@ -381,15 +382,99 @@ def measure_prefill(wname, dev, flush, peaks, last_chunks=0, with_dense=True):
     return res
 
 
-def mapped_ptr(t: torch.Tensor) -> int:
-    """Device address of a pinned host tensor (host memory mapped into the
-    device's address space): kernels read and write it over the bus."""
-    from cuda.bindings import runtime as rt
+def measure_backward(layer, w, q, dev, flush, peaks, kv_host, cpu_threads, with_cpu):
+    """Gradients of one decode query per sequence over the layer's current
+    tree (recsa_decode_backward, then recsa_tree_backward), each timed with
+    CUDA events over 10 runs (L2 flushed before each), with the propagation's
+    HBM roofline; and the fp64 oracle's gradient of one query per unit on a
+    sample of units, on the host cores."""
+    B, H, Hq, D, G = w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim, w.group
+    es = 2
+    stream = torch.cuda.current_stream(dev)
+    J_cap, _ = layer.tree_shape()
+    sel = torch.full((B, H, J_cap, w.k), -1, dtype=torch.int32, device=dev)
+    layer.decode(q, sel_out=sel)
+    _, _, v_rows = layer.query_stats()
+    dout = torch.from_numpy(synth.plain(91, 0, (B, Hq, D), 0.0, 1.0, True)).view(torch.bfloat16).to(dev)
+    layer.zero_grad()
+    dq = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    for _ in range(3):
+        layer.decode_backward(q, dout, sel, dq)
+        layer.tree_backward()
+    t_dec, t_tree = [], []
+    for _ in range(10):
+        for fn, acc in ((lambda: layer.decode_backward(q, dout, sel, dq), t_dec), (layer.tree_backward, t_tree)):
+            flush.fill_(7.0)
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b_.record(stream)
+            torch.cuda.synchronize(dev)
+            acc.append(a.elapsed_time(b_))
+    layer.check()
+    lengths = layer.lengths()
+    b = w.branching
+    # propagation: every token's key read and dk, dv read-modify-written
+    # (fp32); per level the node accumulators read, the inner levels' h and
+    # s written and their children's keys read; the accumulators cleared
+    tree_bytes = 0
+    for L in lengths:
+        tree_bytes += H * L * (D * es + 4 * D * 4)
+        for j in range(1, J_cap + 1):
+            nj = -(-L // b ** j)
+            tree_bytes += H * nj * 2 * D * 4 * 2  # accumulators read + cleared
+            if j >= 2:
+                tree_bytes += H * (nj * 2 * D * 4 + (-(-L // b ** (j - 1))) * D * es)
+    entries = int(sum(v_rows))
+    dec_bytes = entries * (2 * D * es + 4 * D * 4) + B * Hq * D * (2 * es + 4)
+    hbm = float(peaks["hbm_gbs"])
+    dec_ms, tree_ms = statistics.median(t_dec), statistics.median(t_tree)
+    res = {"decode_backward_us": dec_ms * 1e3, "tree_backward_ms": tree_ms,
+           "queries": B * Hq, "entries": entries,
+           "roofline": {"kernel": "bwd_prop_kernel (all levels)", "bound": "hbm",
+                        "achieved": tree_bytes / (tree_ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
+                        "frac": tree_bytes / (tree_ms / 1e3) / 1e9 / hbm, "algorithmic_bytes": tree_bytes,
+                        "traffic": kernel_traffic("bwd_prop_kernel", w.name)},
+           "entry_gbs": dec_bytes / (dec_ms / 1e3) / 1e9,
+           "how": "one decode query per sequence (its selections from recsa_decode), dout ~ N(0,1) bf16; "
+                  "recsa_decode_backward and recsa_tree_backward timed separately, median of 10, L2 flushed"}
+    del layer.dk, layer.dv, layer.dw, layer._bwd_scratch
+    layer.dk = None
+    torch.cuda.empty_cache()
+    if with_cpu:
+        import oracle
 
-    err, dptr = rt.cudaHostGetDevicePointer(t.data_ptr(), 0)
-    if int(err) != 0:
-        raise RuntimeError(f"cudaHostGetDevicePointer: {err}")
-    return int(dptr)
+        L0 = w.length
+        units = [(bb, h) for bb in range(B) for h in range(H)][:max(1, min(cpu_threads, B * H))]
+        Wf = synth.as_f32(synth.workload_pooler(w))
+        storage = oracle.STORE_BF16
+        pool = oracle.pool(len(units))
+        qh = q.view(torch.int16).cpu().numpy()
+        dh = dout.float().cpu().numpy().astype(np.float64)
+
+        def prep(bh):
+            bb, h = bh
+            tr = oracle.Tree(D, b, L0, storage).build(kv_host[0][bb, h], kv_host[1][bb, h], L0, Wf)
+            return tr
+
+        trees = list(pool.map(prep, units))
+
+        def grad(i):
+            bb, h = units[i]
+            qu = synth.as_f32(np.ascontiguousarray(qh[bb, h * G:(h + 1) * G]))
+            return oracle.query_grad(trees[i].K, trees[i].V, kv_host[0][bb, h], kv_host[1][bb, h], L0, qu,
+                                     dh[bb, h * G:(h + 1) * G], Wf, D, b, w.k, G, w.rope_base)
+
+        t0 = time.perf_counter()
+        list(pool.map(grad, range(len(units))))
+        dt = time.perf_counter() - t0
+        pool.shutdown()
+        res["cpu_baseline"] = {"value": len(units) * G / dt, "unit": "query-gradients/s", "cores": len(units),
+                               "kind": "oracle",
+                               "sample": f"oracle.query_grad of one query per unit on {len(units)} units "
+                                         f"(L = {L0}) in parallel, trees built before timing"}
+        res["gpu_query_gradients_s"] = B * Hq / ((dec_ms + tree_ms) / 1e3)
+    return res
 
 
 # -------------------------------------------------------------------- main
@@ -422,7 +507,7 @@ def main():
     B, H, Hq, D = w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim
     L0 = w.length
     W_, K_ = args.warmup, args.steps
-    n_total = 2 * (W_ + K_) + 25
+    n_total = 2 * W_ + 3 * K_ + 30  # decode steps, split and append steps, e2e loops
     cap = L0 + n_total
     seq_off = rank_sequences(rank, B)
     bf = torch.bfloat16
@@ -558,47 +643,85 @@ def main():
     achieved = dec_bytes_per_launch / dec_avg_s / 1e9
 
     # ---- end to end through the public API: every step's q, k_new, v_new
-    # arrive as one pinned host record, cross in one copy and are read in
-    # place; the output is copied back to pinned host memory; both copies
-    # are inside the step's events
+    # arrive as one pinned host record and cross in one copy; the output goes
+    # back to pinned host memory. Double-buffered: step s+1's record uploads
+    # on a side stream while step s's kernel runs, and step s's output copies
+    # back on a third stream. Timed from the first upload to the last
+    # download (events on the compute stream, which waits for the others),
+    # with no L2 flush between steps (a flush would sit inside the region);
+    # the same loop with device-resident inputs and no copies is timed the
+    # same way beside it.
     e2e = None
     if not args.no_e2e:
-        out_h = torch.empty((B, Hq, D), dtype=bf).pin_memory()
         nq, nkv = q_h[0].numel(), kn_h[0].numel()
         rec_h = torch.cat([q_h.reshape(n_total, -1), kn_h.reshape(n_total, -1), vn_h.reshape(n_total, -1)],
                           dim=1).pin_memory()
-        rec_d = torch.empty(nq + 2 * nkv, dtype=bf, device=dev)
-        qb = rec_d[:nq].view(q_d[0].shape)
-        kb = rec_d[nq:nq + nkv].view(kn_d[0].shape)
-        vb = rec_d[nq + nkv:].view(vn_d[0].shape)
+        rec_d = [torch.empty(nq + 2 * nkv, dtype=bf, device=dev) for _ in range(2)]
+        views = [(r[:nq].view(q_d[0].shape), r[nq:nq + nkv].view(kn_d[0].shape), r[nq + nkv:].view(vn_d[0].shape))
+                 for r in rec_d]
+        outs = [torch.empty((B, Hq, D), dtype=bf, device=dev) for _ in range(2)]
+        out_h = [torch.empty((B, Hq, D), dtype=bf).pin_memory() for _ in range(2)]
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-        def e2e_step(s, ev=None):
-            if ev is not None:
-                ev[0].record(stream)
-            rec_d.copy_(rec_h[s], non_blocking=True)
-            layer.append_decode(kb, vb, qb, out)
-            out_h.copy_(out, non_blocking=True)
-            if ev is not None:
-                ev[1].record(stream)
+        def e2e_loop(s0, n, copies=True):
+            ready = [torch.cuda.Event() for _ in range(2)]
+            used = [torch.cuda.Event() for _ in range(2)]
+            copied = [torch.cuda.Event() for _ in range(2)]
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            up.wait_event(t0)
+            down.wait_event(t0)
+            if copies:
+                with torch.cuda.stream(up):
+                    rec_d[0].copy_(rec_h[s0], non_blocking=True)
+                    ready[0].record(up)
+            for i in range(n):
+                cur, nxt = i % 2, (i + 1) % 2
+                if copies:
+                    if i + 1 < n:
+                        with torch.cuda.stream(up):
+                            if i >= 1:
+                                up.wait_event(used[nxt])  # step i - 1 is done with that record
+                            rec_d[nxt].copy_(rec_h[s0 + i + 1], non_blocking=True)
+                            ready[nxt].record(up)
+                    stream.wait_event(ready[cur])
+                    if i >= 2:
+                        stream.wait_event(copied[cur])  # step i - 2's output is back on the host
+                    qb, kb, vb = views[cur]
+                    layer.append_decode(kb, vb, qb, outs[cur])
+                    used[cur].record(stream)
+                    with torch.cuda.stream(down):
+                        down.wait_event(used[cur])
+                        out_h[cur].copy_(outs[cur], non_blocking=True)
+                        copied[cur].record(down)
+                else:
+                    layer.append_decode(kn_d[s0 + i], vn_d[s0 + i], q_d[s0 + i], outs[cur])
+            stream.wait_stream(up)
+            stream.wait_stream(down)
+            t1.record(stream)
+            return t0, t1
 
-        for _ in range(W_):
-            flush.fill_(0.0)
-            e2e_step(s_idx)
-            s_idx += 1
-        ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_)]
+        e2e_loop(s_idx, W_)
+        s_idx += W_
         torch.cuda.synchronize(dev)
         barrier(world, local)
-        for i in range(K_):
-            flush.fill_(0.0)
-            e2e_step(s_idx, ev2[i])
-            s_idx += 1
+        t0, t1 = e2e_loop(s_idx, K_)
+        s_idx += K_
         torch.cuda.synchronize(dev)
         barrier(world, local)
-        e2e_s = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev2) / 1e3, world)
+        e2e_s = max_over_ranks(t0.elapsed_time(t1) / 1e3, world)
+        torch.cuda.synchronize(dev)
+        t0, t1 = e2e_loop(s_idx, K_, copies=False)
+        s_idx += K_
+        torch.cuda.synchronize(dev)
+        same_loop_s = max_over_ranks(t0.elapsed_time(t1) / 1e3, world)
         e2e = {"value": aggregate_rate(world, B, K_, e2e_s), "unit": "query-tok/s",
-               "h2d_bytes_per_step": int(rec_h[0].numel() * es), "d2h_bytes_per_step": int(out_h.numel() * es),
-               "how": "per step: one pinned host record [q | k_new | v_new] copied in, recsa_append_decode, the "
-                      "output copied back to pinned host memory, all inside the step's events"}
+               "h2d_bytes_per_step": int(rec_h[0].numel() * es), "d2h_bytes_per_step": int(out_h[0].numel() * es),
+               "device_same_loop": aggregate_rate(world, B, K_, same_loop_s),
+               "how": "per step: one pinned host record [q | k_new | v_new] copied in (side stream, one step "
+                      "ahead), recsa_append_decode, the output copied back to pinned host memory (third stream); "
+                      "timed from the first upload to the last download, no L2 flush between steps; "
+                      "device_same_loop = the same loop on device-resident inputs, no copies"}
         layer.check()
 
     # ---- dense flash-decode comparator on the same cache
@@ -637,6 +760,11 @@ def main():
                          "refresh of the nodes the new token touched + one query per unit, fp64; trees built and "
                          "queries generated before timing"}
 
+    backward = None
+    if not args.no_backward:
+        backward = measure_backward(layer, w, q_d[0], dev, flush, peaks, (Kh.numpy(), Vh.numpy()),
+                                    os.cpu_count() or 1, rank == 0 and world == 1 and not args.no_cpu_baseline)
+
     prefill = None
     if not args.no_prefill:
         prefill = measure_prefill(args.prefill_workload, dev, flush, peaks)
@@ -661,7 +789,7 @@ def main():
             "build_tree": {"ms": build_ms, "gbs": build_bytes / (build_ms / 1e3) / 1e9,
                            "frac_hbm": build_bytes / (build_ms / 1e3) / 1e9 / hbm},
             "e2e": e2e, "gpu_launches": K_, "clocks": clk, "dense_decode": dense, "cpu_baseline": cpu,
-            "wall_s_timed_loop": wall_s, "input_gen_s": gen_s, "prefill": prefill,
+            "wall_s_timed_loop": wall_s, "input_gen_s": gen_s, "prefill": prefill, "backward": backward,
         }
         print(json.dumps(line), flush=True)
     layer.close()
