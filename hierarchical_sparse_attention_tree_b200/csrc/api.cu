@@ -23,7 +23,7 @@ cudaError_t launch_set_lengths(const TreeParams&, const long long*, cudaStream_t
 cudaError_t launch_bump_lengths(const TreeParams&, long long, cudaStream_t);
 template <typename T, int D, int G>
 cudaError_t launch_decode(const TreeParams&, const void*, const void*, const void*, void*, int*, long long*,
-                          cudaStream_t);
+                          float*, cudaStream_t);
 template <typename T, int D, int G>
 cudaError_t launch_dense(const void*, const void*, const void*, void*, int, long long, long long, float*, int,
                          cudaStream_t);
@@ -37,6 +37,9 @@ cudaError_t launch_prefill_tree_tc(const TreeParams&, const void*, void*, const 
 size_t prefill_tree_scratch_bytes(const TreeParams& p, int C, int Hq);
 bool prefill_tree_supported(int D, int b);
 size_t decode_smem_bytes(int D, int G, int elem, int k, int b, int J_cap, bool fused);
+cudaError_t launch_distill_loss(const float*, const float*, float*, float*, long long, cudaStream_t);
+template <typename T>
+cudaError_t launch_pooler_update(float*, const float*, float, void*, float*, int, cudaStream_t);
 size_t dense_static_scratch_bytes();
 cudaError_t dense_static_scratch(float** out);
 }  // namespace recsa
@@ -378,7 +381,7 @@ recsa_status recsa_decode(recsa_ctx* ctx, const void* q, void* out, int* sel_out
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
     DISPATCH_TD(c.dtype, c.head_dim,
-                DISPATCH_G(ctx->G, e = launch_decode<T, DD, GG>(ctx->p, nullptr, nullptr, q, out, sel_out, rows_out, s)));
+                DISPATCH_G(ctx->G, e = launch_decode<T, DD, GG>(ctx->p, nullptr, nullptr, q, out, sel_out, rows_out, nullptr, s)));
     if (e != cudaSuccess) return cuda_fail(e, "recsa_decode");
     return RECSA_OK;
 }
@@ -396,7 +399,7 @@ recsa_status recsa_append_decode(recsa_ctx* ctx, const void* k_new, const void* 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
     DISPATCH_TD(c.dtype, c.head_dim,
-                DISPATCH_G(ctx->G, e = launch_decode<T, DD, GG>(ctx->p, k_new, v_new, q, out, sel_out, rows_out, s)));
+                DISPATCH_G(ctx->G, e = launch_decode<T, DD, GG>(ctx->p, k_new, v_new, q, out, sel_out, rows_out, nullptr, s)));
     if (e != cudaSuccess) return cuda_fail(e, "recsa_append_decode");
     for (int b = 0; b < c.batch; b++) ctx->len[b] += 1;
     return RECSA_OK;
@@ -697,6 +700,105 @@ recsa_status recsa_tree_backward(recsa_ctx* ctx, float* dk, float* dv, float* dw
     if (maxL > 0) DISPATCH_TD(c.dtype, c.head_dim, e = launch_tree_backward<T, DD>(ctx->p, a, maxL, s));
     if (e == cudaSuccess) e = cudaMemsetAsync(scratch, 0, l.nodes_end, s);
     if (e != cudaSuccess) return cuda_fail(e, "recsa_tree_backward");
+    return RECSA_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------ distillation
+
+namespace {
+// Distillation scratch: [the backward scratch][fp32 output B Hq d][its
+// gradient B Hq d][dq B Hq d][selections B H J_cap k int32][dW d d][loss].
+struct DistillLayout {
+    BwdLayout bwd;
+    size_t out, dout, dq, sel, dw, loss, total;
+};
+DistillLayout distill_layout(const recsa_config* c) {
+    DistillLayout d{};
+    d.bwd = bwd_layout(c);
+    const size_t n = (size_t)c->batch * c->n_q_heads * c->head_dim;
+    const Layout l = layout_for(c);
+    size_t o = d.bwd.total;
+    d.out = o; o = align256(o + n * 4);
+    d.dout = o; o = align256(o + n * 4);
+    d.dq = o; o = align256(o + n * 4);
+    d.sel = o; o = align256(o + (size_t)c->batch * c->n_kv_heads * l.J_cap * c->k * 4);
+    d.dw = o; o = align256(o + (size_t)c->head_dim * c->head_dim * 4);
+    d.loss = o; o = align256(o + 4);
+    d.total = o;
+    return d;
+}
+}  // namespace
+
+extern "C" {
+
+size_t recsa_distill_scratch_bytes(const recsa_config* cfg) {
+    if (check_config(cfg) != RECSA_OK) return 0;
+    return distill_layout(cfg).total;
+}
+
+recsa_status recsa_distill_step(recsa_ctx* ctx, const void* q, const float* target, float lr, float* w_master,
+                                float* loss, float* dw_out, void* scratch, size_t scratch_bytes,
+                                recsa_stream_t stream) {
+    if (!ctx || !q || !target || !w_master || !scratch) return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    if (!aligned(q, 16) || !aligned(target, 16)) return fail(RECSA_ERR_INVALID_ARG, "q/target not 16-byte aligned");
+    if (!aligned(scratch, 256)) return fail(RECSA_ERR_INVALID_ARG, "scratch not 256-byte aligned");
+    if (!(lr >= 0.f)) return fail(RECSA_ERR_INVALID_ARG, "lr must be >= 0");
+    const recsa_config& c = ctx->cfg;
+    const DistillLayout l = distill_layout(&c);
+    if (scratch_bytes < l.total) return fail(RECSA_ERR_INVALID_ARG, "scratch of %zu bytes, %zu needed", scratch_bytes, l.total);
+    long long maxL = 0;
+    for (int b = 0; b < c.batch; b++) {
+        if (ctx->len[b] < 1) return fail(RECSA_ERR_INVALID_ARG, "sequence %d holds no tokens", b);
+        maxL = ctx->len[b] > maxL ? ctx->len[b] : maxL;
+    }
+    char* base = static_cast<char*>(scratch);
+    float* out = reinterpret_cast<float*>(base + l.out);
+    float* dout = reinterpret_cast<float*>(base + l.dout);
+    int* sel = reinterpret_cast<int*>(base + l.sel);
+    float* dw = reinterpret_cast<float*>(base + l.dw);
+    float* lossd = reinterpret_cast<float*>(base + l.loss);
+    const long long n = (long long)c.batch * c.n_q_heads * c.head_dim;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // node accumulators, dW and the loss start at zero
+    cudaError_t e = cudaMemsetAsync(scratch, 0, l.bwd.nodes_end, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dw, 0, (size_t)c.head_dim * c.head_dim * 4, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(lossd, 0, 4, s);
+    // forward (fp32 output, selections kept), loss and its gradient
+    if (e == cudaSuccess)
+        DISPATCH_TD(c.dtype, c.head_dim,
+                    DISPATCH_G(ctx->G, e = launch_decode<T, DD, GG>(ctx->p, nullptr, nullptr, q, nullptr, sel,
+                                                                    nullptr, out, s)));
+    if (e == cudaSuccess) e = launch_distill_loss(out, target, dout, lossd, n, s);
+    // the pooler's gradient only: no token gradients
+    BwdArgs a = bwd_args(ctx, scratch);
+    a.q = q;
+    a.dout = dout;
+    a.dout_f32 = 1;
+    a.sel = sel;
+    a.dq = reinterpret_cast<float*>(base + l.dq);
+    a.dk = nullptr;
+    a.dv = nullptr;
+    a.dw = dw;
+    if (e == cudaSuccess)
+        DISPATCH_TD(c.dtype, c.head_dim, DISPATCH_G(ctx->G, e = launch_decode_backward<T, DD, GG>(ctx->p, a, s)));
+    if (e == cudaSuccess) DISPATCH_TD(c.dtype, c.head_dim, e = launch_tree_backward<T, DD>(ctx->p, a, maxL, s));
+    // update, then every node key again under the new pooler
+    if (e == cudaSuccess) {
+        if (c.dtype == RECSA_BF16)
+            e = launch_pooler_update<__nv_bfloat16>(w_master, dw, lr, const_cast<void*>(ctx->p.Wt), dw_out,
+                                                    c.head_dim, s);
+        else
+            e = launch_pooler_update<float>(w_master, dw, lr, const_cast<void*>(ctx->p.Wt), dw_out, c.head_dim, s);
+    }
+    for (int j = 1; j <= ctx->p.J_cap && e == cudaSuccess; j++) {
+        const long long nodes = (maxL + ctx->p.span[j] - 1) / ctx->p.span[j];
+        if (nodes == 0) continue;
+        DISPATCH_TD(c.dtype, c.head_dim, e = launch_build_level<T, DD>(ctx->p, j, 0, 0, nodes, s));
+    }
+    if (e == cudaSuccess && loss) e = cudaMemcpyAsync(loss, lossd, 4, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "recsa_distill_step");
     return RECSA_OK;
 }
 

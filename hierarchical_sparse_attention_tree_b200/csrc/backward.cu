@@ -248,7 +248,10 @@ __device__ __forceinline__ void load_unit(const TreeParams& p, const BwdArgs& a,
     for (int g = 0; g < G; g++) {
         const long long row = (u * G + g) * D;
         load_pairs<T, D>(reinterpret_cast<const T*>(a.q) + row, lane, v.ql[g], v.qh[g]);
-        load_pairs<T, D>(reinterpret_cast<const T*>(a.dout) + row, lane, v.dl[g], v.dh[g]);
+        if (a.dout_f32)
+            load_pairs<float, D>(reinterpret_cast<const float*>(a.dout) + row, lane, v.dl[g], v.dh[g]);
+        else
+            load_pairs<T, D>(reinterpret_cast<const T*>(a.dout) + row, lane, v.dl[g], v.dh[g]);
     }
     __syncwarp();
 }
@@ -560,18 +563,20 @@ __global__ void __launch_bounds__(BWD_THREADS, 2) bwd_entry_kernel(TreeParams p,
                     aqh[g][i] += c * rkh[i];
                 }
             }
-            float* rk;
-            float* rv;
+            float* rk = nullptr;
+            float* rv = nullptr;
             if (bt.j[t] >= 1) {
                 rk = a.gK[bt.j[t]] + (u * p.rows[bt.j[t]] + bt.m[t]) * D;
                 rv = a.gV[bt.j[t]] + (u * p.rows[bt.j[t]] + bt.m[t]) * D;
-            } else {
+            } else if (a.dk) {
                 const long long row = token_row(tok, u, bt.m[t]);
                 rk = a.dk + row * D;
                 rv = a.dv + row * D;
             }
-            add_pairs<D>(rk, lane, gkl, gkh);
-            add_pairs<D>(rv, lane, gvl, gvh);
+            if (rk) {
+                add_pairs<D>(rk, lane, gkl, gkh);
+                add_pairs<D>(rv, lane, gvl, gvh);
+            }
         }
         xg += nb;
     }
@@ -729,6 +734,19 @@ __global__ void __launch_bounds__(BWD_THREADS, 2)
                 }
                 store_pairs<D>(a.gK[j] + (u * p.rows[j] + m) * D, lane, hlo, hhi);
                 store_pairs<D>(a.gV[j] + (u * p.rows[j] + m) * D, lane, slo, shi);
+            } else if (!a.dk) {
+                // pooler gradient only: the tokens' keys for the mean
+                const T* kb = reinterpret_cast<const T*>(p.K[0]) + token_row(tok, u, m * p.b) * D;
+#pragma unroll 8
+                for (long long c = 0; c < nch; c++) {
+                    float kl[NP], kh[NP];
+                    load_pairs<T, D>(kb + c * D, lane, kl, kh);
+#pragma unroll
+                    for (int i = 0; i < NP; i++) {
+                        mlo[i] += kl[i];
+                        mhi[i] += kh[i];
+                    }
+                }
             } else {
                 // the node's tokens (contiguous rows: a node never straddles
                 // a page): their keys for the mean, dk += h, dv += s

@@ -10,10 +10,10 @@ constexpr int PLAN_INTS = 72;          // valid, J, items, pad, then off[j], nc[
 
 struct BwdArgs {
     const void* q;     // [B][Hq][D], storage type
-    const void* dout;  // [B][Hq][D], storage type
+    const void* dout;  // [B][Hq][D], storage type (fp32 if dout_f32)
     const int* sel;    // [B*H][J_cap][k], the forward's selections
     float* dq;         // [B][Hq][D]
-    float* dk;         // token gradients, the cache's row layout, [rows][D]
+    float* dk;         // token gradients, the cache's row layout, [rows][D] (null: not wanted, with dv)
     float* dv;
     float* dw;         // [D][D], dW[r][c] for W[r][c]
     float* gK[MAXJ + 1];  // node-key gradient accumulators [B*H][rows[j]][D] (j >= 1)
@@ -24,6 +24,7 @@ struct BwdArgs {
     float* ag;         // [B*H][E_cap][G] <dout_g, v_e>
     float* st;         // [B*H][G][3] softmax maximum, denominator, sum_e p_e <dout, v_e>
     int E_cap;
+    int dout_f32;
 };
 
 template <typename T, int D, int G>

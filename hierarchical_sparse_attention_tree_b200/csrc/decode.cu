@@ -45,6 +45,7 @@ struct DecodeArgs {
     const void* v_new;
     const void* q;
     void* out;
+    float* out_f32;       // nullable [B][Hq][D]: the output in fp32 instead of `out`
     int* sel_out;         // nullable [B*H][J_cap][k]
     long long* rows_out;  // nullable [B*H][2]
     int my_max;           // candidates per CTA, upper bound
@@ -723,7 +724,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
             const int g = (rank * SL + i) / D;
             float s = 0.f;
             for (int r = 0; r < CS; r++) s += gat[r * GST + i] * fac[r * G + g];
-            outp[i] = from_f<T>(bad ? 0.f : s * fac[CS * G + g]);
+            const float o = bad ? 0.f : s * fac[CS * G + g];
+            if (a.out_f32)
+                a.out_f32[(u * G) * D + rank * SL + i] = o;
+            else
+                outp[i] = from_f<T>(o);
         }
     }
     if (rank == 0) {
@@ -759,11 +764,11 @@ size_t decode_smem_bytes(int D, int G, int elem, int k, int b, int J_cap, bool f
 // token of every unit, then decode against the grown tree).
 template <typename T, int D, int G>
 cudaError_t launch_decode(const TreeParams& p, const void* k_new, const void* v_new, const void* q, void* out,
-                          int* sel_out, long long* rows_out, cudaStream_t s) {
+                          int* sel_out, long long* rows_out, float* out_f32, cudaStream_t s) {
     const int CS = DEC_CLUSTER;
     const long long maxc = (long long)p.k * p.b > p.b ? (long long)p.k * p.b : p.b;
     const bool fused = k_new != nullptr;
-    DecodeArgs a{k_new, v_new, q, out, sel_out, rows_out, (int)((maxc + CS - 1) / CS), 0};
+    DecodeArgs a{k_new, v_new, q, out, out_f32, sel_out, rows_out, (int)((maxc + CS - 1) / CS), 0};
     a.region0 = (int)decode_region0(D, G, a.my_max, (int)sizeof(T), p.J_cap, fused);
     const size_t smem = a.region0 + decode_smem_tail(D, G, a.my_max);
     auto kern = decode_kernel<T, D, G>;
@@ -792,7 +797,7 @@ cudaError_t launch_decode(const TreeParams& p, const void* k_new, const void* v_
 
 #define RECSA_INST_DEC(T, D, G) \
     template cudaError_t launch_decode<T, D, G>(const TreeParams&, const void*, const void*, const void*, void*, \
-                                                int*, long long*, cudaStream_t);
+                                                int*, long long*, float*, cudaStream_t);
 #define RECSA_INST_DEC_G(T, D) RECSA_INST_DEC(T, D, 1) RECSA_INST_DEC(T, D, 2) RECSA_INST_DEC(T, D, 4) RECSA_INST_DEC(T, D, 8)
 RECSA_INST_DEC_G(float, 64)
 RECSA_INST_DEC_G(float, 128)

@@ -28,6 +28,7 @@ class RecsaLayer:
         self.v_cache = torch.zeros_like(self.k_cache)
         self.workspace = torch.zeros(_r.workspace_bytes(self.cfg), dtype=torch.uint8, device=device)
         w = pooler_w.to(device=device, dtype=dtype).contiguous()
+        self.w_master = w.float().clone()  # fp32 master copy of the pooler (distillation updates it)
         self.ctx = _r.Context(self.cfg, self.k_cache, self.v_cache, self.workspace, w, stream, self.page_table,
                               page_size)
         torch.cuda.current_stream(self.device).synchronize() if stream is None else stream.synchronize()
@@ -127,6 +128,19 @@ class RecsaLayer:
         if getattr(self, "dk", None) is None:
             self.zero_grad()
         self.ctx.tree_backward(self.dk, self.dv, self.dw, self._bwd_scratch, stream)
+
+    def distill_step(self, q, target, lr, dw_out=None, stream=None):
+        """One gradient-descent step of the pooler towards dense attention:
+        target [B][H_q][d] (fp32) are the dense outputs for q. Returns the
+        step's loss (a device scalar); self.w_master holds the new pooler
+        and the tree has been rebuilt under it."""
+        if getattr(self, "_distill_scratch", None) is None:
+            self._distill_scratch = torch.empty(max(self.ctx.distill_scratch_bytes(), 256), dtype=torch.uint8,
+                                                device=self.device)
+        loss = torch.empty((), dtype=torch.float32, device=self.device)
+        self.ctx.distill_step(q, target.contiguous(), lr, self.w_master, self._distill_scratch, loss, dw_out,
+                              stream)
+        return loss
 
     def query_stats(self, stream=None):
         return self.ctx.query_stats(stream)

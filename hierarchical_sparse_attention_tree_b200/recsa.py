@@ -23,7 +23,7 @@ EXPORTS = [
     "recsa_prefill_scratch_bytes", "recsa_prefill", "recsa_get_lengths", "recsa_tree_shape", "recsa_level_arrays",
     "recsa_query_stats", "recsa_check_device", "recsa_last_error", "recsa_destroy", "recsa_dense_decode_scratch_bytes",
     "recsa_dense_decode", "recsa_dense_decode_static", "recsa_backward_scratch_bytes", "recsa_decode_backward",
-    "recsa_tree_backward",
+    "recsa_tree_backward", "recsa_distill_scratch_bytes", "recsa_distill_step",
 ]
 
 
@@ -62,6 +62,8 @@ def lib():
             "recsa_backward_scratch_bytes": (sz, [P(Config)]),
             "recsa_decode_backward": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
             "recsa_tree_backward": (i32, [vp, vp, vp, vp, vp, sz, vp]),
+            "recsa_distill_scratch_bytes": (sz, [P(Config)]),
+            "recsa_distill_step": (i32, [vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, sz, vp]),
             "recsa_append_decode": (i32, [vp, vp, vp, vp, vp, vp, vp, vp]),
             "recsa_prefill_scratch_bytes": (sz, [P(Config), i32]),
             "recsa_prefill": (i32, [vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
@@ -210,6 +212,14 @@ class Context:
     def tree_backward(self, dk, dv, dw, scratch, stream=None):
         _check(lib().recsa_tree_backward(self.handle, _ptr(dk), _ptr(dv), _ptr(dw), _ptr(scratch),
                                          scratch.numel() * scratch.element_size(), _stream(stream)))
+
+    def distill_scratch_bytes(self) -> int:
+        return lib().recsa_distill_scratch_bytes(ctypes.byref(self.cfg))
+
+    def distill_step(self, q, target, lr, w_master, scratch, loss=None, dw_out=None, stream=None):
+        _check(lib().recsa_distill_step(self.handle, _ptr(q), _ptr(target), float(lr), _ptr(w_master), _ptr(loss),
+                                        _ptr(dw_out), _ptr(scratch), scratch.numel() * scratch.element_size(),
+                                        _stream(stream)))
 
     def query_stats(self, stream=None):
         """(depth, k_rows, v_rows) of the last decode, per (sequence, KV head)

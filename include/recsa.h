@@ -245,6 +245,30 @@ recsa_status recsa_decode_backward(recsa_ctx* ctx, const void* q, const void* do
 recsa_status recsa_tree_backward(recsa_ctx* ctx, float* dk, float* dv, float* dw, void* scratch,
                                  size_t scratch_bytes, recsa_stream_t stream);
 
+/* ---------------------------------------------------------------------
+ * One distillation step of the pooler. The RecSA abstract trains the
+ * pooler so that tree attention reproduces dense attention; this is the
+ * plainest reading of that step for decode queries: the loss is the mean
+ * squared difference between the layer's outputs and the caller's dense
+ * attention outputs for the same queries over the same cache,
+ *   loss = sum over (sequence, query head, coordinate) of (out - target)^2 / n,
+ *   n = B * H_q * d,
+ * with the selections of this forward held fixed; W moves by plain gradient
+ * descent, w_master <- w_master - lr * dLoss/dW, the context's pooler takes
+ * the new values (rounded to cfg->dtype) and every node key is rebuilt
+ * under it (as recsa_build_tree over the current lengths).
+ * q [B][H_q][d] in cfg->dtype and target [B][H_q][d] fp32 (device, 16-byte
+ * aligned); w_master [d][d] fp32 device, row-major like the pooler given
+ * to recsa_init (the caller keeps this master copy; updated in place); loss
+ * (nullable) device fp32 scalar, the step's loss before the update; dw_out
+ * (nullable) device [d][d] fp32, the step's gradient. scratch: device
+ * memory of recsa_distill_scratch_bytes(cfg) bytes, 256-byte aligned (no
+ * clearing needed). Asynchronous on `stream`. */
+size_t recsa_distill_scratch_bytes(const recsa_config* cfg);
+recsa_status recsa_distill_step(recsa_ctx* ctx, const void* q, const float* target, float lr, float* w_master,
+                                float* loss, float* dw_out, void* scratch, size_t scratch_bytes,
+                                recsa_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the device error word:
  * RECSA_ERR_DEVICE if a kernel flagged an inconsistent state (bits: 1 a
  * length out of range, 2 a tree shape inconsistent with the lengths, 4 a

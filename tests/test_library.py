@@ -104,3 +104,11 @@ def test_backward_scratch_and_null_arguments():
     assert R.lib().recsa_backward_scratch_bytes(ctypes.byref(bad)) == 0
     assert R.lib().recsa_decode_backward(None, None, None, None, None, None, None, None, 0, None) == R.ERR_INVALID_ARG
     assert R.lib().recsa_tree_backward(None, None, None, None, None, 0, None) == R.ERR_INVALID_ARG
+
+
+def test_distill_scratch_and_null_arguments():
+    cfg = R.make_config(4, 8, 32, 128, 64, 16, 524288)
+    n = R.lib().recsa_distill_scratch_bytes(ctypes.byref(cfg))
+    assert n >= R.lib().recsa_backward_scratch_bytes(ctypes.byref(cfg)) + 3 * 4 * 32 * 128 * 4
+    assert R.lib().recsa_distill_step(None, None, None, ctypes.c_float(0.1), None, None, None, None, 0,
+                                      None) == R.ERR_INVALID_ARG
