@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-distill", action="store_true")
     ap.add_argument("--prefill-workload", default="prefill_524k")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the chunked prefill (profiling): no decode, no baselines")
@@ -477,6 +478,67 @@ def measure_backward(layer, w, q, dev, flush, peaks, kv_host, cpu_threads, with_
     return res
 
 
+def measure_distill(layer, w, q, dev, flush, build_ms, kv_host, cpu_threads, with_cpu):
+    """One distillation step of the pooler (recsa_distill_step: forward,
+    squared error, the pooler's gradient, update, tree rebuild) on the
+    layer's current cache, median of 5 after 2 warm-ups, L2 flushed before
+    each. The dense targets are synthetic N(0, 0.1^2) stand-ins (the step's
+    cost does not depend on them); lr = 0 leaves the pooler, so the tree the
+    rest of the run uses is unchanged. Beside it, the oracle doing the same
+    step (tree build, query, gradient) for a sample of units on the host."""
+    B, H, Hq, D, G = w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim, w.group
+    stream = torch.cuda.current_stream(dev)
+    target = torch.from_numpy(synth.plain(92, 0, (B, Hq, D), 0.0, 0.1)).to(dev)
+    for _ in range(2):
+        layer.distill_step(q, target, 0.0)
+    ts = []
+    for _ in range(5):
+        flush.fill_(8.0)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        loss = layer.distill_step(q, target, 0.0)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        ts.append(a.elapsed_time(b_))
+    layer.check()
+    ms = statistics.median(ts)
+    res = {"step_ms": ms, "tree_rebuild_ms_alone": build_ms, "queries": B * Hq, "loss": float(loss.item()),
+           "how": "recsa_distill_step on the decode workload's cache, one query per sequence, synthetic targets, "
+                  "lr 0; median of 5, L2 flushed"}
+    del layer._distill_scratch
+    layer._distill_scratch = None
+    torch.cuda.empty_cache()
+    if with_cpu:
+        import oracle
+
+        L0, b = w.length, w.branching
+        units = [(bb, h) for bb in range(B) for h in range(H)][:max(1, min(cpu_threads, B * H))]
+        Wf = synth.as_f32(synth.workload_pooler(w))
+        qh = q.view(torch.int16).cpu().numpy()
+        th = target.cpu().numpy().astype(np.float64)
+        n = B * Hq * D
+
+        def unit(bh):
+            bb, h = bh
+            Kt, Vt = kv_host[0][bb, h], kv_host[1][bb, h]
+            tr = oracle.Tree(D, b, L0, oracle.STORE_BF16).build(Kt, Vt, L0, Wf)
+            qu = synth.as_f32(np.ascontiguousarray(qh[bb, h * G:(h + 1) * G]))
+            r = oracle.query_tree(tr, Kt, Vt, qu, w.k, G, w.rope_base)
+            diff = r["out"] - th[bb, h * G:(h + 1) * G]
+            return oracle.query_grad(tr.K, tr.V, Kt, Vt, L0, qu, 2 * diff / n, Wf, D, b, w.k, G, w.rope_base)["dW"]
+
+        pool = oracle.pool(len(units))
+        t0 = time.perf_counter()
+        list(pool.map(unit, units))
+        dt = time.perf_counter() - t0
+        pool.shutdown()
+        res["cpu_baseline"] = {"value": len(units) / dt, "unit": "units/s", "cores": len(units), "kind": "oracle",
+                               "sample": f"the step's tree build, query and gradient for {len(units)} units "
+                                         f"(L = {L0}) in parallel (the update itself omitted)"}
+        res["gpu_units_s"] = B * H / (ms / 1e3)
+    return res
+
+
 # -------------------------------------------------------------------- main
 
 
@@ -765,6 +827,11 @@ def main():
         backward = measure_backward(layer, w, q_d[0], dev, flush, peaks, (Kh.numpy(), Vh.numpy()),
                                     os.cpu_count() or 1, rank == 0 and world == 1 and not args.no_cpu_baseline)
 
+    distill = None
+    if not args.no_distill:
+        distill = measure_distill(layer, w, q_d[0], dev, flush, build_ms, (Kh.numpy(), Vh.numpy()),
+                                  os.cpu_count() or 1, rank == 0 and world == 1 and not args.no_cpu_baseline)
+
     prefill = None
     if not args.no_prefill:
         prefill = measure_prefill(args.prefill_workload, dev, flush, peaks)
@@ -790,6 +857,7 @@ def main():
                            "frac_hbm": build_bytes / (build_ms / 1e3) / 1e9 / hbm},
             "e2e": e2e, "gpu_launches": K_, "clocks": clk, "dense_decode": dense, "cpu_baseline": cpu,
             "wall_s_timed_loop": wall_s, "input_gen_s": gen_s, "prefill": prefill, "backward": backward,
+            "distill": distill,
         }
         print(json.dumps(line), flush=True)
     layer.close()
