@@ -83,6 +83,14 @@ __device__ __forceinline__ void store_pairs(float* row, int lane, const float* l
         *reinterpret_cast<float2*>(row + D / 2 + lane * NP) = make_float2(hi[0], hi[1]);
     }
 }
+// E consecutive floats (E = 2 or 4, naturally aligned) stored at once.
+template <int E>
+__device__ __forceinline__ void store_vecf(float* p, const float* v) {
+    if constexpr (E == 4)
+        *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    else
+        *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+}
 template <int D>
 __device__ __forceinline__ void add_pairs(float* row, int lane, const float* lo, const float* hi) {
     constexpr int NP = D / 64;
@@ -716,6 +724,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 2)
         float mlo[NP], mhi[NP];
 #pragma unroll
         for (int i = 0; i < NP; i++) mlo[i] = mhi[i] = 0.f;
+        bool mean_staged = false;  // the token branch writes the mean row itself
         if (live) {
             float hlo[NP], hhi[NP];
             wt_times<T, D>(sm, sm.g[warp], lane, 1.f / (float)nch, hlo, hhi);
@@ -749,47 +758,67 @@ __global__ void __launch_bounds__(BWD_THREADS, 2)
                 }
             } else {
                 // the node's tokens (contiguous rows: a node never straddles
-                // a page): their keys for the mean, dk += h, dv += s
+                // a page): their keys for the mean, dk += h, dv += s. Here no
+                // rotation pairs are needed, so the rows are read and written
+                // contiguously (E elements per lane, one access per row and
+                // array); h and s change layout through the warp's mean row.
+                constexpr int E = D / 32;
+                float* stage = sm.mean[warp];
+                float hc[E], sc[E], mc[E];
+                store_pairs<D>(stage, lane, hlo, hhi);
+                __syncwarp();
+                load_vec<float, E>(stage + lane * E, hc);
+                __syncwarp();
+                store_pairs<D>(stage, lane, slo, shi);
+                __syncwarp();
+                load_vec<float, E>(stage + lane * E, sc);
+#pragma unroll
+                for (int e = 0; e < E; e++) mc[e] = 0.f;
                 const long long row0 = token_row(tok, u, m * p.b);
-                const T* kb = reinterpret_cast<const T*>(p.K[0]) + row0 * D;
-                float* dkb = a.dk + row0 * D;
-                float* dvb = a.dv + row0 * D;
-                constexpr int U = 4;  // rows in flight per lane and array
+                const T* kb = reinterpret_cast<const T*>(p.K[0]) + row0 * D + lane * E;
+                float* dkb = a.dk + row0 * D + lane * E;
+                float* dvb = a.dv + row0 * D + lane * E;
+                constexpr int U = 8;  // rows in flight per lane and array
                 long long c = 0;
                 for (; c + U <= nch; c += U) {
-                    float kl[U][NP], kh[U][NP], xl[U][NP], xh[U][NP], yl[U][NP], yh[U][NP];
+                    float kx[U][E], xx[U][E], yy[U][E];
 #pragma unroll
                     for (int x = 0; x < U; x++) {
-                        load_pairs<T, D>(kb + (c + x) * D, lane, kl[x], kh[x]);
-                        load_pairs<float, D>(dkb + (c + x) * D, lane, xl[x], xh[x]);
-                        load_pairs<float, D>(dvb + (c + x) * D, lane, yl[x], yh[x]);
+                        load_vec<T, E>(kb + (c + x) * D, kx[x]);
+                        load_vec<float, E>(dkb + (c + x) * D, xx[x]);
+                        load_vec<float, E>(dvb + (c + x) * D, yy[x]);
                     }
 #pragma unroll
                     for (int x = 0; x < U; x++) {
 #pragma unroll
-                        for (int i = 0; i < NP; i++) {
-                            mlo[i] += kl[x][i];
-                            mhi[i] += kh[x][i];
-                            xl[x][i] += hlo[i];
-                            xh[x][i] += hhi[i];
-                            yl[x][i] += slo[i];
-                            yh[x][i] += shi[i];
+                        for (int e = 0; e < E; e++) {
+                            mc[e] += kx[x][e];
+                            xx[x][e] += hc[e];
+                            yy[x][e] += sc[e];
                         }
-                        store_pairs<D>(dkb + (c + x) * D, lane, xl[x], xh[x]);
-                        store_pairs<D>(dvb + (c + x) * D, lane, yl[x], yh[x]);
+                        store_vecf<E>(dkb + (c + x) * D, xx[x]);
+                        store_vecf<E>(dvb + (c + x) * D, yy[x]);
                     }
                 }
                 for (; c < nch; c++) {
-                    float kl[NP], kh[NP];
-                    load_pairs<T, D>(kb + c * D, lane, kl, kh);
+                    float kx[E], xx[E], yy[E];
+                    load_vec<T, E>(kb + c * D, kx);
+                    load_vec<float, E>(dkb + c * D, xx);
+                    load_vec<float, E>(dvb + c * D, yy);
 #pragma unroll
-                    for (int i = 0; i < NP; i++) {
-                        mlo[i] += kl[i];
-                        mhi[i] += kh[i];
+                    for (int e = 0; e < E; e++) {
+                        mc[e] += kx[e];
+                        xx[e] += hc[e];
+                        yy[e] += sc[e];
                     }
-                    add_pairs<D>(dkb + c * D, lane, hlo, hhi);
-                    add_pairs<D>(dvb + c * D, lane, slo, shi);
+                    store_vecf<E>(dkb + c * D, xx);
+                    store_vecf<E>(dvb + c * D, yy);
                 }
+                const float inv_n = 1.f / (float)nch;
+                __syncwarp();
+#pragma unroll
+                for (int e = 0; e < E; e++) stage[lane * E + e] = mc[e] * inv_n;
+                mean_staged = true;
             }
             const float inv_c = 1.f / (float)nch;
 #pragma unroll
@@ -798,7 +827,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 2)
                 mhi[i] *= inv_c;
             }
         }
-        store_pairs<D>(sm.mean[warp], lane, mlo, mhi);
+        if (!mean_staged) store_pairs<D>(sm.mean[warp], lane, mlo, mhi);
         __syncthreads();
         accumulate_dw<T, D>(sm, tid);
     }
