@@ -64,32 +64,12 @@ __global__ void copy_tokens_kernel(TreeParams p, const T* __restrict__ k_new, co
 
 // ---------------------------------------------------------- build level
 
-// One warp per node of level j (unit = blockIdx.y). Recomputes nodes
-// m >= m0 of the tree over L' = len[u] + add tokens, where m0 = 0 for a full
-// build and len[u] / b^j when `add` new tokens were just copied in.
+// One node m of level j of unit u (one warp; kmw: the warp's row of shared
+// memory for the key mean).
 template <typename T, int D>
-__global__ void __launch_bounds__(256) build_level_kernel(TreeParams p, int j, long long add, int from_len) {
+__device__ __forceinline__ void build_node(const TreeParams& p, int j, long long u, long long m, long long L,
+                                           long long n_j, long long n_prev, const T* Wt, float* kmw, int lane) {
     constexpr int DPL = D / 32;  // columns per lane, contiguous
-    extern __shared__ __align__(16) unsigned char smem_b[];
-    T* Wt = reinterpret_cast<T*>(smem_b);                          // [D][D], storage type
-    float* km = reinterpret_cast<float*>(smem_b + D * D * sizeof(T));  // [warps][D]
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    for (int i = threadIdx.x; i < (int)(D * D * sizeof(T) / 16); i += blockDim.x)
-        reinterpret_cast<uint4*>(Wt)[i] = reinterpret_cast<const uint4*>(p.Wt)[i];
-    __syncthreads();
-
-    const long long u = blockIdx.y;
-    const long long L = p.len[u] + add;
-    const long long n_j = level_rows(p, j, L);
-    const long long n_prev = level_rows(p, j - 1, L);
-    const long long m0 = from_len ? p.len[u] / p.span[j] : 0;
-    const long long m = m0 + (long long)blockIdx.x * nwarps + warp;
-    if (m >= n_j) return;
-    if (n_j > p.rows[j] || L > p.cap) {
-        if (lane == 0) flag_error(p.err, ERR_SHAPE);
-        return;
-    }
-
     const bool right_edge = (m == n_j - 1);
     const long long c_lo = m * p.b;
     const long long c_hi = min(c_lo + (long long)p.b, n_prev);
@@ -103,8 +83,61 @@ __global__ void __launch_bounds__(256) build_level_kernel(TreeParams p, int j, l
 #pragma unroll
     for (int e = 0; e < DPL; e++) { ks[e] = 0.f; vs[e] = 0.f; }
 
-    constexpr int U = 8;
-    for (long long c0 = c_lo; c0 < c_hi; c0 += U) {
+    // Right-edge prefix sums: the running sums before the last child.
+    auto keep_edge = [&](long long c) {
+        if (right_edge && c == c_hi - 1) {
+            float* pk = p.PK[j] + u * D + lane * DPL;
+            float* pv = p.PV[j] + u * D + lane * DPL;
+#pragma unroll
+            for (int e = 0; e < DPL; e++) { pk[e] = ks[e]; pv[e] = vs[e]; }
+        }
+    };
+    if constexpr (sizeof(T) == 2 && DPL == 4) {
+        if (j == 1) {
+            // tokens (bf16): the rows stay packed (8 bytes a lane, no
+            // conversion registers) until they are added
+            constexpr int UB = 8;
+            auto add_row = [&](uint2 kr, uint2 vr) {
+                const __nv_bfloat162 k01 = *reinterpret_cast<const __nv_bfloat162*>(&kr.x);
+                const __nv_bfloat162 k23 = *reinterpret_cast<const __nv_bfloat162*>(&kr.y);
+                const __nv_bfloat162 v01 = *reinterpret_cast<const __nv_bfloat162*>(&vr.x);
+                const __nv_bfloat162 v23 = *reinterpret_cast<const __nv_bfloat162*>(&vr.y);
+                ks[0] = ks[0] + __low2float(k01);
+                ks[1] = ks[1] + __high2float(k01);
+                ks[2] = ks[2] + __low2float(k23);
+                ks[3] = ks[3] + __high2float(k23);
+                vs[0] = vs[0] + __low2float(v01);
+                vs[1] = vs[1] + __high2float(v01);
+                vs[2] = vs[2] + __low2float(v23);
+                vs[3] = vs[3] + __high2float(v23);
+            };
+            long long c0 = c_lo;
+            for (; c0 + UB <= c_hi; c0 += UB) {
+                const T* kb0 = Kc + c0 * D;
+                const T* vb0 = Vc + c0 * D;
+                uint2 kr[UB], vr[UB];
+#pragma unroll
+                for (int i = 0; i < UB; i++) {
+                    kr[i] = *reinterpret_cast<const uint2*>(kb0 + i * D);
+                    vr[i] = *reinterpret_cast<const uint2*>(vb0 + i * D);
+                }
+#pragma unroll
+                for (int i = 0; i < UB; i++) {
+                    keep_edge(c0 + i);
+                    add_row(kr[i], vr[i]);
+                }
+            }
+            for (; c0 < c_hi; c0++) {
+                const uint2 kr = *reinterpret_cast<const uint2*>(Kc + c0 * D);
+                const uint2 vr = *reinterpret_cast<const uint2*>(Vc + c0 * D);
+                keep_edge(c0);
+                add_row(kr, vr);
+            }
+        }
+    }
+    constexpr int U = (sizeof(T) == 2 && DPL == 4) ? 4 : 8;  // (bf16, d = 128: only the small levels j >= 2 come here)
+    const bool packed = sizeof(T) == 2 && DPL == 4 && j == 1;
+    for (long long c0 = c_lo; c0 < c_hi && !packed; c0 += U) {
         float kb[U][DPL], vb[U][DPL];
 #pragma unroll
         for (int i = 0; i < U; i++) {
@@ -121,12 +154,7 @@ __global__ void __launch_bounds__(256) build_level_kernel(TreeParams p, int j, l
         for (int i = 0; i < U; i++) {
             long long c = c0 + i;
             if (c < c_hi) {
-                if (right_edge && c == c_hi - 1) {
-                    float* pk = p.PK[j] + u * D + lane * DPL;
-                    float* pv = p.PV[j] + u * D + lane * DPL;
-#pragma unroll
-                    for (int e = 0; e < DPL; e++) { pk[e] = ks[e]; pv[e] = vs[e]; }
-                }
+                keep_edge(c);
 #pragma unroll
                 for (int e = 0; e < DPL; e++) { ks[e] = ks[e] + kb[i][e]; vs[e] = vs[e] + vb[i][e]; }
             }
@@ -143,7 +171,6 @@ __global__ void __launch_bounds__(256) build_level_kernel(TreeParams p, int j, l
     for (int e = 0; e < DPL; e++) { vs_out[e] = vs[e]; vm[e] = __fdiv_rn(vs[e], fcnt); }
     store_vec<T, DPL>(v_out, vm);
 
-    float* kmw = km + warp * D;
 #pragma unroll
     for (int e = 0; e < DPL; e++) kmw[lane * DPL + e] = __fdiv_rn(ks[e], fnc);
     __syncwarp();
@@ -171,6 +198,40 @@ __global__ void __launch_bounds__(256) build_level_kernel(TreeParams p, int j, l
     for (int e = 0; e < DPL; e++) y[e] = (y4[0][e] + y4[1][e]) + (y4[2][e] + y4[3][e]);
     T* k_out = reinterpret_cast<T*>(p.K[j]) + (u * p.rows[j] + m) * D + lane * DPL;
     store_vec<T, DPL>(k_out, y);
+    __syncwarp();  // kmw is read by every lane before the warp's next node writes it
+}
+
+// One warp per node of level j; persistent: the grid walks blocks of
+// `nwarps` consecutive nodes of one unit with a grid stride, so each CTA
+// brings the pooler into shared memory once. Recomputes nodes m >= m0 of
+// the tree over L' = len[u] + add tokens, where m0 = 0 for a full build and
+// len[u] / b^j when `add` new tokens were just copied in.
+template <typename T, int D>
+__global__ void __launch_bounds__(256, 2) build_level_kernel(TreeParams p, int j, long long add, int from_len,
+                                                          long long blocks_per_unit) {
+    extern __shared__ __align__(16) unsigned char smem_b[];
+    T* Wt = reinterpret_cast<T*>(smem_b);                          // [D][D], storage type
+    float* km = reinterpret_cast<float*>(smem_b + D * D * sizeof(T));  // [warps][D]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    for (int i = threadIdx.x; i < (int)(D * D * sizeof(T) / 16); i += blockDim.x)
+        reinterpret_cast<uint4*>(Wt)[i] = reinterpret_cast<const uint4*>(p.Wt)[i];
+    __syncthreads();
+
+    const long long total = (long long)p.B * p.H * blocks_per_unit;
+    for (long long blk = blockIdx.x; blk < total; blk += gridDim.x) {
+        const long long u = blk / blocks_per_unit;
+        const long long L = p.len[u] + add;
+        const long long n_j = level_rows(p, j, L);
+        const long long n_prev = level_rows(p, j - 1, L);
+        const long long m0 = from_len ? p.len[u] / p.span[j] : 0;
+        const long long m = m0 + (blk % blocks_per_unit) * nwarps + warp;
+        if (m >= n_j) continue;
+        if (n_j > p.rows[j] || L > p.cap) {
+            if (lane == 0) flag_error(p.err, ERR_SHAPE);
+            continue;
+        }
+        build_node<T, D>(p, j, u, m, L, n_j, n_prev, Wt, km + warp * D, lane);
+    }
 }
 
 // ----------------------------------------------------------- append one
@@ -229,10 +290,25 @@ cudaError_t launch_build_level(const TreeParams& p, int j, long long add, int fr
     static std::atomic<unsigned long long> attr_done{0};
     cudaError_t e = set_smem_limit(kern, (int)smem, attr_done);
     if (e != cudaSuccess) return e;
-    long long gx = (max_nodes + wpb - 1) / wpb;
-    if (gx < 1) gx = 1;
-    dim3 grid((unsigned)gx, (unsigned)(p.B * p.H));
-    kern<<<grid, threads, smem, s>>>(p, j, add, from_len);
+    long long per_unit = (max_nodes + wpb - 1) / wpb;
+    if (per_unit < 1) per_unit = 1;
+    // resident CTAs per SM and SMs, looked up once per device
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int slots = dev < 64 ? cached[dev].load(std::memory_order_relaxed) : 0;
+    if (slots <= 0) {
+        int sms = 148, per_sm = 1;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+        if (e != cudaSuccess) return e;
+        slots = sms * (per_sm < 1 ? 1 : per_sm);
+        if (dev < 64) cached[dev].store(slots, std::memory_order_relaxed);
+    }
+    const long long total = per_unit * p.B * p.H;
+    const long long grid = total < slots ? total : slots;
+    kern<<<(unsigned)grid, threads, smem, s>>>(p, j, add, from_len, per_unit);
     return cudaGetLastError();
 }
 
