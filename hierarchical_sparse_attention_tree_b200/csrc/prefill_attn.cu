@@ -99,8 +99,8 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
     auto sK = [&](int bf) { return sm + LY::OFF_K + bf * LY::KB; };  // double-buffered key tiles
     auto sV = [&](int bf) { return sm + LY::OFF_V + bf * LY::KB; };  // and value tiles
     unsigned char* sP = sm + LY::OFF_P;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + LY::OFF_BAR);  // 0 q, 1-2 k, 3-4 v, 5 s, 6 o, 7 drain
-    uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 8);          // TMEM base address
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + LY::OFF_BAR);  // 0 q, 1-2 k, 3-4 v, 5-6 s, 7 o, 8 drain
+    uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 10);         // TMEM base address
     float* xmax = reinterpret_cast<float*>(tbase + 4);               // [2][128] row maxima of the two halves
     float* xsum = xmax + 2 * PA_T;                                   // [2][128] row sums
 
@@ -112,14 +112,14 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
     const int row = qt * PA_T + rr;  // this thread's query, offset in the chunk
 
     if (tid == 0) {
-        for (int i = 0; i < 8; i++) mbar_init(&bar[i], 1);
+        for (int i = 0; i < 9; i++) mbar_init(&bar[i], 1);
         fence_mbar_init();
         tma_prefetch_map(&mq);
         tma_prefetch_map(&mk);
         tma_prefetch_map(&mv);
     }
     if (warp == 0) {
-        tmem_alloc(tbase, 256);
+        tmem_alloc(tbase, 512);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -127,7 +127,10 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tbase;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;  // warps w and w + 4 share TMEM lanes
-    const uint32_t tS = tmem + lane_off + half * HK, tO = tmem + lane_off + PA_T + half * HDC;
+    // two S buffers (columns [0, 128) and [128, 256)): the product of the
+    // next key tile runs while this tile's softmax does; O in [256, 256 + d)
+    auto tS = [&](int bf) { return tmem + lane_off + bf * PA_T + half * HK; };
+    const uint32_t tO = tmem + lane_off + 2 * PA_T + half * HDC;
     constexpr uint32_t ID_S = idesc_bf16(PA_T, PA_T, 0, 0), ID_O = idesc_bf16(PA_T, D, 0, 1);
     constexpr float LOG2E = 1.4426950408889634f;
     const float sc2 = a.scale * LOG2E;  // logits in log2 units
@@ -153,18 +156,19 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
         if (!mbar_wait(b, waited & 1u)) timeout = true;
         waited++;
     };
-    auto issue_s = [&](int bf) {
+    auto issue_s = [&](int bf) {  // key buffer bf into S buffer bf (tile kt uses buffers kt & 1)
 #pragma unroll
         for (int ks = 0; ks < D / 16; ks++) {
             const uint32_t off = (uint32_t)((ks >> 2) * LY::TILE + (ks & 3) * 32);
-            mma_bf16_ss(tmem, kmajor_desc(smem_addr(sQ) + off), kmajor_desc(smem_addr(sK(bf)) + off), ID_S, ks > 0);
+            mma_bf16_ss(tmem + bf * PA_T, kmajor_desc(smem_addr(sQ) + off), kmajor_desc(smem_addr(sK(bf)) + off),
+                        ID_S, ks > 0);
         }
     };
     auto issue_pv = [&](int bf, bool acc) {
 #pragma unroll
         for (int ks = 0; ks < PA_T / 16; ks++) {
             const uint32_t aoff = (uint32_t)((ks >> 2) * LY::TILE + (ks & 3) * 32);
-            mma_bf16_ss(tmem + PA_T, kmajor_desc(smem_addr(sP) + aoff),
+            mma_bf16_ss(tmem + 2 * PA_T, kmajor_desc(smem_addr(sP) + aoff),
                         mnmajor_desc(smem_addr(sV(bf)) + (uint32_t)ks * 16 * 128, PA_T), ID_O, acc || ks > 0);
         }
     };
@@ -184,25 +188,30 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
         tc_fence_after();
         if (!timeout) issue_s(0);
         mma_commit(&bar[5]);
+        if (nkt > 1) {
+            wait1(&bar[2], k_wt1);
+            tc_fence_after();
+            if (!timeout) issue_s(1);
+            mma_commit(&bar[6]);
+        }
     }
 
     float m_ref = -INFINITY, l = 0.f;  // log2 units
     bool ok = true;
     for (int kt = 0; kt < nkt; kt++) {
         const int bf = kt & 1;
-        // S of this tile is in TMEM
-        int bad = !mbar_wait(&bar[5], (uint32_t)kt & 1u);
+        // S of this tile is in TMEM (S buffer bf, its (kt / 2)-th use)
+        int bad = !mbar_wait(&bar[5 + bf], (uint32_t)(kt >> 1) & 1u);
         if (__syncthreads_or(bad || timeout)) {
             ok = false;
             break;
         }
         tc_fence_after();
-        // S(kt) has completed: the key buffer of tile kt + 1 (it held tile
-        // kt - 1) is free
-        if (tid == 0 && kt >= 1 && kt + 1 < nkt) load_k(kt + 1);
+        // S(kt) has completed: its key buffer takes tile kt + 2
+        if (tid == 0 && kt + 2 < nkt) load_k(kt + 2);
         float s[HK];
 #pragma unroll
-        for (int c = 0; c < HK / 32; c++) tmem_ld32(tS + c * 32, s + c * 32);
+        for (int c = 0; c < HK / 32; c++) tmem_ld32(tS(bf) + c * 32, s + c * 32);
         tmem_wait_ld();
         float mx = -INFINITY;
         if (kt == qt) {  // the diagonal tile: causal mask (and the chunk's end)
@@ -223,7 +232,7 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
         xmax[half * PA_T + rr] = mx;
         // the previous tile's P V product is done: P and O are free, and so
         // is the value buffer of tile kt - 1, which takes tile kt + 1
-        if (kt > 0) bad = !mbar_wait(&bar[6], (uint32_t)(kt - 1) & 1u);
+        if (kt > 0) bad = !mbar_wait(&bar[7], (uint32_t)(kt - 1) & 1u);
         if (__syncthreads_or(bad)) {  // also publishes xmax
             ok = false;
             break;
@@ -274,16 +283,16 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
             tc_fence_after();
             wait1(&bar[3 + bf], bf ? v_wt1 : v_wt0);
             if (!timeout) issue_pv(bf, kt > 0);
-            mma_commit(&bar[6]);
-            if (kt + 1 < nkt) {
-                wait1(&bar[1 + (bf ^ 1)], bf ? k_wt0 : k_wt1);
-                if (!timeout) issue_s(bf ^ 1);
-                mma_commit(&bar[5]);
+            mma_commit(&bar[7]);
+            if (kt + 2 < nkt) {  // every thread has read S(kt): its buffer takes S(kt + 2)
+                wait1(&bar[1 + bf], bf ? k_wt1 : k_wt0);
+                if (!timeout) issue_s(bf);
+                mma_commit(&bar[5 + bf]);
             }
         }
     }
     if (ok) {
-        const int bad = !mbar_wait(&bar[6], (uint32_t)(nkt - 1) & 1u);
+        const int bad = !mbar_wait(&bar[7], (uint32_t)(nkt - 1) & 1u);
         ok = !__syncthreads_or(bad);
     }
     if (ok) {  // every thread loads (TMEM loads are warp-wide); rows past the chunk store nothing
@@ -310,8 +319,8 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
         flag_error(a.err, ERR_TIMEOUT);
         // let every product and copy still in flight finish before the CTA
         // frees its tensor memory and leaves (each wait bounded)
-        mma_commit(&bar[7]);
-        mbar_wait(&bar[7], 0);
+        mma_commit(&bar[8]);
+        mbar_wait(&bar[8], 0);
         while (k_wt0 < k_iss0) wait1(&bar[1], k_wt0);
         while (k_wt1 < k_iss1) wait1(&bar[2], k_wt1);
         while (v_wt0 < v_iss0) wait1(&bar[3], v_wt0);
@@ -319,7 +328,7 @@ __global__ void __launch_bounds__(PA_THREADS, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 256);
+    if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------ tensor maps
