@@ -1,8 +1,8 @@
 // The pieces of one distillation step of the pooler that are not the
 // forward, the gradient or the tree build: the squared-error loss against
 // dense-attention outputs with its gradient, and the plain gradient-descent
-// update of the pooler (RecSA abstract: the pooler is distilled from dense
-// attention).
+// update of the pooler (RecSA abstract: the pooler is trained so that the
+// tree's attention follows dense attention).
 #include <algorithm>
 
 #include "common.cuh"
