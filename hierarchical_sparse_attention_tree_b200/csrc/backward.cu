@@ -101,6 +101,35 @@ __device__ __forceinline__ void add_pairs(float* row, int lane, const float* lo,
     }
 }
 
+// Sums each of V values (V a power of two, at most 32) over the warp with
+// V - 1 + 5 - log2(V) shuffles: each halving step sends half of the values
+// still held and keeps the other half. Returns the sum of value `which`;
+// the lanes whose lowest 5 - log2(V) bits are zero hold distinct values.
+template <int V>
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[V], int lane, int& which) {
+    int cnt = V;
+    which = 0;
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) {
+        if (cnt > 1) {
+            const int half = cnt / 2;
+            const bool hi = (lane & s) != 0;
+#pragma unroll
+            for (int x = 0; x < V / 2; x++)
+                if (x < half) {
+                    const float send = hi ? v[x] : v[x + half];
+                    const float keep = hi ? v[x + half] : v[x];
+                    v[x] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+                }
+            which += hi ? half : 0;
+            cnt = half;
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], s);
+        }
+    }
+    return v[0];
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -386,27 +415,29 @@ __global__ void __launch_bounds__(BWD_THREADS, 2) bwd_score_kernel(TreeParams p,
                 }
                 continue;
             }
+            // <R(P - i) q_g, k> = <q_g, R(i - P) k>: the key is rotated once
             const float* tab = p.rope + (bt.P[t] - bt.i[t]) * 3 * (D / 2);
-            float lgv[G], agv[G];
+            float rkl[NP], rkh[NP];
+            rot_pairs<D>(tab, lane, klo[t], khi[t], true, rkl, rkh);
+            float part[2 * G];  // this lane's share of the G logits, then of the G <dout_g, v>
 #pragma unroll
             for (int g = 0; g < G; g++) {
-                float rl[NP], rh[NP];
-                rot_pairs<D>(tab, lane, v.ql[g], v.qh[g], false, rl, rh);
                 float s = 0.f, w = 0.f;
 #pragma unroll
                 for (int i = 0; i < NP; i++) {
-                    s += rl[i] * klo[t][i] + rh[i] * khi[t][i];
+                    s += v.ql[g][i] * rkl[i] + v.qh[g][i] * rkh[i];
                     w += v.dl[g][i] * vlo[t][i] + v.dh[g][i] * vhi[t][i];
                 }
-                lgv[g] = warp_sum(s) * p.scale;
-                agv[g] = warp_sum(w);
+                part[g] = s;
+                part[G + g] = w;
             }
-            if (lane == 0) {
-#pragma unroll
-                for (int g = 0; g < G; g++) {
-                    lgx[g] = lgv[g];
-                    agx[g] = agv[g];
-                }
+            int which;
+            const float tot = warp_transpose_sum<2 * G>(part, lane, which);
+            if ((lane & (32 / (2 * G) - 1)) == 0) {  // one lane per value
+                if (which < G)
+                    lgx[which] = tot * p.scale;
+                else
+                    agx[which - G] = tot;
             }
         }
         xg += nb;
@@ -552,25 +583,24 @@ __global__ void __launch_bounds__(BWD_THREADS, 2) bwd_entry_kernel(TreeParams p,
                 dlg[g] = pg[g] * (agt[t][g] - st[g][2]);
             }
             const float* tab = p.rope + (bt.P[t] - bt.i[t]) * 3 * (D / 2);
-            float gkl[NP], gkh[NP], gvl[NP], gvh[NP], rkl[NP], rkh[NP];
+            float gkl[NP], gkh[NP], gvl[NP], gvh[NP], rkl[NP], rkh[NP], sql[NP], sqh[NP];
 #pragma unroll
-            for (int i = 0; i < NP; i++) gkl[i] = gkh[i] = gvl[i] = gvh[i] = 0.f;
+            for (int i = 0; i < NP; i++) sql[i] = sqh[i] = gvl[i] = gvh[i] = 0.f;
             rot_pairs<D>(tab, lane, klo[t], khi[t], true, rkl, rkh);  // R(i - P) k
 #pragma unroll
             for (int g = 0; g < G; g++) {
-                float rl[NP], rh[NP];
-                rot_pairs<D>(tab, lane, v.ql[g], v.qh[g], false, rl, rh);  // R(P - i) q
                 const float c = dlg[g] * p.scale;
 #pragma unroll
                 for (int i = 0; i < NP; i++) {
-                    gkl[i] += c * rl[i];
-                    gkh[i] += c * rh[i];
+                    sql[i] += c * v.ql[g][i];  // sum_g c_g q_g, rotated once below
+                    sqh[i] += c * v.qh[g][i];
                     gvl[i] += pg[g] * v.dl[g][i];
                     gvh[i] += pg[g] * v.dh[g][i];
                     aql[g][i] += c * rkl[i];
                     aqh[g][i] += c * rkh[i];
                 }
             }
+            rot_pairs<D>(tab, lane, sql, sqh, false, gkl, gkh);  // R(P - i) sum_g c_g q_g
             float* rk = nullptr;
             float* rv = nullptr;
             if (bt.j[t] >= 1) {
