@@ -161,10 +161,11 @@ __device__ __forceinline__ int rank_in_lists(const unsigned long long* lists, in
 // Thread 0: request rows [r0, r1) of a level's candidate list (the children
 // of the kept parents par[], b per parent, n_j nodes in the level) from the
 // node rows at `base` into dst, one 1D bulk copy per contiguous piece, all
-// counted on one mbarrier. Out-of-range pieces are flagged, not copied. Kept
-// out of line: it runs a few times per launch, on one thread.
+// counted on one mbarrier. Out-of-range pieces are flagged, not copied.
+// (Inline: as an out-of-line call it cost a register spill around every call
+// site and about a microsecond per step.)
 template <typename T, int D>
-__device__ __noinline__ void issue_rows(T* dst, const T* base, const int* par, int n_j, int b, int r0, int r1,
+__device__ __forceinline__ void issue_rows(T* dst, const T* base, const int* par, int n_j, int b, int r0, int r1,
                                         uint64_t* bar, int* err, const DecPages* pg) {
     // pg set (level 0 of a paged cache): base is the pool and each piece
     // (part of one parent's children, which lie in one page) is translated;
@@ -202,7 +203,8 @@ __device__ __noinline__ void issue_rows(T* dst, const T* base, const int* par, i
     }
 }
 
-// The fused step's append, out of line (one copy of its code): appends the
+// The fused step's append (inline: out of line, its call cost the step about
+// a microsecond of register spills and an instruction fetch): appends the
 // token of unit u at position P, leaves the refreshed node of level jf (the
 // first scored level; jf = 0: the token itself) in patch[0..D) (key) and
 // patch[D..2D) (value), and makes its global writes visible to later bulk
@@ -211,7 +213,7 @@ __device__ __noinline__ void issue_rows(T* dst, const T* base, const int* par, i
 // of the block calls it. False if the pooler copy (on wbar, into the start
 // of smem) did not arrive.
 template <typename T, int D>
-__device__ __noinline__ bool fused_append(AppendDims dims, const LevelRef* lv, long long u, long long P, const T* kn,
+__device__ __forceinline__ bool fused_append(AppendDims dims, const LevelRef* lv, long long u, long long P, const T* kn,
                                           const T* vn, unsigned char* smem, T* patch, int jf, uint64_t* wbar,
                                           int* err, bool fence) {
     const int tid = threadIdx.x;
