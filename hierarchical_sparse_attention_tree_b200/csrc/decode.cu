@@ -616,18 +616,18 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
                     if (c < kk) sm->picked[c] = x;
                 }
                 __syncthreads();
+                // the kept ids in ascending order: the next level's parents
                 if (tid < kk) {
                     const int id = (int)key_id(sm->picked[tid]);
                     int pos = 0;
                     for (int r = 0; r < kk; r++) pos += (int)key_id(sm->picked[r]) < id;
                     sm->chosen[pos] = id;
+                    sm->par[pos] = id;  // no one reads this level's parents any more
+                    if (rank == 0 && a.sel_out) a.sel_out[(u * p.J_cap + (j - 1)) * p.k + pos] = id;
                 }
+                if (rank == 0 && a.sel_out)
+                    for (int x = kk + tid; x < p.k; x += DEC_THREADS) a.sel_out[(u * p.J_cap + (j - 1)) * p.k + x] = -1;
                 if (tid == 0) sm->thresh = sm->picked[kk - 1];
-                __syncthreads();
-                if (rank == 0 && a.sel_out)  // not thread 0: it issues the copies
-                    for (int x = tid - 32; x >= 0 && x < p.k; x += DEC_THREADS - 32)
-                        a.sel_out[(u * p.J_cap + (j - 1)) * p.k + x] = x < kk ? sm->chosen[x] : -1;
-                if (tid < kk) sm->par[tid] = sm->chosen[tid];
                 __syncthreads();
                 // the next level's candidates are the children of the kept nodes
                 nc_next = ncand_of(j - 1, kk);
@@ -678,29 +678,30 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(TreeParams p, De
         if (lane == 0) sm->red[warp][g] = s;
     }
     __syncthreads();
+    // Every CTA merges one slice of the output columns: each CTA sends slice r
+    // of its (unnormalised) output, with its maxima and sums, to CTA r (the
+    // gather area has a place of its own: no barrier is needed before it).
+    // Each column's sum over the entry groups goes straight to its CTA.
+    constexpr int SL = G * D / DEC_CLUSTER;  // output columns per CTA
+    constexpr int GST = SL + 2 * G;          // one source's record in the gather area
+    static_assert((G * D) % DEC_CLUSTER == 0, "output slices");
     for (int idx = tid; idx < G * D; idx += DEC_THREADS) {
         float s = 0.f;
 #pragma unroll
         for (int x = 0; x < NEG; x++) s += egacc[x * G * D + idx];
-        cacc[idx] = s;
+        const int r = idx / SL;
+        cluster.map_shared_rank(gat, r)[rank * GST + (idx - r * SL)] = s;
     }
     if (tid < G) {
         float s = 0.f;
 #pragma unroll
         for (int w = 0; w < W; w++) s += sm->red[w][tid];
-        cml[tid] = sm->M[tid];
-        cml[G + tid] = s;
-    }
-    __syncthreads();  // cacc and cml complete
-    // Every CTA merges one slice of the output columns: each CTA sends slice r
-    // of its (unnormalised) output, with its maxima and sums, to CTA r (the
-    // gather area has a place of its own: no barrier is needed before it).
-    constexpr int SL = G * D / DEC_CLUSTER;  // output columns per CTA
-    constexpr int GST = SL + 2 * G;          // one source's record in the gather area
-    static_assert((G * D) % DEC_CLUSTER == 0, "output slices");
-    for (int x = tid; x < CS * GST; x += DEC_THREADS) {
-        const int r = x / GST, i = x - r * GST;
-        cluster.map_shared_rank(gat, r)[rank * GST + i] = i < SL ? cacc[r * SL + i] : cml[i - SL];
+        const float mx = sm->M[tid];
+        for (int r = 0; r < CS; r++) {
+            float* g_r = cluster.map_shared_rank(gat, r) + rank * GST + SL;
+            g_r[tid] = mx;
+            g_r[G + tid] = s;
+        }
     }
     if (chained && !fenced) fence_proxy_async_global();
     cluster.sync();  // every CTA's gather area is complete
