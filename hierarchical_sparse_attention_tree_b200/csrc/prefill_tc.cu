@@ -141,17 +141,29 @@ __global__ void pf_cand_kernel(TreeParams p, PfArgs a, PfLevel L, PfLevel up, in
 }
 
 // Exclusive scans of the bucket sizes (pairs) and of the tiles per bucket,
-// one CTA of 1024 threads, each scanning a contiguous range; also clears
-// the scatter cursors and stores the tile count.
+// one CTA of 1024 threads, each scanning a contiguous range (a multiple of 4
+// buckets, read and written as int4 with every load of the range in flight
+// at once); also clears the scatter cursors and stores the tile count.
 __global__ void __launch_bounds__(1024) pf_scan_kernel(PfLevel L, int n, int TP, int* err) {
     __shared__ int sp[1024], st[1024];
     const int tid = threadIdx.x;
-    const int per = (n + 1023) / 1024, lo = min(n, tid * per), hi = min(n, lo + per);
+    const int per = (((n + 1023) / 1024) + 3) & ~3;
+    const int lo = min(n, tid * per), hi = min(n, lo + per);
+    const int nv = (hi - lo) / 4;  // whole int4 groups (lo is a multiple of 4)
     int cp = 0, ct = 0;
-    for (int i = lo; i < hi; i++) {
-        const int c = L.cnt[i];
-        cp += c;
-        ct += (c + TP - 1) / TP;
+    {
+        const int4* c4 = reinterpret_cast<const int4*>(L.cnt + lo);
+#pragma unroll 8
+        for (int v = 0; v < nv; v++) {
+            const int4 c = c4[v];
+            cp += (c.x + c.y) + (c.z + c.w);
+            ct += (c.x + TP - 1) / TP + (c.y + TP - 1) / TP + (c.z + TP - 1) / TP + (c.w + TP - 1) / TP;
+        }
+        for (int i = lo + 4 * nv; i < hi; i++) {
+            const int c = L.cnt[i];
+            cp += c;
+            ct += (c + TP - 1) / TP;
+        }
     }
     sp[tid] = cp;
     st[tid] = ct;
@@ -164,13 +176,31 @@ __global__ void __launch_bounds__(1024) pf_scan_kernel(PfLevel L, int n, int TP,
         __syncthreads();
     }
     int rp = sp[tid] - cp, rt = st[tid] - ct;
-    for (int i = lo; i < hi; i++) {
-        const int c = L.cnt[i];
-        L.off[i] = rp;
-        L.toff[i] = rt;
-        L.cursor[i] = 0;
-        rp += c;
-        rt += (c + TP - 1) / TP;
+    {
+        const int4* c4 = reinterpret_cast<const int4*>(L.cnt + lo);
+        int4* o4 = reinterpret_cast<int4*>(L.off + lo);
+        int4* t4 = reinterpret_cast<int4*>(L.toff + lo);
+        int4* z4 = reinterpret_cast<int4*>(L.cursor + lo);
+#pragma unroll 4
+        for (int v = 0; v < nv; v++) {
+            const int4 c = c4[v];
+            int4 o, t;
+            o.x = rp; t.x = rt; rp += c.x; rt += (c.x + TP - 1) / TP;
+            o.y = rp; t.y = rt; rp += c.y; rt += (c.y + TP - 1) / TP;
+            o.z = rp; t.z = rt; rp += c.z; rt += (c.z + TP - 1) / TP;
+            o.w = rp; t.w = rt; rp += c.w; rt += (c.w + TP - 1) / TP;
+            o4[v] = o;
+            t4[v] = t;
+            z4[v] = make_int4(0, 0, 0, 0);
+        }
+        for (int i = lo + 4 * nv; i < hi; i++) {
+            const int c = L.cnt[i];
+            L.off[i] = rp;
+            L.toff[i] = rt;
+            L.cursor[i] = 0;
+            rp += c;
+            rt += (c + TP - 1) / TP;
+        }
     }
     if (tid == 1023) {
         const int total = st[1023];
@@ -641,6 +671,60 @@ __device__ __forceinline__ int warp_sum(int n) {
     return n;
 }
 
+// The register path of pf_select_kernel for lists of at most 32 * KPL
+// candidates: KPL scores per lane; the k-th largest found bit by bit on the
+// order-preserving 32-bit keys; keys equal to it taken in index order until
+// k are kept. Returns the number kept (k).
+template <int KPL>
+__device__ __forceinline__ int select_regs(const float* srow, int nc, int k, int lane, const int* par, int b,
+                                           int* kept, int* selrow) {
+    auto cand_id = [&](int i) { return par[i / b] * b + i % b; };
+    int nk = 0;
+    unsigned fk[KPL];
+#pragma unroll
+    for (int x = 0; x < KPL; x++) {
+        const int i = x * 32 + lane;
+        fk[x] = i < nc ? float_key(srow[i]) : 0u;  // 0: below every real key
+    }
+    unsigned thr = 0u;
+    for (int bit = 31; bit >= 0; bit--) {
+        const unsigned c = thr | (1u << bit);
+        int n = 0;
+#pragma unroll
+        for (int x = 0; x < KPL; x++) n += fk[x] >= c;
+        if (warp_sum(n) >= k) thr = c;
+    }
+    int gt = 0;
+#pragma unroll
+    for (int x = 0; x < KPL; x++) gt += fk[x] > thr;
+    int need_eq = k - warp_sum(gt);  // keys equal to the k-th score, smallest indices first
+#pragma unroll
+    for (int x = 0; x < KPL; x++) {
+        const int i = x * 32 + lane;
+        const unsigned meq = __ballot_sync(0xffffffffu, i < nc && fk[x] == thr);
+        const unsigned take = need_eq <= 0 ? 0u : (__popc(meq) <= need_eq ? meq : [&]() {
+            unsigned m = meq, r = 0u;
+            for (int c = 0; c < need_eq; c++) {
+                const unsigned low = m & (~m + 1u);
+                r |= low;
+                m ^= low;
+            }
+            return r;
+        }());
+        need_eq -= __popc(take);
+        const bool in = i < nc && (fk[x] > thr || ((take >> lane) & 1u));
+        const unsigned m = __ballot_sync(0xffffffffu, in);
+        if (in) {
+            const int pos = nk + __popc(m & ((1u << lane) - 1u));
+            const int id = cand_id(i);
+            kept[pos] = id;
+            if (selrow) selrow[pos] = id;
+        }
+        nk += __popc(m);
+    }
+    return nk;
+}
+
 __global__ void __launch_bounds__(SEL_WARPS * 32) pf_select_kernel(TreeParams p, PfArgs a, PfLevel L, PfLevel up,
                                                                    int j) {
     extern __shared__ unsigned long long skeys[];  // [SEL_WARPS][maxc] when maxc > 32 * SEL_KPL
@@ -678,49 +762,16 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) pf_select_kernel(TreeParams p,
     }
     const float* srow = a.S + idx * (long long)a.maxc;
     int nk = 0;  // kept so far (uniform)
-    if (nc <= 32 * SEL_KPL) {
-        unsigned fk[SEL_KPL];
-#pragma unroll
-        for (int x = 0; x < SEL_KPL; x++) {
-            const int i = x * 32 + lane;
-            fk[x] = i < nc ? float_key(srow[i]) : 0u;  // 0: below every real key
-        }
-        unsigned thr = 0u;
-        for (int bit = 31; bit >= 0; bit--) {
-            const unsigned c = thr | (1u << bit);
-            int n = 0;
-#pragma unroll
-            for (int x = 0; x < SEL_KPL; x++) n += fk[x] >= c;
-            if (warp_sum(n) >= k) thr = c;
-        }
-        int gt = 0;
-#pragma unroll
-        for (int x = 0; x < SEL_KPL; x++) gt += fk[x] > thr;
-        int need_eq = k - warp_sum(gt);  // keys equal to the k-th score, smallest indices first
-#pragma unroll
-        for (int x = 0; x < SEL_KPL; x++) {
-            const int i = x * 32 + lane;
-            const unsigned meq = __ballot_sync(0xffffffffu, i < nc && fk[x] == thr);
-            const unsigned take = need_eq <= 0 ? 0u : (__popc(meq) <= need_eq ? meq : [&]() {
-                unsigned m = meq, r = 0u;
-                for (int c = 0; c < need_eq; c++) {
-                    const unsigned low = m & (~m + 1u);
-                    r |= low;
-                    m ^= low;
-                }
-                return r;
-            }());
-            need_eq -= __popc(take);
-            const bool in = i < nc && (fk[x] > thr || ((take >> lane) & 1u));
-            const unsigned m = __ballot_sync(0xffffffffu, in);
-            if (in) {
-                const int pos = nk + __popc(m & ((1u << lane) - 1u));
-                const int id = cand_id(i);
-                kept[pos] = id;
-                if (selrow) selrow[pos] = id;
-            }
-            nk += __popc(m);
-        }
+    if (nc <= 32 * SEL_KPL) {  // as many registers per lane as the list needs
+        const int kpl = (nc + 31) / 32;
+        if (kpl <= 4)
+            nk = select_regs<4>(srow, nc, k, lane, par, b, kept, selrow);
+        else if (kpl <= 8)
+            nk = select_regs<8>(srow, nc, k, lane, par, b, kept, selrow);
+        else if (kpl <= 16)
+            nk = select_regs<16>(srow, nc, k, lane, par, b, kept, selrow);
+        else
+            nk = select_regs<SEL_KPL>(srow, nc, k, lane, par, b, kept, selrow);
     } else {
         unsigned long long* key = skeys + (long long)warp * a.maxc;
         for (int i = lane; i < nc; i += 32)
