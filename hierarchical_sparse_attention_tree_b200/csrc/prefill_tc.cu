@@ -725,10 +725,91 @@ __device__ __forceinline__ int select_regs(const float* srow, int nc, int k, int
     return nk;
 }
 
+// Larger lists (more than 128 candidates, k <= 32): a threshold T0 = the
+// k-th largest of the 32 lane maxima bounds the k-th largest key from below
+// (at least k keys, those maxima, are >= T0), so every key of the result,
+// ties included, is >= T0. Those keys are packed in index order into the
+// warp's shared buffers (usually a few dozen), and the same bitwise search
+// and tie rule as select_regs run over them only. The result is exactly
+// select_regs's.
+template <int KPL>
+__device__ __forceinline__ int select_compact(const float* srow, int nc, int k, int lane, const int* par, int b,
+                                              int* kept, int* selrow, unsigned* ckey, int* cidx) {
+    auto cand_id = [&](int i) { return par[i / b] * b + i % b; };
+    unsigned fk[KPL];
+    unsigned lm = 0u;
+#pragma unroll
+    for (int x = 0; x < KPL; x++) {
+        const int i = x * 32 + lane;
+        fk[x] = i < nc ? float_key(srow[i]) : 0u;
+        lm = fk[x] > lm ? fk[x] : lm;
+    }
+    // T0: the k-th largest lane maximum (bit by bit over one value per lane)
+    unsigned t0 = 0u;
+    for (int bit = 31; bit >= 0; bit--) {
+        const unsigned c = t0 | (1u << bit);
+        if (__popc(__ballot_sync(0xffffffffu, lm >= c)) >= k) t0 = c;
+    }
+    // the keys >= T0, in index order
+    int m = 0;
+#pragma unroll
+    for (int x = 0; x < KPL; x++) {
+        const int i = x * 32 + lane;
+        const bool in = i < nc && fk[x] >= t0;
+        const unsigned bm = __ballot_sync(0xffffffffu, in);
+        if (in) {
+            const int pos = m + __popc(bm & ((1u << lane) - 1u));
+            ckey[pos] = fk[x];
+            cidx[pos] = i;
+        }
+        m += __popc(bm);
+    }
+    __syncwarp();
+    unsigned thr = 0u;
+    for (int bit = 31; bit >= 0; bit--) {
+        const unsigned c = thr | (1u << bit);
+        int n = 0;
+        for (int y = lane; y < m; y += 32) n += ckey[y] >= c;
+        if (warp_sum(n) >= k) thr = c;
+    }
+    int gt = 0;
+    for (int y = lane; y < m; y += 32) gt += ckey[y] > thr;
+    int need_eq = k - warp_sum(gt);
+    int nk = 0;
+    for (int y0 = 0; y0 < m; y0 += 32) {
+        const int y = y0 + lane;
+        const unsigned key = y < m ? ckey[y] : 0u;
+        const unsigned meq = __ballot_sync(0xffffffffu, y < m && key == thr);
+        const unsigned take = need_eq <= 0 ? 0u : (__popc(meq) <= need_eq ? meq : [&]() {
+            unsigned mm = meq, r = 0u;
+            for (int c = 0; c < need_eq; c++) {
+                const unsigned low = mm & (~mm + 1u);
+                r |= low;
+                mm ^= low;
+            }
+            return r;
+        }());
+        need_eq -= __popc(take);
+        const bool in = y < m && (key > thr || ((take >> lane) & 1u));
+        const unsigned bm = __ballot_sync(0xffffffffu, in);
+        if (in) {
+            const int pos = nk + __popc(bm & ((1u << lane) - 1u));
+            const int id = cand_id(cidx[y]);
+            kept[pos] = id;
+            if (selrow) selrow[pos] = id;
+        }
+        nk += __popc(bm);
+    }
+    __syncwarp();  // the buffers are free for the warp's next list
+    return nk;
+}
+
 __global__ void __launch_bounds__(SEL_WARPS * 32) pf_select_kernel(TreeParams p, PfArgs a, PfLevel L, PfLevel up,
                                                                    int j) {
     extern __shared__ unsigned long long skeys[];  // [SEL_WARPS][maxc] when maxc > 32 * SEL_KPL
     __shared__ int sids[SEL_WARPS][TP_KMAX];
+    __shared__ unsigned ckey[SEL_WARPS][32 * SEL_KPL];  // select_compact's packed keys and indices
+    __shared__ int cidx[SEL_WARPS][32 * SEL_KPL];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long idx = blockIdx.x * (long long)SEL_WARPS + warp;
     const long long U = (long long)p.B * p.H;
@@ -766,12 +847,14 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) pf_select_kernel(TreeParams p,
         const int kpl = (nc + 31) / 32;
         if (kpl <= 4)
             nk = select_regs<4>(srow, nc, k, lane, par, b, kept, selrow);
-        else if (kpl <= 8)
-            nk = select_regs<8>(srow, nc, k, lane, par, b, kept, selrow);
-        else if (kpl <= 16)
-            nk = select_regs<16>(srow, nc, k, lane, par, b, kept, selrow);
-        else
+        else if (k > 32)
             nk = select_regs<SEL_KPL>(srow, nc, k, lane, par, b, kept, selrow);
+        else if (kpl <= 8)
+            nk = select_compact<8>(srow, nc, k, lane, par, b, kept, selrow, ckey[warp], cidx[warp]);
+        else if (kpl <= 16)
+            nk = select_compact<16>(srow, nc, k, lane, par, b, kept, selrow, ckey[warp], cidx[warp]);
+        else
+            nk = select_compact<SEL_KPL>(srow, nc, k, lane, par, b, kept, selrow, ckey[warp], cidx[warp]);
     } else {
         unsigned long long* key = skeys + (long long)warp * a.maxc;
         for (int i = lane; i < nc; i += 32)
