@@ -126,3 +126,15 @@ def test_prefill_131k_sampled():
                                      max_chunks_checked={0, 1, 31})
     parity.record("test_prefill_131k_sampled", w.name, "staged", rep)
     assert rep["checked"] >= 40, rep
+
+
+@pytest.mark.parametrize("k", [16, 40])
+def test_prefill_selection_paths(k):
+    """b = 64 over trees of 12K to 65K tokens: level-1 candidate lists of about
+    190, 320, 640 and 1024 (the selection's 8, 16 and 32 keys-per-lane paths,
+    and, with k = 40 > 32, the register path without the lane-maximum cut)."""
+    w = small(batch=1, n_kv_heads=2, group=4, head_dim=128, branching=64, k=k)
+    _, _, _, _, _, rep = run_prefill(w, 17 * 4096, 4096, lambda ci, C: [0, 1, 2047, C - 1],
+                                     max_chunks_checked={3, 5, 10, 16})
+    parity.record("test_prefill_selection_paths", f"bf16 69632 tokens, chunks of 4096, b=64 k={k}", "staged", rep)
+    assert rep["checked"] >= 24, rep
