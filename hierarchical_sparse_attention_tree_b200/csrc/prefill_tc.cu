@@ -417,12 +417,29 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
     const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(p.V[j]);
     const long long ustride = j == 0 ? p.cap : p.rows[j];
     const int pr = tid / G, g = tid % G;  // this thread's row: pair pr, head g
+    // Each tile's descriptor, its unit's length, this thread's pair and the
+    // pair's candidate count are loaded one tile ahead (a chain of dependent
+    // loads that then overlaps the previous tile's products).
+    int4 tile_n = make_int4(0, 0, 0, 0);
+    long long S_n = 0;
+    int pk_n = 0, nc_n = 0;
+    if ((int)blockIdx.x < ntiles) {
+        tile_n = L.tiles[blockIdx.x];
+        S_n = p.len[tile_n.x];
+        if (pr < tile_n.w) {
+            pk_n = L.pairs[tile_n.z + pr];
+            nc_n = L.nc[tile_n.x * a.C + (pk_n >> 6)];
+        }
+    }
     for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x) {
-        const int4 tile = L.tiles[ti];
+        const int4 tile = tile_n;
         const long long u = tile.x;
         const int par = tile.y, first = tile.z, npairs = tile.w;
         const int bseq = (int)(u / p.H), h = (int)(u % p.H);
-        const long long S = p.len[u];
+        const long long S = S_n;
+        const int pk_cur = pk_n, nc_cur = nc_n;
+        const bool has_next = ti + (int)gridDim.x < ntiles;
+        if (has_next) tile_n = L.tiles[ti + gridDim.x];
         const long long n_j = j == 0 ? S : ceil_div_ll(S, p.span[j]);
         const int nchild = (int)min((long long)b, n_j - (long long)par * b);
         // first child row (a page of tokens at level 0 of a paged cache)
@@ -430,12 +447,11 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
         const bool valid = pr < npairs;
         int t = 0, r = 0, P = -1;
         if (valid) {
-            const int pk = L.pairs[first + pr];
-            t = pk >> 6;
-            r = pk & 63;
-            const int nc = L.nc[u * a.C + t];
-            P = (j == 0 ? nc + t : nc - 1) - r * b;  // the query's angle for this parent's block
+            t = pk_cur >> 6;
+            r = pk_cur & 63;
+            P = (j == 0 ? nc_cur + t : nc_cur - 1) - r * b;  // the query's angle for this parent's block
         }
+        (void)first;
         const int hq = h * G + g;
         const long long orow = ((long long)bseq * a.C + t) * a.Hq + hq;  // (sequence, token, head)
         const bool qok = valid && P >= 0 && P < p.npos;
@@ -470,13 +486,16 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
                     *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
             }
         }
-        // the next tile's child rows into L2 while this one is computed
-        if (ti + (int)gridDim.x < ntiles) {
-            const int4 nt = L.tiles[ti + gridDim.x];
+        // the next tile's child rows into L2 while this one is computed, and
+        // the next links of its metadata chain
+        if (has_next) {
+            const int4 nt = tile_n;
             const long long nrow = j == 0 ? token_row(token_map(p), nt.x, (long long)nt.y * b)
                                           : (long long)nt.x * ustride + (long long)nt.y * b;
             if (tid * 64 < b * D) prefetch_l2(kb + nrow * D + tid * 64);
             if (MODE == MODE_VALUE && tid * 64 < b * D) prefetch_l2(vb + nrow * D + tid * 64);
+            S_n = p.len[nt.x];
+            pk_n = pr < nt.w ? L.pairs[nt.z + pr] : 0;
         }
         // ---- operands: the rotated query and keys, split hi / lo
         // (the largest-logit pass of the tokens needs only an approximate
@@ -503,6 +522,7 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
             const uint4 z = make_uint4(0, 0, 0, 0);
             put_chunk<D, LO>(o < nchild ? ka[x] : z, o < nchild ? kbv[x] : z, cs, c * 8, sBh, sBl, o, NB);
         }
+        if (has_next && pr < tile_n.w) nc_n = L.nc[tile_n.x * a.C + (pk_n >> 6)];
         if (MODE == MODE_VALUE) cp_async_wait_all();
         fence_proxy_async_shared();
         tc_fence_before();
