@@ -28,7 +28,7 @@ struct ScoreLayout {
     static constexpr int P2 = PL / 2;
     static constexpr int LPC = HD / PL;
     static constexpr int CPW = 32 / LPC;
-    static constexpr int NC = G >= 8 ? 2 : (LPC / G >= 4 ? 4 : LPC / G);  // candidates per group and step
+    static constexpr int NC = 2;  // candidates per group and step (more made the step slower: code size, spills)
     static_assert(G <= LPC && 32 % LPC == 0 && G <= 8, "scoring layout");
 };
 
