@@ -604,10 +604,11 @@ recsa_status recsa_dense_decode_static(const void* k_cache, const void* v_cache,
 namespace {
 // Backward scratch: [node-key accumulators, levels 1..J_cap][node-value
 // accumulators, levels 1..J_cap] (fp32, [B*H][rows[j]][d] each; the prefix
-// the tree pass clears) then the per-call plan, logits, <dout, v> and
-// softmax statistics.
+// the tree pass clears) then W^T h per node of levels 2..J_cap (written
+// before it is read), the per-call plan, logits, <dout, v> and softmax
+// statistics.
 struct BwdLayout {
-    size_t gK[MAXJ + 1], gV[MAXJ + 1], nodes_end, plan, ubase, lg, ag, st, total;
+    size_t gK[MAXJ + 1], gV[MAXJ + 1], gW[MAXJ + 1], nodes_end, plan, ubase, lg, ag, st, total;
     int E_cap;
 };
 BwdLayout bwd_layout(const recsa_config* c) {
@@ -619,6 +620,7 @@ BwdLayout bwd_layout(const recsa_config* c) {
     for (int j = 1; j <= l.J_cap; j++) { b.gK[j] = o; o = align256(o + units * (size_t)l.rows[j] * D * 4); }
     for (int j = 1; j <= l.J_cap; j++) { b.gV[j] = o; o = align256(o + units * (size_t)l.rows[j] * D * 4); }
     b.nodes_end = o;
+    for (int j = 2; j <= l.J_cap; j++) { b.gW[j] = o; o = align256(o + units * (size_t)l.rows[j] * D * 4); }
     long long maxc = (long long)c->k * c->branching;
     if (maxc < c->branching) maxc = c->branching;
     b.E_cap = (int)((l.J_cap + 1) * maxc);
@@ -637,6 +639,7 @@ BwdArgs bwd_args(const recsa_ctx* ctx, void* scratch) {
     for (int j = 1; j <= ctx->p.J_cap; j++) {
         a.gK[j] = reinterpret_cast<float*>(base + l.gK[j]);
         a.gV[j] = reinterpret_cast<float*>(base + l.gV[j]);
+        if (j >= 2) a.gW[j] = reinterpret_cast<float*>(base + l.gW[j]);
     }
     a.plan = reinterpret_cast<int*>(base + l.plan);
     a.ubase = reinterpret_cast<int*>(base + l.ubase);

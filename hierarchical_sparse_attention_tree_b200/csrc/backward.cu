@@ -631,6 +631,8 @@ struct PropSmem {
     float dw[D * D];
     float g[BWD_NODES_PER_PASS][D];
     float mean[BWD_NODES_PER_PASS][D];
+    float hp[D];    // a shared parent's h (pairs layout), for dW
+    float msum[D];  // the pass's means summed
     T W[D * D];
 };
 
@@ -661,6 +663,46 @@ __device__ __forceinline__ void accumulate_dw(PropSmem<T, D>& sm, int tid) {
             acc.y += gr[w] * mv.y;
             acc.z += gr[w] * mv.z;
             acc.w += gr[w] * mv.w;
+        }
+        dst[c] = acc;
+    }
+}
+
+// The same when the pass's nodes share one parent: g_m = own_m + hp for
+// every node, so sum_m g_m mean_m^T = hp msum^T + sum_m own_m mean_m^T, and
+// the own rows (sm.g) are zero but for the nodes that were entries.
+template <typename T, int D>
+__device__ __forceinline__ void accumulate_dw_shared(PropSmem<T, D>& sm, int tid) {
+    constexpr int CW = D * D / BWD_THREADS;
+    const int r = tid % D, cb = tid / D;
+    const float hr = sm.hp[r];
+    float gr[BWD_NODES_PER_PASS];
+    bool any = false;
+#pragma unroll
+    for (int w = 0; w < BWD_NODES_PER_PASS; w++) {
+        gr[w] = sm.g[w][r];
+        any |= gr[w] != 0.f;
+    }
+    if (!any && hr == 0.f) return;
+    float4* dst = reinterpret_cast<float4*>(&sm.dw[r * D + cb * CW]);
+#pragma unroll 4
+    for (int c = 0; c < CW / 4; c++) {
+        float4 acc = dst[c];
+        const float4 ms = reinterpret_cast<const float4*>(&sm.msum[cb * CW])[c];
+        acc.x += hr * ms.x;
+        acc.y += hr * ms.y;
+        acc.z += hr * ms.z;
+        acc.w += hr * ms.w;
+        if (any) {
+#pragma unroll
+            for (int w = 0; w < BWD_NODES_PER_PASS; w++) {
+                if (gr[w] == 0.f) continue;
+                const float4 mv = reinterpret_cast<const float4*>(&sm.mean[w][cb * CW])[c];
+                acc.x += gr[w] * mv.x;
+                acc.y += gr[w] * mv.y;
+                acc.z += gr[w] * mv.z;
+                acc.w += gr[w] * mv.w;
+            }
         }
         dst[c] = acc;
     }
@@ -717,13 +759,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 2)
     const long long total = (long long)p.B * p.H * chunks_per_unit;
     for (long long ch = blockIdx.x; ch < total; ch += gridDim.x) {
         const long long u = ch / chunks_per_unit;
-        const long long m = (ch % chunks_per_unit) * BWD_NODES_PER_PASS + warp;
+        const long long m0 = (ch % chunks_per_unit) * BWD_NODES_PER_PASS;
+        const long long m = m0 + warp;
         const long long L = p.len[u];
         const bool live = L >= 1 && m < level_rows(p, j, L);
+        // every node of the pass under one parent (or none, at the top): its
+        // W^T h comes precomputed, and dW takes one outer product for it
+        const bool shared = top || (m0 / p.b == (m0 + BWD_NODES_PER_PASS - 1) / p.b);
         __syncthreads();  // W loaded / the previous pass's staged rows consumed
-        float glo[NP], ghi[NP], slo[NP], shi[NP];
+        float glo[NP], ghi[NP], slo[NP], shi[NP], plo[NP], phi[NP], wlo[NP], whi[NP];
 #pragma unroll
-        for (int i = 0; i < NP; i++) glo[i] = ghi[i] = slo[i] = shi[i] = 0.f;
+        for (int i = 0; i < NP; i++) glo[i] = ghi[i] = slo[i] = shi[i] = plo[i] = phi[i] = wlo[i] = whi[i] = 0.f;
         long long nch = 1;
         if (live) {
             load_pairs<float, D>(a.gK[j] + (u * p.rows[j] + m) * D, lane, glo, ghi);
@@ -734,31 +780,65 @@ __global__ void __launch_bounds__(BWD_THREADS, 2)
                 slo[i] *= inv_t;
                 shi[i] *= inv_t;
             }
-            if (!top) {  // the parent's h and s (already propagated)
+            if (!top) {  // the parent's h and s (already propagated), and W^T h
                 const long long par = (u * p.rows[j + 1] + m / p.b) * D;
-                float hl[NP], hh[NP], sl[NP], sh[NP];
-                load_pairs<float, D>(a.gK[j + 1] + par, lane, hl, hh);
+                float sl[NP], sh[NP];
+                load_pairs<float, D>(a.gK[j + 1] + par, lane, plo, phi);
                 load_pairs<float, D>(a.gV[j + 1] + par, lane, sl, sh);
+                if (shared) load_pairs<float, D>(a.gW[j + 1] + par, lane, wlo, whi);
 #pragma unroll
                 for (int i = 0; i < NP; i++) {
-                    glo[i] += hl[i];
-                    ghi[i] += hh[i];
                     slo[i] += sl[i];
                     shi[i] += sh[i];
                 }
             }
             nch = n_children(p, j, m, L);
         }
-        store_pairs<D>(sm.g[warp], lane, glo, ghi);
+        if (!shared) {  // g = own + parent h, staged whole
+#pragma unroll
+            for (int i = 0; i < NP; i++) {
+                glo[i] += plo[i];
+                ghi[i] += phi[i];
+            }
+        }
+        store_pairs<D>(sm.g[warp], lane, glo, ghi);  // shared: the own part only (zero unless an entry)
+        if (shared && warp == 0) store_pairs<D>(sm.hp, lane, plo, phi);
         __syncwarp();
         float mlo[NP], mhi[NP];
 #pragma unroll
         for (int i = 0; i < NP; i++) mlo[i] = mhi[i] = 0.f;
         bool mean_staged = false;  // the token branch writes the mean row itself
         if (live) {
+            const float inv_c = 1.f / (float)nch;
             float hlo[NP], hhi[NP];
-            wt_times<T, D>(sm, sm.g[warp], lane, 1.f / (float)nch, hlo, hhi);
+            bool own = true;
+            if (shared) {
+                bool nz = false;
+#pragma unroll
+                for (int i = 0; i < NP; i++) nz |= glo[i] != 0.f || ghi[i] != 0.f;
+                own = __any_sync(0xffffffffu, nz);
+            }
+            if (own) {
+                wt_times<T, D>(sm, sm.g[warp], lane, 1.f, hlo, hhi);
+            } else {
+#pragma unroll
+                for (int i = 0; i < NP; i++) hlo[i] = hhi[i] = 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < NP; i++) {  // h = (W^T g) / children, W^T g = W^T own + W^T h_parent
+                hlo[i] = (hlo[i] + wlo[i]) * inv_c;
+                hhi[i] = (hhi[i] + whi[i]) * inv_c;
+            }
             if (j > 1) {
+                // W^T h for this node's children (their shared-parent passes),
+                // through the warp's mean row, which is free until the mean
+                float* stage = sm.mean[warp];
+                store_pairs<D>(stage, lane, hlo, hhi);
+                __syncwarp();
+                float xlo[NP], xhi[NP];
+                wt_times<T, D>(sm, stage, lane, 1.f, xlo, xhi);
+                __syncwarp();
+                store_pairs<D>(a.gW[j] + (u * p.rows[j] + m) * D, lane, xlo, xhi);
                 // mean of the stored child keys, then h and s in place for the children
                 const T* kb = reinterpret_cast<const T*>(p.K[j - 1]) + (u * p.rows[j - 1] + m * p.b) * D;
 #pragma unroll 8
@@ -850,7 +930,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 2)
                 for (int e = 0; e < E; e++) stage[lane * E + e] = mc[e] * inv_n;
                 mean_staged = true;
             }
-            const float inv_c = 1.f / (float)nch;
 #pragma unroll
             for (int i = 0; i < NP; i++) {
                 mlo[i] *= inv_c;
@@ -859,7 +938,18 @@ __global__ void __launch_bounds__(BWD_THREADS, 2)
         }
         if (!mean_staged) store_pairs<D>(sm.mean[warp], lane, mlo, mhi);
         __syncthreads();
-        accumulate_dw<T, D>(sm, tid);
+        if (shared) {
+            for (int c = tid; c < D; c += BWD_THREADS) {
+                float t = 0.f;
+#pragma unroll
+                for (int w = 0; w < BWD_NODES_PER_PASS; w++) t += sm.mean[w][c];
+                sm.msum[c] = t;
+            }
+            __syncthreads();
+            accumulate_dw_shared<T, D>(sm, tid);
+        } else {
+            accumulate_dw<T, D>(sm, tid);
+        }
     }
     __syncthreads();
     for (int i = tid; i < D * D; i += BWD_THREADS)

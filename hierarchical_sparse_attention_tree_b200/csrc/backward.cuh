@@ -18,6 +18,7 @@ struct BwdArgs {
     float* dw;         // [D][D], dW[r][c] for W[r][c]
     float* gK[MAXJ + 1];  // node-key gradient accumulators [B*H][rows[j]][D] (j >= 1)
     float* gV[MAXJ + 1];  // node-value gradient accumulators
+    float* gW[MAXJ + 1];  // W^T h per node of levels 2..J_cap (the tree pass writes, then reads it)
     int* plan;         // [B*H][PLAN_INTS]
     int* ubase;        // [B*H + 1] first item of each unit in the list of all units' items
     float* lg;         // [B*H][E_cap][G] logits (-inf: not an entry)

@@ -115,6 +115,27 @@ def test_decode_backward_matches_oracle(bf16, D, G):
     _check_layer(layer, w, K, V, synth.as_f32(Wp), lengths, [(q_np, dout_np, gsel, parity.to_f64(dq))])
 
 
+@pytest.mark.parametrize("bf16,D,b", [(True, 128, 5), (False, 64, 12), (True, 64, 3)])
+def test_backward_mixed_parents_matches_oracle(bf16, D, b):
+    """Branching factors that are not multiples of the propagation's
+    eight-node pass: passes whose nodes have different parents (the general
+    path) next to passes under one parent (the shared path), on every level."""
+    w = small(batch=2, n_kv_heads=2, group=4, head_dim=D, branching=b, k=3, bf16=bf16)
+    lengths = [777, 2050]
+    K, V, runs = synth.cache_arrays(w, max(lengths))
+    layer, Wp = make_layer(w, 4096)
+    layer.load(parity.to_dev(K, bf16), parity.to_dev(V, bf16), lengths)
+    q_np = per_seq_queries(w, runs, 0, lengths)
+    _, gsel, _ = run_decode(layer, w, q_np)
+    dout_np = _dout(w, 2)
+    layer.zero_grad()
+    dq = layer.decode_backward(parity.to_dev(q_np, bf16), parity.to_dev(dout_np, bf16), torch.from_numpy(gsel).cuda())
+    layer.tree_backward()
+    torch.cuda.synchronize()
+    layer.check()
+    _check_layer(layer, w, K, V, synth.as_f32(Wp), lengths, [(q_np, dout_np, gsel, parity.to_f64(dq))])
+
+
 def test_backward_sums_queries_and_clears_accumulators():
     """Two queries back-propagated before one tree pass give the sum of their
     gradients; a second tree pass adds nothing (the accumulators were cleared)."""

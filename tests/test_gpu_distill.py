@@ -70,9 +70,9 @@ def oracle_step(layer, w, K, V, Wf, lengths, q_np, target, trees):
     return loss, dW
 
 
-@pytest.mark.parametrize("bf16,D", [(False, 64), (True, 128)])
-def test_distill_step_matches_oracle_and_rebuild(bf16, D):
-    w = small(batch=2, n_kv_heads=2, group=4, head_dim=D, branching=8, k=3, bf16=bf16)
+@pytest.mark.parametrize("bf16,D,b", [(False, 64, 8), (True, 128, 8), (True, 128, 5)])
+def test_distill_step_matches_oracle_and_rebuild(bf16, D, b):
+    w = small(batch=2, n_kv_heads=2, group=4, head_dim=D, branching=b, k=3, bf16=bf16)
     lengths = [600, 1500]
     K, V, runs = synth.cache_arrays(w, max(lengths))
     layer, Wp = make_layer(w, 2048)
