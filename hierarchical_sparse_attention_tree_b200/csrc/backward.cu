@@ -101,6 +101,99 @@ __device__ __forceinline__ void add_pairs(float* row, int lane, const float* lo,
     }
 }
 
+// Eight consecutive floats in one 256-bit access (sm_100); the address must
+// be 32-byte aligned.
+__device__ __forceinline__ void ld8f(const float* p, float* r) {
+    asm volatile("ld.global.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]), "=f"(r[7])
+                 : "l"(p));
+}
+__device__ __forceinline__ void st8f(float* p, const float* v) {
+    asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(v[0]), "f"(v[1]),
+                 "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+                 : "memory");
+}
+
+// The level-1 sweep over one node's nch tokens (rows row0 .. row0 + nch - 1,
+// contiguous): dk += h, dv += s for every token, and the sum of the tokens'
+// keys returned in mc (this lane's eight columns). Each lane takes eight
+// consecutive columns of a row, so a warp covers 32 / (D / 8) rows per
+// access, with 256-bit loads and stores of dk and dv (32-byte aligned rows;
+// the key rows aligned to eight elements). bf16 keys stay packed until they
+// are added. hc, sc: h and s at this lane's columns.
+template <typename T, int D>
+__device__ __forceinline__ void sweep_tokens_v8(const T* K0, float* dk, float* dv, long long row0, long long nch,
+                                                int lane, const float* hc, const float* sc, float* mc) {
+    constexpr bool PACKED = sizeof(T) == 2;
+    constexpr int LPR = D / 8, RPI = 32 / LPR;    // lanes per row, rows per access
+    constexpr int UR = PACKED ? 4 : 3;            // accesses in flight per lane and array
+    constexpr int KW = PACKED ? 4 : 8;            // 32-bit words of one lane's key piece
+    const int rsub = lane / LPR, col = (lane % LPR) * 8;
+    const T* kp = K0 + (row0 + rsub) * D + col;
+    float* dkp = dk + (row0 + rsub) * D + col;
+    float* dvp = dv + (row0 + rsub) * D + col;
+#pragma unroll
+    for (int e = 0; e < 8; e++) mc[e] = 0.f;
+    auto add_row = [&](const uint32_t* kw, float* xx, float* yy) {
+#pragma unroll
+        for (int e = 0; e < 8; e++) {
+            mc[e] += PACKED ? __uint_as_float(e & 1 ? kw[e / 2] & 0xFFFF0000u : kw[e / 2] << 16)
+                            : __uint_as_float(kw[e]);
+            xx[e] += hc[e];
+            yy[e] += sc[e];
+        }
+    };
+    auto load_key = [&](const T* src, uint32_t* kw) {
+        if constexpr (PACKED) {
+            const uint4 v = *reinterpret_cast<const uint4*>(src);
+            kw[0] = v.x;
+            kw[1] = v.y;
+            kw[2] = v.z;
+            kw[3] = v.w;
+        } else {
+            float t8[8];
+            ld8f(reinterpret_cast<const float*>(src), t8);
+#pragma unroll
+            for (int e = 0; e < 8; e++) kw[e] = __float_as_uint(t8[e]);
+        }
+    };
+    constexpr int STEP = RPI * UR;
+    long long c = rsub;
+    // whole groups: every row of the UR accesses exists
+    for (; c + (UR - 1) * RPI < nch; c += STEP, kp += STEP * D, dkp += STEP * D, dvp += STEP * D) {
+        uint32_t kw[UR][KW];
+        float xx[UR][8], yy[UR][8];
+#pragma unroll
+        for (int x = 0; x < UR; x++) {
+            load_key(kp + x * RPI * D, kw[x]);
+            ld8f(dkp + x * RPI * D, xx[x]);
+            ld8f(dvp + x * RPI * D, yy[x]);
+        }
+#pragma unroll
+        for (int x = 0; x < UR; x++) {
+            add_row(kw[x], xx[x], yy[x]);
+            st8f(dkp + x * RPI * D, xx[x]);
+            st8f(dvp + x * RPI * D, yy[x]);
+        }
+    }
+    // the rest, one access at a time
+    for (; c < nch; c += RPI, kp += RPI * D, dkp += RPI * D, dvp += RPI * D) {
+        uint32_t kw[KW];
+        float xx[8], yy[8];
+        load_key(kp, kw);
+        ld8f(dkp, xx);
+        ld8f(dvp, yy);
+        add_row(kw, xx, yy);
+        st8f(dkp, xx);
+        st8f(dvp, yy);
+    }
+    // the lanes that share columns (one per row of an access) add up
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1)
+#pragma unroll
+        for (int e = 0; e < 8; e++) mc[e] += __shfl_xor_sync(0xffffffffu, mc[e], off);
+}
+
 // Sums each of V values (V a power of two, at most 32) over the warp with
 // V - 1 + 5 - log2(V) shuffles: each halving step sends half of the values
 // still held and keeps the other half. Returns the sum of value `which`;
@@ -757,6 +850,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 2)
     const TokenMap tok = token_map(p);
     const bool top = j == p.J_cap;
     const long long total = (long long)p.B * p.H * chunks_per_unit;
+    // 256-bit token sweep when every row of the key cache, dk and dv starts
+    // where such an access may (else 64/128-bit accesses)
+    const bool wide = a.dk && (reinterpret_cast<uintptr_t>(p.K[0]) % (8 * sizeof(T))) == 0 &&
+                      ((reinterpret_cast<uintptr_t>(a.dk) | reinterpret_cast<uintptr_t>(a.dv)) % 32) == 0;
     for (long long ch = blockIdx.x; ch < total; ch += gridDim.x) {
         const long long u = ch / chunks_per_unit;
         const long long m0 = (ch % chunks_per_unit) * BWD_NODES_PER_PASS;
@@ -866,6 +963,29 @@ __global__ void __launch_bounds__(BWD_THREADS, 2)
                         mhi[i] += kh[i];
                     }
                 }
+            } else if (wide) {
+                // the node's tokens (contiguous rows: a node never straddles
+                // a page), 256-bit accesses: h and s at this lane's eight
+                // columns (the lanes of the other rows of an access hold the
+                // same ones) through the warp's mean row
+                float* stage = sm.mean[warp];
+                const int col = (lane % (D / 8)) * 8;
+                float hc[8], sc[8], mc[8];
+                store_pairs<D>(stage, lane, hlo, hhi);
+                __syncwarp();
+                load_vec<float, 8>(stage + col, hc);
+                __syncwarp();
+                store_pairs<D>(stage, lane, slo, shi);
+                __syncwarp();
+                load_vec<float, 8>(stage + col, sc);
+                sweep_tokens_v8<T, D>(reinterpret_cast<const T*>(p.K[0]), a.dk, a.dv, token_row(tok, u, m * p.b), nch,
+                                      lane, hc, sc, mc);
+                const float inv_n = 1.f / (float)nch;
+                __syncwarp();
+                if (lane < D / 8)
+#pragma unroll
+                    for (int e = 0; e < 8; e++) stage[col + e] = mc[e] * inv_n;
+                mean_staged = true;
             } else {
                 // the node's tokens (contiguous rows: a node never straddles
                 // a page): their keys for the mean, dk += h, dv += s. Here no
@@ -875,6 +995,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 2)
                 constexpr int E = D / 32;
                 float* stage = sm.mean[warp];
                 float hc[E], sc[E], mc[E];
+                const long long row0 = token_row(tok, u, m * p.b);
                 store_pairs<D>(stage, lane, hlo, hhi);
                 __syncwarp();
                 load_vec<float, E>(stage + lane * E, hc);
@@ -884,7 +1005,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 2)
                 load_vec<float, E>(stage + lane * E, sc);
 #pragma unroll
                 for (int e = 0; e < E; e++) mc[e] = 0.f;
-                const long long row0 = token_row(tok, u, m * p.b);
                 const T* kb = reinterpret_cast<const T*>(p.K[0]) + row0 * D + lane * E;
                 float* dkb = a.dk + row0 * D + lane * E;
                 float* dvb = a.dv + row0 * D + lane * E;

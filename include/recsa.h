@@ -241,7 +241,11 @@ recsa_status recsa_decode_backward(recsa_ctx* ctx, const void* q, const void* do
                                    float* dk, float* dv, void* scratch, size_t scratch_bytes, recsa_stream_t stream);
 
 /* Carries the node accumulators in `scratch` into dk, dv and dw (see
- * above), level by level from the top, and clears them. */
+ * above), level by level from the top, and clears them. dk, dv, dw: device,
+ * 16-byte aligned (RECSA_ERR_INVALID_ARG otherwise); when dk, dv are 32-byte
+ * aligned (and the key cache aligned to eight elements) every token row is
+ * updated with 256-bit accesses, else with 128-bit ones: the same dk, dv, and
+ * dw up to the order of its fp32 sums. */
 recsa_status recsa_tree_backward(recsa_ctx* ctx, float* dk, float* dv, float* dw, void* scratch,
                                  size_t scratch_bytes, recsa_stream_t stream);
 

@@ -136,6 +136,44 @@ def test_backward_mixed_parents_matches_oracle(bf16, D, b):
     _check_layer(layer, w, K, V, synth.as_f32(Wp), lengths, [(q_np, dout_np, gsel, parity.to_f64(dq))])
 
 
+@pytest.mark.parametrize("bf16,D", [(True, 128), (False, 64)])
+def test_backward_token_sweep_alignment(bf16, D):
+    """dk, dv that start 16 bytes past a 32-byte boundary (allowed by the
+    ABI) take the 64/128-bit token sweep; aligned ones the 256-bit sweep.
+    The two give the same dk, dv bit for bit (one add per element) and the
+    same dW up to the order of the key sums; the unaligned run is also
+    checked against the oracle."""
+    w = small(batch=2, n_kv_heads=2, group=4, head_dim=D, branching=8, k=3, bf16=bf16)
+    lengths = [517, 3001]
+    K, V, runs = synth.cache_arrays(w, max(lengths))
+    layer, Wp = make_layer(w, 4096)
+    layer.load(parity.to_dev(K, bf16), parity.to_dev(V, bf16), lengths)
+    q_np = per_seq_queries(w, runs, 0, lengths)
+    _, gsel, _ = run_decode(layer, w, q_np)
+    dout_np = _dout(w, 3)
+    q, dout, sel = parity.to_dev(q_np, bf16), parity.to_dev(dout_np, bf16), torch.from_numpy(gsel).cuda()
+    layer.zero_grad()
+    layer.decode_backward(q, dout, sel)
+    layer.tree_backward()
+    torch.cuda.synchronize()
+    layer.check()
+    dk_a, dv_a, dw_a = layer.dk.clone(), layer.dv.clone(), layer.dw.clone()
+    assert layer.dk.data_ptr() % 32 == 0 and layer.dv.data_ptr() % 32 == 0
+    n = layer.dk.numel()
+    bufs = [torch.zeros(n + 4, dtype=torch.float32, device="cuda") for _ in range(2)]
+    layer.dk = bufs[0][4:].view(dk_a.shape)
+    layer.dv = bufs[1][4:].view(dv_a.shape)
+    assert layer.dk.data_ptr() % 32 == 16 and layer.dv.data_ptr() % 32 == 16
+    layer.dw.zero_()
+    dq = layer.decode_backward(q, dout, sel)
+    layer.tree_backward()
+    torch.cuda.synchronize()
+    layer.check()
+    assert torch.equal(layer.dk, dk_a) and torch.equal(layer.dv, dv_a)
+    assert torch.allclose(layer.dw, dw_a, rtol=1e-5, atol=1e-6 * dw_a.abs().max().item())
+    _check_layer(layer, w, K, V, synth.as_f32(Wp), lengths, [(q_np, dout_np, gsel, parity.to_f64(dq))])
+
+
 def test_backward_sums_queries_and_clears_accumulators():
     """Two queries back-propagated before one tree pass give the sum of their
     gradients; a second tree pass adds nothing (the accumulators were cleared)."""
