@@ -314,7 +314,8 @@ __device__ __forceinline__ uint32_t f2_bf2(float2 x) {
 // HD + f + 8) by the table's (cos, sin), in packed fp32 (the same arithmetic
 // as the decode path's scoring), and stores both halves at `row` of two
 // K-major swizzled operands of `rows` rows: hi = bf16(x) and, if LO,
-// lo = bf16(x - hi). cs: cos [2], sin [2], -sin [2] as float4.
+// lo = bf16(x - hi). cs: cos [2], sin [2] as float4 (x b (-s) is the exact
+// negation of b s, so -sin is not loaded).
 template <int D, bool LO>
 __device__ __forceinline__ void put_chunk(uint4 xa_raw, uint4 xb_raw, const float4* cs, int f,
                                           unsigned char* hi_base, unsigned char* lo_base, int row, int rows) {
@@ -325,8 +326,8 @@ __device__ __forceinline__ void put_chunk(uint4 xa_raw, uint4 xb_raw, const floa
                           make_float2(cs[1].z, cs[1].w)};
     const float2 s2[4] = {make_float2(cs[2].x, cs[2].y), make_float2(cs[2].z, cs[2].w), make_float2(cs[3].x, cs[3].y),
                           make_float2(cs[3].z, cs[3].w)};
-    const float2 n2[4] = {make_float2(cs[4].x, cs[4].y), make_float2(cs[4].z, cs[4].w), make_float2(cs[5].x, cs[5].y),
-                          make_float2(cs[5].z, cs[5].w)};
+    const float2 n2[4] = {make_float2(-cs[2].x, -cs[2].y), make_float2(-cs[2].z, -cs[2].w),
+                          make_float2(-cs[3].x, -cs[3].y), make_float2(-cs[3].z, -cs[3].w)};
     uint32_t ha[4], la[4], hb[4], lb[4];
     const float2 m1 = make_float2(-1.f, -1.f);
 #pragma unroll
@@ -349,12 +350,12 @@ __device__ __forceinline__ void put_chunk(uint4 xa_raw, uint4 xb_raw, const floa
         *reinterpret_cast<uint4*>(lo_base + ob) = make_uint4(lb[0], lb[1], lb[2], lb[3]);
     }
 }
-// The table's cos, sin and -sin of frequencies [f, f + 8) of row `tab`.
+// The table's cos and sin of frequencies [f, f + 8) of row `tab`.
 template <int D>
 __device__ __forceinline__ void load_cs(const float* tab, int f, float4* cs) {
     constexpr int HD = D / 2;
 #pragma unroll
-    for (int x = 0; x < 3; x++) {
+    for (int x = 0; x < 2; x++) {
         cs[2 * x] = __ldg(reinterpret_cast<const float4*>(tab + x * HD + f));
         cs[2 * x + 1] = __ldg(reinterpret_cast<const float4*>(tab + x * HD + f + 4));
     }
@@ -503,7 +504,7 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
         constexpr bool LO = MODE != MODE_MAX;
         {
             const float* tab = p.rope + (size_t)(qok ? P : 0) * 3 * HD;
-            float4 cs[6], cn[6];
+            float4 cs[4], cn[4];
             load_cs<D>(tab, 0, cs);
             const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
@@ -511,19 +512,37 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
                 if (c + 1 < NCH) load_cs<D>(tab, (c + 1) * 8, cn);
                 put_chunk<D, LO>(qok ? qa[c] : z, qok ? qb[c] : z, cs, c * 8, sAh, sAl, tid, 128);
 #pragma unroll
-                for (int i = 0; i < 6; i++) cs[i] = cn[i];
+                for (int i = 0; i < 4; i++) cs[i] = cn[i];
             }
         }
 #pragma unroll
         for (int x = 0; x < BU; x++) {
             const int unit = tid + x * TP_THREADS, o = unit / NCH, c = unit % NCH;
-            float4 cs[6];
+            float4 cs[4];
             load_cs<D>(p.rope + (size_t)o * 3 * HD, c * 8, cs);
             const uint4 z = make_uint4(0, 0, 0, 0);
             put_chunk<D, LO>(o < nchild ? ka[x] : z, o < nchild ? kbv[x] : z, cs, c * 8, sBh, sBl, o, NB);
         }
         if (has_next && pr < tile_n.w) nc_n = L.nc[tile_n.x * a.C + (pk_n >> 6)];
-        if (MODE == MODE_VALUE) cp_async_wait_all();
+        // value pass: the children this token kept (not entries) and its
+        // reference maximum, loaded before the products so that their
+        // latency overlaps them
+        unsigned long long keep[(NB + 63) / 64];
+#pragma unroll
+        for (int x = 0; x < (NB + 63) / 64; x++) keep[x] = 0ull;
+        unsigned mk = 0u;
+        if (MODE == MODE_VALUE) {
+            if (valid && j > 0) {
+                const int* kl = L.kept + (u * a.C + t) * k;
+                const int nk = L.nkept[u * a.C + t];
+                for (int x = 0; x < nk; x++) {
+                    const int o = kl[x] - par * b;
+                    if (o >= 0 && o < NB) keep[o >> 6] |= 1ull << (o & 63);
+                }
+            }
+            mk = valid ? a.mkey[orow] : 0u;
+            cp_async_wait_all();
+        }
         fence_proxy_async_shared();
         tc_fence_before();
         __syncthreads();
@@ -588,18 +607,6 @@ __global__ void __launch_bounds__(TP_THREADS, 2) pf_tile_kernel(TreeParams p, Pf
         if (MODE == MODE_VALUE) {
             // weights of the entries: every token; above, the children this
             // token did not keep
-            unsigned long long keep[(NB + 63) / 64];
-#pragma unroll
-            for (int x = 0; x < (NB + 63) / 64; x++) keep[x] = 0ull;
-            if (valid && j > 0) {
-                const int* kl = L.kept + (u * a.C + t) * k;
-                const int nk = L.nkept[u * a.C + t];
-                for (int x = 0; x < nk; x++) {
-                    const int o = kl[x] - par * b;
-                    if (o >= 0 && o < NB) keep[o >> 6] |= 1ull << (o & 63);
-                }
-            }
-            const unsigned mk = valid ? a.mkey[orow] : 0u;
             const float mref = mk ? key_float(mk) : 0.f;
             constexpr float LOG2E = 1.4426950408889634f;
             const float mref2 = mref * LOG2E;
