@@ -1,4 +1,4 @@
-// Candidate scoring shared by the decode and prefill kernels.
+// Candidate scoring of the decode kernel (the prefill scores on tensor cores).
 //
 // Logit of a candidate at index i among its level's candidates, for query
 // head g with the query at index P (RecSA abstract: every entry is RoPE-rotated
