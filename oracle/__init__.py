@@ -60,6 +60,8 @@ def _load():
             lib.orc_query_grad.restype = i32
             lib.orc_query_grad.argtypes = [i32, i32, i32, i32, dbl, i64, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp,
                                            vp]
+            lib.orc_cluster_order.restype = i32
+            lib.orc_cluster_order.argtypes = [vp, i32, i64, i32, i32, vp, vp]
             lib.orc_query.restype = i32
             lib.orc_query.argtypes = [i32, i32, i32, i32, dbl, i64, vp, vp, vp, vp, i32, vp, vp, i64, vp, vp, vp, vp,
                                       vp]
@@ -195,6 +197,22 @@ def query_grad(tree_K, tree_V, Ktok, Vtok, T, q, dout, W, d, b, k, G, rope_base)
     if J < 0:
         raise ValueError("oracle gradient rejected its arguments")
     return dict(dq=dq, dK=dK, dV=dV, dW=dW, J=J)
+
+
+def cluster_order(Ktok, T: int, b: int, Z) -> np.ndarray:
+    """LSA-style clustered order of tokens [0, T) (reading R13 in
+    recsa_oracle.c): int32 [T], the token index at each position. Ktok: the
+    unit's keys [>= T][d] (float32, or bf16 bit patterns as int16); Z: the
+    learned directions, float32 [>= levels(T, b)][d]."""
+    lib = _load()
+    Kt, dt = _tok(Ktok)
+    Zf = np.ascontiguousarray(Z, dtype=np.float32)
+    d = Kt.shape[-1]
+    perm = np.zeros(T, dtype=np.int32)
+    J = lib.orc_cluster_order(Kt.ctypes.data, dt, T, d, b, Zf.ctypes.data, perm.ctypes.data)
+    if J < 0:
+        raise ValueError("oracle clustered order rejected its arguments")
+    return perm
 
 
 def query_tree(tree: Tree, Ktok, Vtok, q, k, G, rope_base, Kloc=None, Vloc=None, T=None):

@@ -45,6 +45,19 @@
  *   R11 RoPE: rotate-half pairs (i, i + d/2), theta_i = base^(-2i/d).
  *   R12 node keys and values are rounded to the storage type once, when
  *      formed; child keys are read as stored.
+ *   R13 LSA-style variant ("Latent Sparse Attention" abstract: keys are
+ *      clustered hierarchically in a learned latent space and queries score
+ *      the hierarchy of clusters; nothing more is given): a balanced
+ *      hierarchical partition with the tree's own fan-out. Level j has one
+ *      learned direction Z_j and the latent coordinate z_j(t) = <Z_j, k_t>
+ *      (fp64, summed in index order). From the top level J down to level 1,
+ *      the tokens of every block of b^(j+1) consecutive positions of the
+ *      current order are sorted by (z_j, token index); the level-j nodes of
+ *      the tree over the reordered tokens are then blocks of b^j positions
+ *      whose z_j ranges follow one another inside their parent. The tree,
+ *      the descent and the attention are the method's own over the
+ *      reordered cache (a RoPE index is a position among candidates, so the
+ *      tokens' original order does not enter).
  *
  * Parity unpinned: R6 at levels >= 1 (the query position there; level 0 is
  * pinned by the dense equivalence), R7's absence of a subtree-size bias, and
@@ -556,4 +569,53 @@ int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, co
     free(dKn); free(dVn); free(sel); free(out); free(cand); free(next); free(e_lev); free(e_id); free(e_rank);
     free(e_pos); free(lg); free(kv); free(vv); free(qd); free(r1); free(r2);
     return ok ? J : -1;
+}
+
+/* ---------------------------------------------- clustered order (R13) */
+
+typedef struct {
+    double z;
+    long long id;
+} latent;
+
+static int by_latent(const void* a, const void* b) {
+    const latent* x = (const latent*)a;
+    const latent* y = (const latent*)b;
+    if (x->z < y->z) return -1;
+    if (x->z > y->z) return 1;
+    return (x->id > y->id) - (x->id < y->id);
+}
+
+int orc_cluster_order(const void* Ktok, int tok_dtype, long long T, int d, int b, const float* Z, int* perm) {
+    if (T < 1 || d < 1 || b < 2 || !Ktok || !Z || !perm) return -1;
+    long long n[ORC_MAXLEV + 1];
+    const int J = orc_levels(T, b, n);
+    long long* ord = (long long*)malloc(sizeof(long long) * (size_t)T);
+    latent* seg = (latent*)malloc(sizeof(latent) * (size_t)T);
+    if (!ord || !seg) {
+        free(ord);
+        free(seg);
+        return -1;
+    }
+    for (long long p = 0; p < T; p++) ord[p] = p;
+    for (int j = J; j >= 1; j--) {
+        const long long S = ipow_sat(b, j + 1); /* the parent blocks (one block at the top) */
+        const float* Zj = Z + (size_t)(j - 1) * d;
+        for (long long s0 = 0; s0 < T; s0 += S) {
+            const long long s1 = s0 + S < T ? s0 + S : T;
+            for (long long p = s0; p < s1; p++) {
+                const long long t = ord[p];
+                double z = 0.0;
+                for (int e = 0; e < d; e++) z = z + (double)Zj[e] * tok_at(Ktok, tok_dtype, t * d + e);
+                seg[p - s0].z = z + 0.0; /* -0 and +0 are one value */
+                seg[p - s0].id = t;
+            }
+            qsort(seg, (size_t)(s1 - s0), sizeof(latent), by_latent);
+            for (long long p = s0; p < s1; p++) ord[p] = seg[p - s0].id;
+        }
+    }
+    for (long long p = 0; p < T; p++) perm[p] = (int)ord[p];
+    free(ord);
+    free(seg);
+    return J;
 }

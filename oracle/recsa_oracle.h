@@ -74,6 +74,15 @@ int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, co
                    const double* const* Vnode, const void* Ktok, const void* Vtok, int tok_dtype, const float* W,
                    const float* q, const double* dout, double* dq, double* dKtok, double* dVtok, double* dW);
 
+/* LSA-style clustered order of T tokens ("Latent Sparse Attention"
+ * abstract: keys clustered hierarchically in a learned latent space, queries
+ * scoring the hierarchy of clusters). Reading R13 (see the .c file): level j
+ * of the tree over the reordered tokens groups them by the latent coordinate
+ * z_j(t) = <Z row j-1, k_t>. Z is float32 [J][d] (J = levels(T, b); rows
+ * beyond J unused); perm [T] receives the token index placed at each
+ * position. Returns J, or -1 on bad arguments / allocation failure. */
+int orc_cluster_order(const void* Ktok, int tok_dtype, long long T, int d, int b, const float* Z, int* perm);
+
 #ifdef __cplusplus
 }
 #endif
