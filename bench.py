@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-distill", action="store_true")
+    ap.add_argument("--no-cluster", action="store_true")
     ap.add_argument("--prefill-workload", default="prefill_524k")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the chunked prefill (profiling): no decode, no baselines")
@@ -539,6 +540,102 @@ def measure_distill(layer, w, q, dev, flush, build_ms, kv_host, cpu_threads, wit
     return res
 
 
+def measure_cluster(layer, w, q, dev, flush, peaks, kv_host, steps, cpu_threads, with_cpu):
+    """LSA-style variant on the decode workload's tokens: recsa_cluster_load
+    (the clustered order of every unit's first L tokens under seeded learned
+    directions, the rows placed in that order, the tree built), median of 3
+    after a warm-up, L2 flushed; then decode steps (recsa_decode) over the
+    clustered tree. Roofline of the clustering: the bytes its kernels move by
+    design (per level the key rows read and the records written, every pass of
+    the sorting network reading and writing all records, the rows placed)
+    against the measured copy bandwidth. Beside it, the oracle computing the
+    same order for a sample of units on the host cores."""
+    B, H, D = w.batch, w.n_kv_heads, w.head_dim
+    L0, b = w.length, w.branching
+    stream = torch.cuda.current_stream(dev)
+    J_cap, _ = layer.tree_shape()
+    Z = torch.from_numpy(synth.plain(903, 0, (J_cap, D), 0.0, 1.0, False)).to(dev)
+    ksrc = layer.k_cache[:, :, :L0].contiguous()
+    vsrc = layer.v_cache[:, :, :L0].contiguous()
+    perm = torch.empty((B, H, layer.cfg.capacity), dtype=torch.int32, device=dev)
+    scratch = torch.empty(layer.ctx.cluster_scratch_bytes(), dtype=torch.uint8, device=dev)
+    layer.ctx.cluster_load(ksrc, vsrc, [L0] * B, Z, perm, scratch)
+    ts = []
+    for _ in range(3):
+        flush.fill_(6.0)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        layer.ctx.cluster_load(ksrc, vsrc, [L0] * B, Z, perm, scratch)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        ts.append(a.elapsed_time(b_))
+    layer.check()
+    ms = statistics.median(ts)
+    # the sorting network's own traffic (records of 24 bytes, all levels)
+    J, _ = oracle_levels(L0, b)
+    n = B * H * L0
+    n_pad, TILE, es = 1024, 1024, 2
+    while n_pad < n:
+        n_pad <<= 1
+    lg = n_pad.bit_length() - 1
+    passes = 1 + sum((s_ - 10) + 1 for s_ in range(11, lg + 1))  # first tile launch; per stage: global passes + tile
+    level_bytes = n * D * es + n_pad * 24 * 2 + passes * n_pad * 48
+    cl_bytes = J * level_bytes + n * (4 * D * es + 4)
+    gbs = cl_bytes / (ms / 1e3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+    # decode over the clustered tree (the fused append would add its token
+    # outside the clustered order; decode alone, on the clustered cache)
+    out = torch.empty((B, w.n_q_heads, D), dtype=torch.bfloat16, device=dev)
+    rows = torch.zeros((B, H, 2), dtype=torch.int64, device=dev)
+    for _ in range(3):
+        layer.decode(q, out)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(7.0)
+        evs[i][0].record(stream)
+        layer.decode(q, out, rows_out=rows if i == 0 else None)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    layer.check()
+    dms = [e[0].elapsed_time(e[1]) for e in evs]
+    rows_np = rows.cpu().numpy()
+    res = {"workload": f"{B} sequences x {H} KV heads x {L0} tokens (the decode workload's keys), b = {b}",
+           "cluster_ms": ms, "levels": J, "records": n,
+           "roofline": {"kernel": "recsa_cluster_load (all its launches)", "bound": "hbm", "achieved": gbs,
+                        "peak": hbm, "unit": "GB/s", "frac": gbs / hbm, "algorithmic_bytes": cl_bytes,
+                        "sort_passes_per_level": passes, "traffic": None},
+           "decode_ms": sum(dms) / steps, "decode_query_tok_s": B / (sum(dms) / steps / 1e3),
+           "rows_per_query": {"k_rows": float(rows_np[..., 0].mean()), "v_rows": float(rows_np[..., 1].mean())},
+           "how": "recsa_cluster_load median of 3 (L2 flushed), then recsa_decode steps over the clustered tree"}
+    del ksrc, vsrc, scratch
+    torch.cuda.empty_cache()
+    if with_cpu:
+        import oracle
+
+        units = [(bb, h) for bb in range(B) for h in range(H)][:max(1, min(cpu_threads, B * H))]
+        Zh = Z.cpu().numpy()
+        pool = oracle.pool(len(units))
+        t0 = time.perf_counter()
+        list(pool.map(lambda bh: oracle.cluster_order(kv_host[0][bh[0], bh[1]], L0, b, Zh), units))
+        dt = time.perf_counter() - t0
+        pool.shutdown()
+        res["cpu_baseline"] = {"value": len(units) * L0 / dt, "unit": "tokens/s", "cores": len(units), "kind": "oracle",
+                               "sample": f"oracle.cluster_order of {len(units)} units (L = {L0}) in parallel"}
+        res["gpu_tokens_s"] = n / (ms / 1e3)
+    return res
+
+
+def oracle_levels(T, b):
+    """Levels of the tree over T tokens (the first j >= 1 with
+    ceil(T / b^j) <= b) and the level sizes."""
+    n, j = [T], 0
+    while True:
+        j += 1
+        n.append(-(-n[-1] // b))
+        if n[-1] <= b:
+            return j, n
+
+
 # -------------------------------------------------------------------- main
 
 
@@ -835,6 +932,11 @@ def main():
         distill = measure_distill(layer, w, q_d[0], dev, flush, build_ms, (Kh.numpy(), Vh.numpy()),
                                   os.cpu_count() or 1, rank == 0 and world == 1 and not args.no_cpu_baseline)
 
+    cluster = None
+    if not args.no_cluster:
+        cluster = measure_cluster(layer, w, q_d[0], dev, flush, peaks, (Kh.numpy(), Vh.numpy()), 32,
+                                  os.cpu_count() or 1, rank == 0 and world == 1 and not args.no_cpu_baseline)
+
     prefill = None
     if not args.no_prefill:
         prefill = measure_prefill(args.prefill_workload, dev, flush, peaks)
@@ -860,7 +962,7 @@ def main():
                            "frac_hbm": build_bytes / (build_ms / 1e3) / 1e9 / hbm},
             "e2e": e2e, "gpu_launches": K_, "clocks": clk, "dense_decode": dense, "cpu_baseline": cpu,
             "wall_s_timed_loop": wall_s, "input_gen_s": gen_s, "prefill": prefill, "backward": backward,
-            "distill": distill,
+            "distill": distill, "cluster": cluster,
         }
         print(json.dumps(line), flush=True)
     layer.close()

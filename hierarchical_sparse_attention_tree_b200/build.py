@@ -14,7 +14,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "librecsa.so")
-SOURCES = ["api.cu", "tree.cu", "decode.cu", "dense.cu", "prefill_attn.cu", "prefill_tc.cu", "backward.cu", "distill.cu"]
+SOURCES = ["api.cu", "tree.cu", "decode.cu", "dense.cu", "prefill_attn.cu", "prefill_tc.cu", "backward.cu", "distill.cu",
+           "cluster.cu"]
 HEADERS = [os.path.join(CSRC, h) for h in ("common.cuh", "score.cuh", "append.cuh", "tc.cuh", "backward.cuh")] + \
     [os.path.join(ROOT, "include", "recsa.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -1,6 +1,8 @@
 // Host side of the C ABI declared in include/recsa.h: argument checks,
 // workspace layout, RoPE table, kernel dispatch. Every launch goes on the
 // caller's stream; nothing here allocates device memory.
+#include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -38,6 +40,11 @@ size_t prefill_tree_scratch_bytes(const TreeParams& p, int C, int Hq);
 bool prefill_tree_supported(int D, int b);
 size_t decode_smem_bytes(int D, int G, int elem, int k, int b, int J_cap, bool fused);
 cudaError_t launch_distill_loss(const float*, const float*, float*, float*, long long, cudaStream_t);
+long long cluster_records(long long units, long long cap);
+size_t cluster_rec_bytes(long long units, long long cap);
+template <typename T, int D>
+cudaError_t launch_cluster(const TreeParams&, const void*, const void*, long long, const float*, const long long*,
+                           long long, int, int*, void*, cudaStream_t);
 template <typename T>
 cudaError_t launch_pooler_update(float*, const float*, float, void*, float*, int, cudaStream_t);
 size_t dense_static_scratch_bytes();
@@ -803,6 +810,70 @@ recsa_status recsa_distill_step(recsa_ctx* ctx, const void* q, const float* targ
     if (e == cudaSuccess && loss) e = cudaMemcpyAsync(loss, lossd, 4, cudaMemcpyDeviceToDevice, s);
     if (e != cudaSuccess) return cuda_fail(e, "recsa_distill_step");
     return RECSA_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------ clustered order
+
+namespace {
+// Levels of the tree over L >= 1 tokens (the first j >= 1 with ceil(L / b^j) <= b).
+int levels_of(long long L, int b) {
+    int j = 1;
+    long long s = b;
+    while (j < MAXJ && (L + s - 1) / s > b) {
+        s = s > LLONG_MAX / b ? LLONG_MAX : s * b;
+        j++;
+    }
+    return j;
+}
+}  // namespace
+
+extern "C" {
+
+size_t recsa_cluster_scratch_bytes(const recsa_config* cfg) {
+    if (check_config(cfg) != RECSA_OK) return 0;
+    const long long units = (long long)cfg->batch * cfg->n_kv_heads;
+    return align256(cluster_rec_bytes(units, cfg->capacity)) + align256((size_t)(cfg->batch + 1) * 8);
+}
+
+recsa_status recsa_cluster_load(recsa_ctx* ctx, const void* k_src, const void* v_src, long long src_len,
+                                const long long* lengths, const float* Z, int* perm, void* scratch,
+                                size_t scratch_bytes, recsa_stream_t stream) {
+    if (!ctx || !k_src || !v_src || !lengths || !Z || !perm || !scratch)
+        return fail(RECSA_ERR_INVALID_ARG, "NULL argument");
+    if (!aligned(k_src, 16) || !aligned(v_src, 16) || !aligned(Z, 16) || !aligned(perm, 4))
+        return fail(RECSA_ERR_INVALID_ARG, "k_src/v_src/Z not 16-byte or perm not 4-byte aligned");
+    if (!aligned(scratch, 256)) return fail(RECSA_ERR_INVALID_ARG, "scratch not 256-byte aligned");
+    if (ctx->p.pages) return fail(RECSA_ERR_UNSUPPORTED, "the clustered order needs a contiguous cache");
+    const recsa_config& c = ctx->cfg;
+    if (scratch_bytes < recsa_cluster_scratch_bytes(&c))
+        return fail(RECSA_ERR_INVALID_ARG, "scratch of %zu bytes, %zu needed", scratch_bytes,
+                    recsa_cluster_scratch_bytes(&c));
+    if (src_len < 1 || src_len > INT_MAX) return fail(RECSA_ERR_INVALID_ARG, "src_len %lld outside [1, 2^31)", src_len);
+    std::vector<long long> sstart((size_t)c.batch + 1, 0);
+    int J_max = 0;
+    for (int b = 0; b < c.batch; b++) {
+        if (lengths[b] < 0 || lengths[b] > c.capacity || lengths[b] > src_len)
+            return fail(RECSA_ERR_CAPACITY, "length %lld of sequence %d outside [0, min(capacity, src_len)]",
+                        lengths[b], b);
+        sstart[b + 1] = sstart[b] + lengths[b];
+        if (lengths[b] > 0) J_max = std::max(J_max, levels_of(lengths[b], c.branching));
+    }
+    const long long n = (long long)c.n_kv_heads * sstart[c.batch];
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (n > 0) {
+        char* base = static_cast<char*>(scratch);
+        long long* sstart_dev =
+            reinterpret_cast<long long*>(base + align256(cluster_rec_bytes((long long)c.batch * c.n_kv_heads, c.capacity)));
+        e = cudaMemcpyAsync(sstart_dev, sstart.data(), sstart.size() * 8, cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess)
+            DISPATCH_TD(c.dtype, c.head_dim,
+                        e = launch_cluster<T, DD>(ctx->p, k_src, v_src, src_len, Z, sstart_dev, n, J_max, perm, base, s));
+        if (e != cudaSuccess) return cuda_fail(e, "recsa_cluster_load");
+    }
+    return recsa_build_tree(ctx, lengths, stream);
 }
 
 }  // extern "C"

@@ -57,6 +57,22 @@ class RecsaLayer:
             self.v_cache[:, :, :L].copy_(V, non_blocking=True)
         self.ctx.build_tree(lengths, stream)
 
+    def load_clustered(self, K: torch.Tensor, V: torch.Tensor, lengths, Z: torch.Tensor, stream=None):
+        """LSA-style variant: place tokens [B][H][L][d] into the cache in the
+        clustered order of the learned directions Z [J_cap][d] (fp32) and build
+        the tree over them. Returns perm [B][H][capacity] (int32, device):
+        the source token at each cache position (positions < lengths[b])."""
+        if getattr(self, "_cluster_scratch", None) is None:
+            self._cluster_scratch = torch.empty(self.ctx.cluster_scratch_bytes(), dtype=torch.uint8,
+                                                device=self.device)
+        K = K.to(device=self.device, dtype=self.dtype).contiguous()
+        V = V.to(device=self.device, dtype=self.dtype).contiguous()
+        Z = Z.to(device=self.device, dtype=torch.float32).contiguous()
+        perm = torch.full((self.cfg.batch, self.cfg.n_kv_heads, self.cfg.capacity), -1, dtype=torch.int32,
+                          device=self.device)
+        self.ctx.cluster_load(K, V, lengths, Z, perm, self._cluster_scratch, stream)
+        return perm
+
     def tokens(self, b: int, L: int):
         """Keys and values [H][L][d] of sequence b's first L tokens (read
         back through the page table when paged)."""

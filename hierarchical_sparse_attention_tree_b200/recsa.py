@@ -23,7 +23,8 @@ EXPORTS = [
     "recsa_prefill_scratch_bytes", "recsa_prefill", "recsa_get_lengths", "recsa_tree_shape", "recsa_level_arrays",
     "recsa_query_stats", "recsa_check_device", "recsa_last_error", "recsa_destroy", "recsa_dense_decode_scratch_bytes",
     "recsa_dense_decode", "recsa_dense_decode_static", "recsa_backward_scratch_bytes", "recsa_decode_backward",
-    "recsa_tree_backward", "recsa_distill_scratch_bytes", "recsa_distill_step",
+    "recsa_tree_backward", "recsa_distill_scratch_bytes", "recsa_distill_step", "recsa_cluster_scratch_bytes",
+    "recsa_cluster_load",
 ]
 
 
@@ -64,6 +65,8 @@ def lib():
             "recsa_tree_backward": (i32, [vp, vp, vp, vp, vp, sz, vp]),
             "recsa_distill_scratch_bytes": (sz, [P(Config)]),
             "recsa_distill_step": (i32, [vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, sz, vp]),
+            "recsa_cluster_scratch_bytes": (sz, [P(Config)]),
+            "recsa_cluster_load": (i32, [vp, vp, vp, i64, P(i64), vp, vp, vp, sz, vp]),
             "recsa_append_decode": (i32, [vp, vp, vp, vp, vp, vp, vp, vp]),
             "recsa_prefill_scratch_bytes": (sz, [P(Config), i32]),
             "recsa_prefill": (i32, [vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
@@ -212,6 +215,15 @@ class Context:
     def tree_backward(self, dk, dv, dw, scratch, stream=None):
         _check(lib().recsa_tree_backward(self.handle, _ptr(dk), _ptr(dv), _ptr(dw), _ptr(scratch),
                                          scratch.numel() * scratch.element_size(), _stream(stream)))
+
+    def cluster_scratch_bytes(self) -> int:
+        return lib().recsa_cluster_scratch_bytes(ctypes.byref(self.cfg))
+
+    def cluster_load(self, k_src, v_src, lengths, Z, perm, scratch, stream=None):
+        arr = (ctypes.c_longlong * self.cfg.batch)(*[int(x) for x in lengths])
+        _check(lib().recsa_cluster_load(self.handle, _ptr(k_src), _ptr(v_src), int(k_src.shape[2]), arr, _ptr(Z),
+                                        _ptr(perm), _ptr(scratch), scratch.numel() * scratch.element_size(),
+                                        _stream(stream)))
 
     def distill_scratch_bytes(self) -> int:
         return lib().recsa_distill_scratch_bytes(ctypes.byref(self.cfg))

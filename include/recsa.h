@@ -282,6 +282,44 @@ recsa_status recsa_check_device(recsa_ctx* ctx, recsa_stream_t stream);
 const char* recsa_last_error(void);
 void recsa_destroy(recsa_ctx* ctx);
 
+/* ---------------------------------------------------------------------
+ * LSA-style variant: the tree over a clustered token order. The "Latent
+ * Sparse Attention" abstract clusters the keys hierarchically in a learned
+ * latent space and lets the queries score the hierarchy of clusters. Read
+ * with this tree's fan-out b: level j has one learned direction Z_j and the
+ * latent coordinate z_j(t) = <Z_j, k_t> (fp64, summed in index order); from
+ * the top level down, the tokens of every block of b^(j+1) consecutive
+ * positions of the current order are sorted by (z_j, token index). The
+ * level-j nodes of the tree over the reordered tokens are then blocks of b^j
+ * positions whose z_j ranges follow one another inside their parent; the
+ * descent and the attention over that tree are the method's own (a RoPE
+ * index is a position among candidates, so the original order does not
+ * enter). Contiguous caches only.
+ *
+ * recsa_cluster_load: for every sequence b and KV head h, orders the source
+ * tokens [0, lengths[b]) as above (the level count J of that length), writes
+ * the order to perm and the reordered key and value rows into the cache
+ * (positions [0, lengths[b])), then builds the tree as recsa_build_tree
+ * does. Afterwards recsa_decode runs over the clustered tree; an append adds
+ * its token at the right edge, outside the clustered order.
+ *   k_src, v_src  device [B][H_kv][src_len][d] in cfg->dtype, 16-byte aligned,
+ *                 read only;
+ *   lengths       host [B], 0 <= lengths[b] <= min(capacity, src_len);
+ *   Z             device fp32 [J_cap][d] (recsa_tree_shape gives J_cap), row
+ *                 j - 1 the direction of level j, 16-byte aligned;
+ *   perm          device int32 [B][H_kv][capacity]: perm[b][h][p] = the source
+ *                 token index placed at cache position p (p < lengths[b]; the
+ *                 rest untouched);
+ *   scratch       device, recsa_cluster_scratch_bytes(cfg) bytes, 256-byte
+ *                 aligned, no contents needed.
+ * RECSA_ERR_INVALID_ARG / RECSA_ERR_CAPACITY (nothing launched) for NULL or
+ * misaligned pointers, a short scratch, src_len outside [1, 2^31) or a length
+ * out of range; RECSA_ERR_UNSUPPORTED for a paged context. */
+size_t recsa_cluster_scratch_bytes(const recsa_config* cfg);
+recsa_status recsa_cluster_load(recsa_ctx* ctx, const void* k_src, const void* v_src, long long src_len,
+                                const long long* lengths, const float* Z, int* perm, void* scratch,
+                                size_t scratch_bytes, recsa_stream_t stream);
+
 /* Comparator, not part of the method: dense GQA flash-decode of one query
  * per sequence over every cached token, keys used as stored (no RoPE).
  * k_cache, v_cache [B][H_kv][L_stride][d], q, out [B][H_q][d], bf16 or fp32.
