@@ -200,7 +200,7 @@ def query_grad(tree_K, tree_V, Ktok, Vtok, T, q, dout, W, d, b, k, G, rope_base)
 
 
 def cluster_order(Ktok, T: int, b: int, Z) -> np.ndarray:
-    """LSA-style clustered order of tokens [0, T) (reading R13 in
+    """LSA-style clustered order of tokens [0, T) (reading R20 in
     recsa_oracle.c): int32 [T], the token index at each position. Ktok: the
     unit's keys [>= T][d] (float32, or bf16 bit patterns as int16); Z: the
     learned directions, float32 [>= levels(T, b)][d]."""

@@ -45,7 +45,7 @@
  *   R11 RoPE: rotate-half pairs (i, i + d/2), theta_i = base^(-2i/d).
  *   R12 node keys and values are rounded to the storage type once, when
  *      formed; child keys are read as stored.
- *   R13 LSA-style variant ("Latent Sparse Attention" abstract: keys are
+ *   R20 LSA-style variant ("Latent Sparse Attention" abstract: keys are
  *      clustered hierarchically in a learned latent space and queries score
  *      the hierarchy of clusters; nothing more is given): a balanced
  *      hierarchical partition with the tree's own fan-out. Level j has one
@@ -571,7 +571,7 @@ int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, co
     return ok ? J : -1;
 }
 
-/* ---------------------------------------------- clustered order (R13) */
+/* ---------------------------------------------- clustered order (R20) */
 
 typedef struct {
     double z;

@@ -76,7 +76,7 @@ int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, co
 
 /* LSA-style clustered order of T tokens ("Latent Sparse Attention"
  * abstract: keys clustered hierarchically in a learned latent space, queries
- * scoring the hierarchy of clusters). Reading R13 (see the .c file): level j
+ * scoring the hierarchy of clusters). Reading R20 (see the .c file): level j
  * of the tree over the reordered tokens groups them by the latent coordinate
  * z_j(t) = <Z row j-1, k_t>. Z is float32 [J][d] (J = levels(T, b); rows
  * beyond J unused); perm [T] receives the token index placed at each

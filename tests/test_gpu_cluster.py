@@ -9,7 +9,7 @@ rows (the source rows in that order, bit for bit), every tree level
 (check_nodes over the reordered tokens) and decode outputs and selections
 (check_units over the reordered cache, staged and free). Source: the "Latent
 Sparse Attention" abstract (keys clustered hierarchically in a learned latent
-space, queries scoring the hierarchy of clusters), reading R13.
+space, queries scoring the hierarchy of clusters), reading R20.
 """
 import numpy as np
 import pytest

@@ -8,7 +8,7 @@ in (z_1, index) order; with every direction equal to one coordinate axis the
 order is numpy's stable argsort along it; identical keys keep the token order.
 Source: the "Latent Sparse Attention" abstract (keys clustered hierarchically
 in a learned latent space, queries scoring the hierarchy of clusters) and the
-reading R13 of recsa_oracle.c.
+reading R20 of recsa_oracle.c.
 """
 import numpy as np
 import pytest
