@@ -578,7 +578,8 @@ def measure_cluster(layer, w, q, dev, flush, peaks, kv_host, steps, cpu_threads,
     while n_pad < n:
         n_pad <<= 1
     lg = n_pad.bit_length() - 1
-    passes = 1 + sum((s_ - 10) + 1 for s_ in range(11, lg + 1))  # first tile launch; per stage: global passes + tile
+    # first tile launch; per stage: the global distances two per pass, then a tile launch
+    passes = 1 + sum((s_ - 10 + 1) // 2 + 1 for s_ in range(11, lg + 1))
     level_bytes = n * D * es + n_pad * 24 * 2 + passes * n_pad * 48
     cl_bytes = J * level_bytes + n * (4 * D * es + 4)
     gbs = cl_bytes / (ms / 1e3) / 1e9

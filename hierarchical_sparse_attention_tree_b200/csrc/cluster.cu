@@ -13,7 +13,7 @@
 // The order is one bitonic sort per level over every unit's tokens at once:
 // records (unit | block, order key of z, token) in one array padded to a
 // power of two; stages with partner distance below CL_TILE run in shared
-// memory, the longer distances one global pass each. z is summed in fp64 in
+// memory, the longer distances two per global pass. z is summed in fp64 in
 // index order with separately rounded products (the decision of an integer
 // order taken in one stated precision).
 #include <climits>
@@ -167,6 +167,27 @@ __global__ void __launch_bounds__(256) cl_pass_kernel(ClRec* rec, long long n_pa
     }
 }
 
+// Two distances j and j / 2 of stage k in one pass (j / 2 >= CL_TILE): each
+// thread holds the four records i0, i0 + j/2, i0 + j, i0 + 3j/2 (bits j and
+// j/2 of i0 clear), which the two steps only exchange among themselves, and
+// applies the distance-j then the distance-j/2 compare-exchanges.
+__global__ void __launch_bounds__(256) cl_pass2_kernel(ClRec* rec, long long n_pad, long long k, long long j) {
+    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n_pad / 4) return;
+    const long long h = j >> 1;
+    const long long i0 = (t & (h - 1)) | ((t & ~(h - 1)) << 2);
+    const bool asc = (i0 & k) == 0;
+    ClRec a = rec[i0], b = rec[i0 + h], c = rec[i0 + j], d = rec[i0 + j + h];
+    cl_cmpx(a, c, asc);
+    cl_cmpx(b, d, asc);
+    cl_cmpx(a, b, asc);
+    cl_cmpx(c, d, asc);
+    rec[i0] = a;
+    rec[i0 + h] = b;
+    rec[i0 + j] = c;
+    rec[i0 + j + h] = d;
+}
+
 // The order after the last level: perm[u][pos] = the token placed at pos, and
 // the token's key and value rows copied there (one warp per record).
 template <typename T, int D>
@@ -214,12 +235,15 @@ cudaError_t launch_cluster(const TreeParams& p, const void* ksrc, const void* vs
     a.n_pad = CL_TILE;
     while (a.n_pad < n) a.n_pad <<= 1;
     const unsigned gk = (unsigned)((a.n_pad + 255) / 256), gp = (unsigned)((a.n_pad / 2 + 255) / 256);
+    const unsigned gp2 = (unsigned)((a.n_pad / 4 + 255) / 256);
     const unsigned gt = (unsigned)(a.n_pad / CL_TILE);
     for (int j = J_max; j >= 1; j--) {
         cl_keys_kernel<T, D><<<gk, 256, 0, s>>>(p, a, j, j == J_max);
         cl_tile_kernel<<<gt, CL_THREADS, 0, s>>>(a.rec, 0, 1);
         for (long long k = 2 * CL_TILE; k <= a.n_pad; k <<= 1) {
-            for (long long jj = k >> 1; jj >= CL_TILE; jj >>= 1) cl_pass_kernel<<<gp, 256, 0, s>>>(a.rec, a.n_pad, k, jj);
+            long long jj = k >> 1;
+            for (; (jj >> 1) >= CL_TILE; jj >>= 2) cl_pass2_kernel<<<gp2, 256, 0, s>>>(a.rec, a.n_pad, k, jj);
+            if (jj >= CL_TILE) cl_pass_kernel<<<gp, 256, 0, s>>>(a.rec, a.n_pad, k, jj);
             cl_tile_kernel<<<gt, CL_THREADS, 0, s>>>(a.rec, k, 0);
         }
         const cudaError_t e = cudaGetLastError();
