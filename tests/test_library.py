@@ -112,3 +112,21 @@ def test_distill_scratch_and_null_arguments():
     assert n >= R.lib().recsa_backward_scratch_bytes(ctypes.byref(cfg)) + 3 * 4 * 32 * 128 * 4
     assert R.lib().recsa_distill_step(None, None, None, ctypes.c_float(0.1), None, None, None, None, 0,
                                       None) == R.ERR_INVALID_ARG
+
+
+def test_cluster_scratch_and_null_arguments():
+    """The clustered order's scratch: one 24-byte record per token of every
+    unit at capacity, padded to a power of two (at least one 1024-record
+    tile), plus the sequences' start offsets; NULL arguments are rejected on
+    the host."""
+    tail = 256  # [B + 1] offsets, one 256-byte-aligned block
+    cfg = R.make_config(4, 8, 32, 128, 64, 16, 524288)
+    assert R.lib().recsa_cluster_scratch_bytes(ctypes.byref(cfg)) == (1 << 24) * 24 + tail
+    cfg = R.make_config(4, 8, 32, 128, 64, 16, 524289)
+    assert R.lib().recsa_cluster_scratch_bytes(ctypes.byref(cfg)) == (1 << 25) * 24 + tail
+    cfg = R.make_config(1, 1, 4, 64, 8, 3, 10)
+    assert R.lib().recsa_cluster_scratch_bytes(ctypes.byref(cfg)) == 1024 * 24 + tail
+    bad = R.make_config(1, 8, 32, 96, 64, 16, 1024)
+    assert R.lib().recsa_cluster_scratch_bytes(ctypes.byref(bad)) == 0
+    lengths = (ctypes.c_longlong * 1)(10)
+    assert R.lib().recsa_cluster_load(None, None, None, 10, lengths, None, None, None, 0, None) == R.ERR_INVALID_ARG
