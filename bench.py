@@ -56,7 +56,7 @@ def parse():
                     help="run only the chunked prefill (profiling): no decode, no baselines")
     ap.add_argument("--prefill-last", type=int, default=0,
                     help="build the tree over all but the last N chunks at once, then prefill only those N")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU-baseline sample")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="time limit of the oracle CPU-baseline sample (seconds)")
     ap.add_argument("--settle-s", type=float, default=0.3, help="decode-only launches before timing (clock sampling)")
     return ap.parse_args()
 
@@ -189,12 +189,12 @@ def aggregate_rate(world: int, batch: int, steps: int, max_seconds: float) -> fl
 # --------------------------------------------------------- oracle baseline
 
 
-def oracle_decode_steps(w, K, V, Wp, runs, length0, n_steps, budget_s, seq_ids, threads):
+def oracle_decode_steps(w, K, V, Wp, runs, length0, n_steps, limit_s, seq_ids, threads):
     """The fp64 oracle doing the decode workload's steps for the given
     sequences, every (sequence, KV head) unit in parallel on `threads` host
     threads: per step and per unit, refresh the nodes the new token touched,
     then one query. The trees are built and every step's queries generated
-    before the timed loop. Stops at n_steps or when budget_s is spent.
+    before the timed loop. Stops at n_steps or after limit_s seconds.
     Returns (steps done, seconds, query tokens, threads used)."""
     import oracle
 
@@ -227,7 +227,7 @@ def oracle_decode_steps(w, K, V, Wp, runs, length0, n_steps, budget_s, seq_ids, 
 
         list(pool.map(unit, units))
         done += 1
-        if time.perf_counter() - t0 > budget_s:
+        if time.perf_counter() - t0 > limit_s:
             break
     dt = time.perf_counter() - t0
     pool.shutdown()
