@@ -60,6 +60,9 @@ def _load():
             lib.orc_query_grad.restype = i32
             lib.orc_query_grad.argtypes = [i32, i32, i32, i32, dbl, i64, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp,
                                            vp]
+            lib.orc_query_grad_local.restype = i32
+            lib.orc_query_grad_local.argtypes = [i32, i32, i32, i32, dbl, i64, vp, vp, vp, vp, i32, vp, vp, i64, vp,
+                                                 vp, vp, vp, vp, vp, vp, vp, vp]
             lib.orc_cluster_order.restype = i32
             lib.orc_cluster_order.argtypes = [vp, i32, i64, i32, i32, vp, vp]
             lib.orc_query.restype = i32
@@ -175,9 +178,13 @@ def query(tree_K, tree_V, Ktok, Vtok, T, q, d, b, k, G, rope_base, Kloc=None, Vl
     return dict(out=out, sel=sel[:J], margin=margin[:J], k_rows=int(rows[0]), v_rows=int(rows[1]), J=J)
 
 
-def query_grad(tree_K, tree_V, Ktok, Vtok, T, q, dout, W, d, b, k, G, rope_base):
-    """Gradients of one decode query with the selections held fixed.
-    Returns dict(dq [G][d], dK [T][d], dV [T][d], dW [d][d]) in fp64."""
+def query_grad(tree_K, tree_V, Ktok, Vtok, T, q, dout, W, d, b, k, G, rope_base, Kloc=None, Vloc=None):
+    """Gradients of one query with the selections held fixed: a decode query,
+    or (Kloc, Vloc given) a prefill query with its chunk's own causal tokens.
+    Returns dict(dq [G][d], dK [T][d], dV [T][d], dW [d][d]) in fp64, and
+    dKloc, dVloc [nloc][d] for the local tokens."""
+    if Kloc is not None and len(Kloc):
+        return _query_grad_local(tree_K, tree_V, Ktok, Vtok, T, q, dout, W, d, b, k, G, rope_base, Kloc, Vloc)
     lib = _load()
     kt, dt = _tok(Ktok)
     vt, _ = _tok(Vtok)
@@ -213,6 +220,34 @@ def cluster_order(Ktok, T: int, b: int, Z) -> np.ndarray:
     if J < 0:
         raise ValueError("oracle clustered order rejected its arguments")
     return perm
+
+
+def _query_grad_local(tree_K, tree_V, Ktok, Vtok, T, q, dout, W, d, b, k, G, rope_base, Kloc, Vloc):
+    lib = _load()
+    kt, dt = _tok(Ktok)
+    vt, _ = _tok(Vtok)
+    kl, dt2 = _tok(Kloc)
+    vl, _ = _tok(Vloc)
+    if dt2 != dt:
+        raise ValueError("local tokens must have the cache's dtype")
+    nloc = kl.shape[0]
+    Jt, _ = levels(T, b)
+    qf = np.ascontiguousarray(q, dtype=np.float32)
+    do = np.ascontiguousarray(dout, dtype=np.float64)
+    Wf = np.ascontiguousarray(W, dtype=np.float32)
+    dq = np.zeros((G, d))
+    dK, dV = np.zeros((max(T, 1), d)), np.zeros((max(T, 1), d))
+    dKl, dVl = np.zeros((nloc, d)), np.zeros((nloc, d))
+    dW = np.zeros((d, d))
+    Kp = [None] + [np.ascontiguousarray(x, dtype=np.float64) for x in tree_K[1:Jt + 1]]
+    Vp = [None] + [np.ascontiguousarray(x, dtype=np.float64) for x in tree_V[1:Jt + 1]]
+    J = lib.orc_query_grad_local(d, b, k, G, rope_base, T, _ptr_array(Kp), _ptr_array(Vp), kt.ctypes.data,
+                                 vt.ctypes.data, dt, kl.ctypes.data, vl.ctypes.data, nloc, Wf.ctypes.data,
+                                 qf.ctypes.data, do.ctypes.data, dq.ctypes.data, dK.ctypes.data, dV.ctypes.data,
+                                 dKl.ctypes.data, dVl.ctypes.data, dW.ctypes.data)
+    if J < 0:
+        raise ValueError("oracle gradient rejected its arguments")
+    return dict(dq=dq, dK=dK[:T], dV=dV[:T], dW=dW, dKloc=dKl, dVloc=dVl, J=J)
 
 
 def query_tree(tree: Tree, Ktok, Vtok, q, k, G, rope_base, Kloc=None, Vloc=None, T=None):

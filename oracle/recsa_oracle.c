@@ -370,10 +370,19 @@ int orc_query(int d, int b, int k, int G, double rope_base, long long T, const d
 
 /* ----------------------------------------------------------- gradients */
 
-/* Gradient of one decode query's output (orc_query with no local tokens)
- * with the selections held fixed (they are not differentiable): given
- * dout [G][d], returns dq [G][d] (overwritten) and adds into dKtok, dVtok
- * [T][d] and dW [d][d] the gradients with respect to the token keys and
+/* Coordinate i of entry (level, id): a node row (level >= 1), a token row
+ * (level 0) or a row of the chunk's own tokens (level -1). */
+static double entry_at(const double* const* node, const void* tok, const void* loc, int tok_dtype, int level,
+                       long long id, int d, int i) {
+    if (level > 0) return node[level][id * d + i];
+    return tok_at(level == 0 ? tok : loc, tok_dtype, id * d + i);
+}
+
+/* Gradient of one query's output (orc_query; a decode query, or a prefill
+ * query with its chunk's own causal tokens Kloc, Vloc [nloc][d], whose
+ * gradients go to dKloc, dVloc) with the selections held fixed (they are not
+ * differentiable): given dout [G][d], returns dq [G][d] (overwritten) and adds
+ * into dKtok, dVtok [T][d] and dW [d][d] the gradients with respect to the token keys and
  * values and the pooler, through the direct token entries and through the
  * summaries (a node value is the mean of its subtree's token values, a node
  * key is W times the mean of its children's stored keys; storage rounding is
@@ -387,10 +396,13 @@ int orc_query(int d, int b, int k, int G, double rope_base, long long T, const d
  * dW, and each token gets W^T g_parent / children(parent) for its level-1
  * parent plus, for every ancestor a, dv_a / tokens(a).
  * Returns J, or -1 on bad arguments / allocation failure. */
-int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, const double* const* Knode,
-                   const double* const* Vnode, const void* Ktok, const void* Vtok, int tok_dtype, const float* W,
-                   const float* q, const double* dout, double* dq, double* dKtok, double* dVtok, double* dW) {
-    if (d <= 0 || d % 2 || b < 2 || k < 1 || G < 1 || T < 1) return -1;
+static int query_grad_impl(int d, int b, int k, int G, double rope_base, long long T, const double* const* Knode,
+                           const double* const* Vnode, const void* Ktok, const void* Vtok, int tok_dtype,
+                           const void* Kloc, const void* Vloc, long long nloc, const float* W, const float* q,
+                           const double* dout, double* dq, double* dKtok, double* dVtok, double* dKloc, double* dVloc,
+                           double* dW) {
+    if (d <= 0 || d % 2 || b < 2 || k < 1 || G < 1 || T < 0 || nloc < 0 || T + nloc < 1) return -1;
+    if (nloc > 0 && (!Kloc || !Vloc || !dKloc || !dVloc)) return -1;
     long long n[ORC_MAXLEV + 1];
     int J = orc_levels(T, b, n);
     int* sel = (int*)malloc(sizeof(int) * (size_t)(J * k + 1));
@@ -401,7 +413,7 @@ int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, co
         return -1;
     }
     /* the forward's selections */
-    if (orc_query(d, b, k, G, rope_base, T, Knode, Vnode, Ktok, Vtok, tok_dtype, NULL, NULL, 0, q, out, sel, NULL,
+    if (orc_query(d, b, k, G, rope_base, T, Knode, Vnode, Ktok, Vtok, tok_dtype, Kloc, Vloc, nloc, q, out, sel, NULL,
                   NULL) != J) {
         free(sel);
         free(out);
@@ -409,7 +421,7 @@ int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, co
     }
     double scale = 1.0 / sqrt((double)d);
     long long max_cand = (long long)k * b > b ? (long long)k * b : b;
-    long long max_ent = (long long)(J + 1) * max_cand + 1;
+    long long max_ent = (long long)(J + 1) * max_cand + nloc + 1;
     long long* cand = (long long*)malloc(sizeof(long long) * (size_t)max_cand);
     long long* next = (long long*)malloc(sizeof(long long) * (size_t)max_cand);
     int* e_lev = (int*)malloc(sizeof(int) * (size_t)max_ent);
@@ -458,17 +470,26 @@ int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, co
             memcpy(cand, next, sizeof(long long) * (size_t)nn);
             nc = nn;
         }
+        /* level 0: the tokens, then the chunk's own causal tokens (level -1);
+         * the query sits at the last index of that list (R6, R9) */
         for (long long i = 0; i < nc; i++) {
             e_lev[n_ent] = 0;
             e_id[n_ent] = cand[i];
             e_rank[n_ent] = i;
-            e_pos[n_ent] = nc - 1;
+            e_pos[n_ent] = nc + nloc - 1;
+            n_ent++;
+        }
+        for (long long i = 0; i < nloc; i++) {
+            e_lev[n_ent] = -1;
+            e_id[n_ent] = i;
+            e_rank[n_ent] = nc + i;
+            e_pos[n_ent] = nc + nloc - 1;
             n_ent++;
         }
         /* logits and softmax per head */
         for (long long e = 0; e < n_ent; e++) {
             for (int i = 0; i < d; i++)
-                kv[i] = e_lev[e] ? Knode[e_lev[e]][e_id[e] * d + i] : tok_at(Ktok, tok_dtype, e_id[e] * d + i);
+                kv[i] = entry_at(Knode, Ktok, Kloc, tok_dtype, e_lev[e], e_id[e], d, i);
             rope(kv, e_rank[e], d, rope_base, r1);
             for (int g = 0; g < G; g++) {
                 for (int i = 0; i < d; i++) qd[i] = (double)q[g * d + i];
@@ -486,7 +507,7 @@ int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, co
             for (long long e = 0; e < n_ent; e++) {
                 double p = exp(lg[e * G + g] - mx) / den, a = 0.0;
                 for (int i = 0; i < d; i++) {
-                    vv[i] = e_lev[e] ? Vnode[e_lev[e]][e_id[e] * d + i] : tok_at(Vtok, tok_dtype, e_id[e] * d + i);
+                    vv[i] = entry_at(Vnode, Vtok, Vloc, tok_dtype, e_lev[e], e_id[e], d, i);
                     a += dout[g * d + i] * vv[i];
                 }
                 Dg += p * a;
@@ -495,18 +516,20 @@ int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, co
             for (long long e = 0; e < n_ent; e++) {
                 double p = exp(lg[e * G + g] - mx) / den, a = 0.0;
                 for (int i = 0; i < d; i++) {
-                    vv[i] = e_lev[e] ? Vnode[e_lev[e]][e_id[e] * d + i] : tok_at(Vtok, tok_dtype, e_id[e] * d + i);
+                    vv[i] = entry_at(Vnode, Vtok, Vloc, tok_dtype, e_lev[e], e_id[e], d, i);
                     a += dout[g * d + i] * vv[i];
                 }
                 double dl = p * (a - Dg);
                 /* dq: the key rotated by i - P; dk: the query rotated by P - i */
                 for (int i = 0; i < d; i++)
-                    kv[i] = e_lev[e] ? Knode[e_lev[e]][e_id[e] * d + i] : tok_at(Ktok, tok_dtype, e_id[e] * d + i);
+                    kv[i] = entry_at(Knode, Ktok, Kloc, tok_dtype, e_lev[e], e_id[e], d, i);
                 rope(kv, e_rank[e] - e_pos[e], d, rope_base, r1);
                 for (int i = 0; i < d; i++) qd[i] = (double)q[g * d + i];
                 rope(qd, e_pos[e] - e_rank[e], d, rope_base, r2);
-                double* dk = e_lev[e] ? dKn[e_lev[e]] + e_id[e] * d : dKtok + e_id[e] * d;
-                double* dv = e_lev[e] ? dVn[e_lev[e]] + e_id[e] * d : dVtok + e_id[e] * d;
+                double* dk = e_lev[e] > 0 ? dKn[e_lev[e]] + e_id[e] * d
+                                          : (e_lev[e] == 0 ? dKtok : dKloc) + e_id[e] * d;
+                double* dv = e_lev[e] > 0 ? dVn[e_lev[e]] + e_id[e] * d
+                                          : (e_lev[e] == 0 ? dVtok : dVloc) + e_id[e] * d;
                 for (int i = 0; i < d; i++) {
                     dq[g * d + i] += dl * scale * r1[i];
                     dk[i] += dl * scale * r2[i];
@@ -569,6 +592,23 @@ int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, co
     free(dKn); free(dVn); free(sel); free(out); free(cand); free(next); free(e_lev); free(e_id); free(e_rank);
     free(e_pos); free(lg); free(kv); free(vv); free(qd); free(r1); free(r2);
     return ok ? J : -1;
+}
+
+int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, const double* const* Knode,
+                   const double* const* Vnode, const void* Ktok, const void* Vtok, int tok_dtype, const float* W,
+                   const float* q, const double* dout, double* dq, double* dKtok, double* dVtok, double* dW) {
+    if (T < 1) return -1;
+    return query_grad_impl(d, b, k, G, rope_base, T, Knode, Vnode, Ktok, Vtok, tok_dtype, NULL, NULL, 0, W, q, dout,
+                           dq, dKtok, dVtok, NULL, NULL, dW);
+}
+
+int orc_query_grad_local(int d, int b, int k, int G, double rope_base, long long T, const double* const* Knode,
+                         const double* const* Vnode, const void* Ktok, const void* Vtok, int tok_dtype,
+                         const void* Kloc, const void* Vloc, long long nloc, const float* W, const float* q,
+                         const double* dout, double* dq, double* dKtok, double* dVtok, double* dKloc, double* dVloc,
+                         double* dW) {
+    return query_grad_impl(d, b, k, G, rope_base, T, Knode, Vnode, Ktok, Vtok, tok_dtype, Kloc, Vloc, nloc, W, q,
+                           dout, dq, dKtok, dVtok, dKloc, dVloc, dW);
 }
 
 /* ---------------------------------------------- clustered order (R20) */

@@ -74,6 +74,15 @@ int orc_query_grad(int d, int b, int k, int G, double rope_base, long long T, co
                    const double* const* Vnode, const void* Ktok, const void* Vtok, int tok_dtype, const float* W,
                    const float* q, const double* dout, double* dq, double* dKtok, double* dVtok, double* dW);
 
+/* The same for a prefill query: the tree over tokens [0, T) (T may be 0)
+ * plus the chunk's own causal tokens Kloc, Vloc [nloc][d] (as in orc_query);
+ * their gradients are added into dKloc, dVloc [nloc][d]. Returns J, or -1. */
+int orc_query_grad_local(int d, int b, int k, int G, double rope_base, long long T, const double* const* Knode,
+                         const double* const* Vnode, const void* Ktok, const void* Vtok, int tok_dtype,
+                         const void* Kloc, const void* Vloc, long long nloc, const float* W, const float* q,
+                         const double* dout, double* dq, double* dKtok, double* dVtok, double* dKloc, double* dVloc,
+                         double* dW);
+
 /* LSA-style clustered order of T tokens ("Latent Sparse Attention"
  * abstract: keys clustered hierarchically in a learned latent space, queries
  * scoring the hierarchy of clusters). Reading R20 (see the .c file): level j

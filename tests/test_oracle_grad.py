@@ -160,3 +160,85 @@ def test_gradient_linear_in_dout():
     g2 = _grad(K, V, W, q, 2 * dout, T, d, b, k, G, base)
     for key in ("dK", "dV", "dW", "dq"):
         np.testing.assert_allclose(g2[key], 2 * g1[key], rtol=1e-13, atol=1e-15)
+
+
+# ------------------------------------------------------- prefill queries
+# A prefill query of a chunk sees the tree over the tokens before the chunk
+# plus the chunk's own causal tokens, which follow the level-0 candidates in
+# the index order (reading R9); the gradient reaches those local tokens too.
+
+
+def _forward_local(K, V, W, q, Kl, Vl, T, d, b, k, G, base):
+    if T > 0:
+        tree = oracle.build_tree(K, V, T, d, b, W, F64)
+        r = oracle.query(tree.K, tree.V, K, V, T, q, d, b, k, G, base, Kloc=Kl, Vloc=Vl)
+    else:
+        r = oracle.query([None], [None], K, V, 0, q, d, b, k, G, base, Kloc=Kl, Vloc=Vl)
+    return r["out"], r["sel"], r
+
+
+def _grad_local(K, V, W, q, Kl, Vl, dout, T, d, b, k, G, base):
+    if T > 0:
+        tree = oracle.build_tree(K, V, T, d, b, W, F64)
+        tK, tV = tree.K, tree.V
+    else:
+        tK = tV = [None]
+    return oracle.query_grad(tK, tV, K, V, T, q, dout, W, d, b, k, G, base, Kloc=Kl, Vloc=Vl)
+
+
+LOCAL_CASES = [  # T, nloc, b, k, G, d
+    (37, 5, 4, 1, 1, 8),
+    (300, 9, 4, 2, 3, 8),
+    (130, 4, 5, 2, 2, 16),
+    (0, 7, 4, 2, 2, 8),   # the first chunk: no tree, the chunk's causal tokens only
+]
+
+
+@pytest.mark.parametrize("T,nloc,b,k,G,d", LOCAL_CASES)
+@pytest.mark.parametrize("which", ["K", "V", "W", "q", "Kl", "Vl"])
+def test_prefill_directional_finite_difference(T, nloc, b, k, G, d, which):
+    if T == 0 and which in ("K", "V", "W"):
+        pytest.skip("no tree: nothing depends on these")
+    base = 100.0
+    K, V = _rand(21, (max(T, 1), d)), _rand(22, (max(T, 1), d))
+    Kl, Vl, q = _rand(23, (nloc, d)), _rand(24, (nloc, d)), _rand(25, (G, d))
+    W = _rand(26, (d, d), 1.3 / math.sqrt(d))
+    dout = _rand(27, (G, d)).astype(np.float64)
+    args = dict(K=K, V=V, W=W, q=q, Kl=Kl, Vl=Vl)
+    out, sel, r = _forward_local(**args, T=T, d=d, b=b, k=k, G=G, base=base)
+    assert np.all(r["margin"] > 1e-3), "pick inputs without a near tie"
+    g = _grad_local(**args, dout=dout, T=T, d=d, b=b, k=k, G=G, base=base)
+    grads = dict(K=g["dK"], V=g["dV"], W=g["dW"], q=g["dq"], Kl=g["dKloc"], Vl=g["dVloc"])
+    rng = np.random.default_rng(hash((T, nloc, b, k, G, d, which)) % 2**32)
+    u = rng.standard_normal(args[which].shape)
+    if which in ("K", "V"):
+        u[T:] = 0.0
+    xp, xm, delta = _step(args[which], u, 1e-3)
+    fp = _forward_local(**{**args, which: xp}, T=T, d=d, b=b, k=k, G=G, base=base)
+    fm = _forward_local(**{**args, which: xm}, T=T, d=d, b=b, k=k, G=G, base=base)
+    assert np.array_equal(fp[1], sel) and np.array_equal(fm[1], sel), "the step changed a selection"
+    fd = float(np.sum(dout * (fp[0] - fm[0])))
+    an = float(np.sum(grads[which] * delta[:grads[which].shape[0]]))
+    assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (which, fd, an)
+
+
+@pytest.mark.parametrize("T,nloc,b", [(0, 1, 2), (0, 12, 4), (50, 7, 4), (200, 33, 16)])
+def test_prefill_dense_equivalence(T, nloc, b):
+    """Nothing dropped (k at least every level's size): the prefill query is
+    dense causal RoPE attention over the tokens before the chunk followed by
+    the chunk's own tokens, so its gradients are torch autograd's of that, and
+    the pooler gets none."""
+    d, G, base = 16, 2, 1e4
+    K, V = _rand(31, (max(T, 1), d)), _rand(32, (max(T, 1), d))
+    Kl, Vl, q = _rand(33, (nloc, d)), _rand(34, (nloc, d)), _rand(35, (G, d))
+    W = _rand(36, (d, d), 1 / math.sqrt(d))
+    dout = _rand(37, (G, d)).astype(np.float64)
+    kmax = max(oracle.levels(T, b)[1][1:]) if T > 0 else 1
+    g = _grad_local(K, V, W, q, Kl, Vl, dout, T, d, b, kmax, G, base)
+    dK, dV, dq = _dense_torch_grads(np.concatenate([K[:T], Kl]), np.concatenate([V[:T], Vl]), q, dout, base)
+    np.testing.assert_allclose(g["dK"], dK[:T], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(g["dV"], dV[:T], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(g["dKloc"], dK[T:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(g["dVloc"], dV[T:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(g["dq"], dq, rtol=0, atol=1e-12)
+    assert not g["dW"].any()
