@@ -479,7 +479,31 @@ def measure_backward(layer, w, q, dev, flush, peaks, kv_host, cpu_threads, with_
     return res
 
 
-def measure_distill(layer, w, q, dev, flush, build_ms, kv_host, cpu_threads, with_cpu):
+def distill_token_pass_bytes(H, lengths, D, b, J_cap, es):
+    """Bytes of the distillation step's passes over every token, which
+    dominate it: the pooler-only propagation (every token's key read; per
+    level the node accumulators read and cleared, the inner levels' h and s
+    written and their children's keys read) and the rebuild of every level
+    (the tokens' keys and values read, the level-1 keys, values and fp32 value
+    sums written; each upper level reading its children's keys and value sums
+    and writing its own). The decode, loss, entry gradients and update (about
+    0.1 GB at 524K x 4) are not counted."""
+    total = 0
+    for L in lengths:
+        total += H * L * D * es
+        for j in range(1, J_cap + 1):
+            nj = -(-L // b ** j)
+            total += H * nj * 2 * D * 4 * 2
+            if j >= 2:
+                total += H * (nj * 2 * D * 4 + (-(-L // b ** (j - 1))) * D * es)
+        total += H * (2 * L * D * es + (-(-L // b)) * D * (2 * es + 4))
+        for j in range(2, J_cap + 1):
+            nj, nprev = -(-L // b ** j), -(-L // b ** (j - 1))
+            total += H * (nprev * D * (es + 4) + nj * D * (2 * es + 4))
+    return total
+
+
+def measure_distill(layer, w, q, dev, flush, build_ms, peaks, kv_host, cpu_threads, with_cpu):
     """One distillation step of the pooler (recsa_distill_step: forward,
     squared error, the pooler's gradient, update, tree rebuild) on the
     layer's current cache, median of 5 after 2 warm-ups, L2 flushed before
@@ -503,7 +527,13 @@ def measure_distill(layer, w, q, dev, flush, build_ms, kv_host, cpu_threads, wit
         ts.append(a.elapsed_time(b_))
     layer.check()
     ms = statistics.median(ts)
+    pass_bytes = distill_token_pass_bytes(H, layer.lengths(), D, w.branching, layer.tree_shape()[0], 2)
+    hbm = float(peaks["hbm_gbs"])
     res = {"step_ms": ms, "tree_rebuild_ms_alone": build_ms, "queries": B * Hq, "loss": float(loss.item()),
+           "roofline": {"kernel": "recsa_distill_step (its passes over every token)", "bound": "hbm",
+                        "achieved": pass_bytes / (ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
+                        "frac": pass_bytes / (ms / 1e3) / 1e9 / hbm, "algorithmic_bytes": pass_bytes,
+                        "traffic": None},
            "how": "recsa_distill_step on the decode workload's cache, one query per sequence, synthetic targets, "
                   "lr 0; median of 5, L2 flushed"}
     del layer._distill_scratch
@@ -930,7 +960,7 @@ def main():
 
     distill = None
     if not args.no_distill:
-        distill = measure_distill(layer, w, q_d[0], dev, flush, build_ms, (Kh.numpy(), Vh.numpy()),
+        distill = measure_distill(layer, w, q_d[0], dev, flush, build_ms, peaks, (Kh.numpy(), Vh.numpy()),
                                   os.cpu_count() or 1, rank == 0 and world == 1 and not args.no_cpu_baseline)
 
     cluster = None
