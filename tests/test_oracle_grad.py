@@ -242,3 +242,53 @@ def test_prefill_dense_equivalence(T, nloc, b):
     np.testing.assert_allclose(g["dVloc"], dV[T:], rtol=0, atol=1e-12)
     np.testing.assert_allclose(g["dq"], dq, rtol=0, atol=1e-12)
     assert not g["dW"].any()
+
+
+def test_prefill_chunk_gradient_is_dense_causal():
+    """A whole chunk: query i of the chunk sees the tree over the T earlier
+    tokens and the chunk's tokens 0..i. With nothing dropped, the gradients
+    summed over the chunk's queries are torch autograd's of dense causal RoPE
+    attention of the chunk's queries over all T + C tokens."""
+    T, C, b, d, G, base = 50, 6, 4, 16, 2, 1e4
+    K, V = _rand(41, (T, d)), _rand(42, (T, d))
+    Kc, Vc = _rand(43, (C, d)), _rand(44, (C, d))
+    Q = _rand(45, (C, G, d))
+    W = _rand(46, (d, d), 1 / math.sqrt(d))
+    dO = _rand(47, (C, G, d)).astype(np.float64)
+    kmax = max(oracle.levels(T, b)[1][1:])
+    dK, dV, dKc, dVc = np.zeros((T, d)), np.zeros((T, d)), np.zeros((C, d)), np.zeros((C, d))
+    dQ = np.zeros((C, G, d))
+    for i in range(C):
+        g = _grad_local(K, V, W, Q[i], Kc[:i + 1], Vc[:i + 1], dO[i], T, d, b, kmax, G, base)
+        dK += g["dK"]
+        dV += g["dV"]
+        dKc[:i + 1] += g["dKloc"]
+        dVc[:i + 1] += g["dVloc"]
+        dQ[i] = g["dq"]
+        assert not g["dW"].any()
+    # dense causal attention of the chunk's queries (positions T .. T + C - 1)
+    h = d // 2
+    theta = base ** (-torch.arange(h, dtype=torch.float64) * 2 / d)
+    X = torch.tensor(np.concatenate([K, Kc]), dtype=torch.float64, requires_grad=True)
+    Y = torch.tensor(np.concatenate([V, Vc]), dtype=torch.float64, requires_grad=True)
+    Qt = torch.tensor(Q, dtype=torch.float64, requires_grad=True)
+
+    def rot(x, pos):
+        z = torch.complex(x[..., :h], x[..., h:]) * torch.polar(torch.ones_like(pos[..., None] * theta),
+                                                                 pos[..., None] * theta)
+        return torch.cat([z.real, z.imag], dim=-1)
+
+    n = T + C
+    kr = rot(X, torch.arange(n, dtype=torch.float64))
+    pos_q = (T + torch.arange(C, dtype=torch.float64))[:, None].expand(C, G)
+    qr = rot(Qt, pos_q)
+    s = torch.einsum("cgd,nd->cgn", qr, kr) / math.sqrt(d)
+    mask = torch.arange(n)[None, :] > (T + torch.arange(C))[:, None]
+    s = s.masked_fill(mask[:, None, :], float("-inf"))
+    out = torch.einsum("cgn,nd->cgd", torch.softmax(s, dim=-1), Y)
+    (out * torch.tensor(dO)).sum().backward()
+    np.testing.assert_allclose(dK, X.grad[:T].numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dV, Y.grad[:T].numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dKc, X.grad[T:].numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dVc, Y.grad[T:].numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dQ, Qt.grad.numpy(), rtol=0, atol=1e-12)
